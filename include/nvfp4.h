@@ -1,0 +1,208 @@
+/*
+ * nvfp4.h -- C ABI of the B200 (sm_100a) NVFP4 library: quantize, dequantize,
+ * block-scaled W4A4 GEMM and the fused linear / MLP step.
+ *
+ * The format (NVFP4 wiki page, newton.com.tw, section "技術原理"): each value
+ * is a 4-bit E2M1 element (1 sign, 2 exponent, 1 mantissa bit; magnitudes
+ * 0, 0.5, 1, 1.5, 2, 3, 4, 6); every 16 consecutive values along a row share
+ * one E4M3 FP8 block scale; one FP32 scale covers the whole tensor.  That is
+ * about 4.5 bits per value.
+ *
+ * The GEMM consumes NVFP4 weights AND NVFP4 activations directly on the
+ * block-scaled FP4 tensor cores, with no dequantize-to-16-bit step (aixq.cc
+ * article on Unsloth Dynamic NVFP4, section "核心差异：W4A4 vs W4A16").
+ *
+ * Arithmetic (the pages give the structure; these are the rules):
+ *   tensor scale   g = fl32(amax / 2688)                 (2688 = 6 * 448)
+ *   block scale    s = E4M3_rne_satfinite(fl32(bamax / fl32(6 * g)))  (g==0: s=0)
+ *   element        d = fl32(dec(s) * g); r = fl32(1/d); v = fl32(x * r);
+ *                  code = E2M1_rne_satfinite(v) (ties to the even magnitude
+ *                  index; sign kept for values that round to zero);
+ *                  a block with d == 0 or 1/d == inf has all codes 0.
+ *   dequantize     y = fl32(fl32(e * dec(s)) * g)
+ *   GEMM           y[m][n] = fl32(acc[m][n] * fl32(gA * gB)),
+ *                  acc = sum_k (eA*sA)(eB*sB) accumulated in fp32 by the tensor
+ *                  cores; bf16 output is the RNE rounding of that fp32 value.
+ *
+ * Conventions for every entry point:
+ *   - All pointers are DEVICE pointers owned by the caller, 16-byte aligned.
+ *     Row pitches (ld, in elements) must keep every row 16-byte aligned.
+ *   - Calls are asynchronous and stream-ordered on `stream`; none allocates
+ *     memory and none synchronises, except nvfp4_get_device_status.
+ *   - Argument errors are returned synchronously and launch nothing.
+ *     NVFP4_ERR_CUDA wraps a failed launch (the CUDA error is left for
+ *     cudaGetLastError).  Device-side give-ups (a bounded wait that ran out)
+ *     are OR-ed into the status word at the start of the workspace and read by
+ *     nvfp4_get_device_status.
+ *   - Requires a compute-capability 10.0 GPU (B200); NVFP4_ERR_ARCH otherwise.
+ *     There is no CPU fallback.
+ *   - Workspace: `ws` points to at least nvfp4_workspace_bytes(...) bytes of
+ *     device memory.  Zero-fill it once after allocating; the library keeps a
+ *     sticky status word in its first 16 bytes and uses the rest as scratch.
+ *     Calls that share one workspace must not overlap on the GPU.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                      /* same type as cudaStream_t */
+typedef struct CUstream_st *nvfp4_stream_t;
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,           /* NULL pointer, negative size, mismatched shapes */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 2,     /* cols % 16 (quantize) or K % 64 (GEMM) not 0 */
+    NVFP4_ERR_MISALIGNED = 3,            /* a pointer or row pitch not 16-byte aligned */
+    NVFP4_ERR_WORKSPACE = 4,             /* ws NULL or smaller than required */
+    NVFP4_ERR_CUDA = 5,                  /* a CUDA runtime/driver call or launch failed */
+    NVFP4_ERR_TIMEOUT = 6,               /* a device-side bounded wait gave up */
+    NVFP4_ERR_ARCH = 7                   /* current device is not sm_100 */
+} nvfp4_status;
+
+typedef enum {
+    NVFP4_F32 = 0,
+    NVFP4_BF16 = 1
+} nvfp4_dtype;
+
+typedef enum {
+    NVFP4_OP_QUANTIZE = 0,
+    NVFP4_OP_DEQUANTIZE = 1,
+    NVFP4_OP_GEMM = 2,
+    NVFP4_OP_LINEAR_FUSED = 3
+} nvfp4_op;
+
+typedef enum {
+    NVFP4_EPI_STORE = 0,                 /* y = x_q . w_q^T * gx * gw */
+    NVFP4_EPI_SILU_MUL_REQUANT = 1       /* h = SiLU(x.w^T) * (x.w_up^T), quantized to NVFP4 */
+} nvfp4_epilogue;
+
+/*
+ * One NVFP4 tensor [rows][cols], quantized along cols (the GEMM's K).
+ *   codes        [rows][cols/2] bytes; byte j of a row holds element 2j in its
+ *                low nibble and element 2j+1 in its high nibble; sign in bit 3.
+ *   scales       E4M3 block scales in the tiled layout the tensor cores read:
+ *                rows padded to R128 = roundup(rows,128), blocks per row padded
+ *                to KB4 = roundup(cols/16, 4).  The scale of block kb of row r
+ *                is the byte at
+ *                  ((r/128)*(KB4/4) + kb/4)*512 + (r%32)*16 + ((r/32)%4)*4 + kb%4
+ *                so each 128-row x 64-column slab is one contiguous 512-byte
+ *                atom.  Padding bytes are written as 0 by nvfp4_quantize.
+ *                Size: nvfp4_scales_bytes(rows, cols).
+ *   tensor_scale one fp32 in device memory: g = amax / 2688.
+ */
+typedef struct {
+    uint8_t *codes;
+    uint8_t *scales;
+    float *tensor_scale;
+    int64_t rows;
+    int64_t cols;
+} nvfp4_tensor;
+
+/* Bytes of the packed codes: rows * cols / 2. */
+NVFP4_API size_t nvfp4_codes_bytes(int64_t rows, int64_t cols);
+
+/* Bytes of the tiled scale array: roundup(rows,128) * roundup(cols/16,4). */
+NVFP4_API size_t nvfp4_scales_bytes(int64_t rows, int64_t cols);
+
+/* Workspace bytes an operation needs for the given shape (M rows of
+ * activations, N rows of weights, K reduction length; quantize/dequantize use
+ * M = rows, K = cols).  Always at least 256 (the status word). */
+NVFP4_API size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K);
+
+/*
+ * Quantize x [rows][cols] (row pitch ld elements, dtype xt) to NVFP4 into
+ * `out` (out->rows == rows, out->cols == cols, cols % 16 == 0).
+ * Two passes: a reduction of the tensor amax into per-CTA partial maxima in
+ * ws, then a pass that derives g on the device (no host synchronisation),
+ * writes *out->tensor_scale, and encodes each 16-element block.
+ * NVFP4 wiki page, section "技術原理" (two-level microblock scaling).
+ */
+NVFP4_API nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype xt, int64_t rows, int64_t cols,
+                            int64_t ld, const nvfp4_tensor *out, void *ws, size_t ws_bytes,
+                            nvfp4_stream_t stream);
+
+/*
+ * Dequantize q into y [q->rows][q->cols] (row pitch ldy elements, dtype yt):
+ * y = fl32(fl32(e * dec(s)) * g), rounded to bf16 by RNE when yt is BF16.
+ * This is the decode step a W4A16 path would run before a 16-bit GEMM
+ * (aixq.cc article, section "核心差异：W4A4 vs W4A16"); here it is an
+ * inspection / interoperability path, not part of the GEMM.
+ */
+NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor *q, void *y, nvfp4_dtype yt, int64_t ldy,
+                              nvfp4_stream_t stream);
+
+/*
+ * y[M][N] = (A . B^T) * gA * gB with A = a [M][K], B = b [N][K] (K = a->cols
+ * = b->cols, K % 64 == 0), both NVFP4, consumed directly by tcgen05
+ * block-scaled FP4 MMAs with fp32 accumulation in tensor memory.  y has row
+ * pitch ldy (elements) and dtype yt (BF16 or F32).  W4A4 linear layer: a is
+ * the activations, b the weights.
+ */
+NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y, nvfp4_dtype yt,
+                        int64_t ldy, void *ws, size_t ws_bytes, nvfp4_stream_t stream);
+
+/*
+ * The W4A4 linear layer from high-precision activations.
+ *   x [M][K] (pitch ldx, dtype xt) is quantized to NVFP4 on the device
+ *   ("dynamic" per-call scaling of the activations), then multiplied with the
+ *   pre-quantized weights.
+ *   epilogue == NVFP4_EPI_STORE: y [M][w->rows] = x_q . w^T * gx * gw
+ *     (w_up, y_q ignored; y required, dtype yt, pitch ldy).
+ *   epilogue == NVFP4_EPI_SILU_MUL_REQUANT: gate = x_q . w^T, up = x_q . w_up^T
+ *     (w_up->rows == w->rows), h = SiLU(gate) * up in fp32, SiLU(z) =
+ *     z / (1 + exp(-z)); h is quantized to NVFP4 into y_q (y_q->rows == M,
+ *     y_q->cols == w->rows) with its own tensor scale over all of h, ready to be
+ *     the activation operand of the next (down-projection) nvfp4_gemm.  If y is
+ *     not NULL it receives h itself in fp32 (yt must be F32), for inspection.
+ *   If x_q is not NULL it receives the quantized activations (x_q->rows == M,
+ *   x_q->cols == K); otherwise they live in ws.
+ */
+NVFP4_API nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                const nvfp4_tensor *w, const nvfp4_tensor *w_up,
+                                nvfp4_epilogue epilogue, void *y, nvfp4_dtype yt, int64_t ldy,
+                                const nvfp4_tensor *y_q, const nvfp4_tensor *x_q,
+                                void *ws, size_t ws_bytes, nvfp4_stream_t stream);
+
+/*
+ * Synchronise `stream`, read the sticky device status word in ws, clear it,
+ * and return it (NVFP4_OK when no device-side wait gave up since the last
+ * read).  Also returns NVFP4_ERR_CUDA if the stream reports an error.
+ */
+NVFP4_API nvfp4_status nvfp4_get_device_status(void *ws, nvfp4_stream_t stream);
+
+/*
+ * Launch one single-thread kernel that waits, with the library's bounded wait,
+ * on a shared-memory barrier that nothing ever completes, giving up after
+ * timeout_us microseconds.  The give-up path records NVFP4_ERR_TIMEOUT in the
+ * status word of ws, exactly as a stalled pipeline stage of the GEMM would.
+ * Used to test the failure-detection path without hanging a GPU.
+ */
+NVFP4_API nvfp4_status nvfp4_selftest_bounded_wait(void *ws, uint32_t timeout_us, nvfp4_stream_t stream);
+
+/* Bound, in microseconds, of every device-side wait of later launches
+ * (default 2,000,000).  Returns the previous value. */
+NVFP4_API uint32_t nvfp4_set_wait_timeout_us(uint32_t timeout_us);
+
+/* Human-readable name of a status code. */
+NVFP4_API const char *nvfp4_status_string(nvfp4_status status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+NVFP4_API int nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

@@ -1,0 +1,240 @@
+"""Python binding of the B200 NVFP4 library (``libnvfp4.so``, C ABI in
+``include/nvfp4.h``).
+
+Argument marshalling only: every step of quantization, dequantization and the
+W4A4 block-scaled GEMM runs in the library's CUDA kernels.  PyTorch supplies
+device memory and the current stream.  There is no CPU fallback: importing
+this package fails loudly when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m nvfp4_block_scaled_21_b200.build` "
+        "(nvcc, sm_100a). The package has no CPU fallback.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# status codes (include/nvfp4.h)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_WORKSPACE, ERR_CUDA, \
+    ERR_TIMEOUT, ERR_ARCH = range(8)
+F32, BF16 = 0, 1
+OP_QUANTIZE, OP_DEQUANTIZE, OP_GEMM, OP_LINEAR_FUSED = range(4)
+EPI_STORE, EPI_SILU_MUL_REQUANT = 0, 1
+
+EXPORTED = (
+    "nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize",
+    "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_linear_fused", "nvfp4_get_device_status",
+    "nvfp4_selftest_bounded_wait", "nvfp4_set_wait_timeout_us", "nvfp4_status_string",
+    "nvfp4_version",
+)
+
+
+class CTensor(ctypes.Structure):
+    """``nvfp4_tensor`` of the C ABI."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("tensor_scale", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64)]
+
+
+_P, _I64, _SZ, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+_T = ctypes.POINTER(CTensor)
+
+_lib.nvfp4_codes_bytes.argtypes = [_I64, _I64]
+_lib.nvfp4_codes_bytes.restype = _SZ
+_lib.nvfp4_scales_bytes.argtypes = [_I64, _I64]
+_lib.nvfp4_scales_bytes.restype = _SZ
+_lib.nvfp4_workspace_bytes.argtypes = [_I, _I64, _I64, _I64]
+_lib.nvfp4_workspace_bytes.restype = _SZ
+_lib.nvfp4_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _T, _P, _SZ, _P]
+_lib.nvfp4_quantize.restype = _I
+_lib.nvfp4_dequantize.argtypes = [_T, _P, _I, _I64, _P]
+_lib.nvfp4_dequantize.restype = _I
+_lib.nvfp4_gemm.argtypes = [_T, _T, _P, _I, _I64, _P, _SZ, _P]
+_lib.nvfp4_gemm.restype = _I
+_lib.nvfp4_linear_fused.argtypes = [_P, _I, _I64, _I64, _I64, _T, _T, _I, _P, _I, _I64, _T, _T,
+                                    _P, _SZ, _P]
+_lib.nvfp4_linear_fused.restype = _I
+_lib.nvfp4_get_device_status.argtypes = [_P, _P]
+_lib.nvfp4_get_device_status.restype = _I
+_lib.nvfp4_selftest_bounded_wait.argtypes = [_P, ctypes.c_uint32, _P]
+_lib.nvfp4_selftest_bounded_wait.restype = _I
+_lib.nvfp4_set_wait_timeout_us.argtypes = [ctypes.c_uint32]
+_lib.nvfp4_set_wait_timeout_us.restype = ctypes.c_uint32
+_lib.nvfp4_status_string.argtypes = [_I]
+_lib.nvfp4_status_string.restype = ctypes.c_char_p
+_lib.nvfp4_version.argtypes = []
+_lib.nvfp4_version.restype = _I
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def status_string(status: int) -> str:
+    return _lib.nvfp4_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise NVFP4Error(status, where)
+
+
+def version() -> int:
+    return _lib.nvfp4_version()
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded ``libnvfp4.so`` (raw C ABI)."""
+    return _lib
+
+
+# ---------------------------------------------------------------------------
+# torch marshalling
+# ---------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return _torch().cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+@dataclass
+class NVFP4Tensor:
+    """Device buffers of one NVFP4 tensor [rows][cols] (see ``nvfp4_tensor``)."""
+    codes: "object"          # uint8 [rows, cols/2]
+    scales: "object"         # uint8 [nvfp4_scales_bytes]
+    tensor_scale: "object"   # float32 [4] (element 0 is g; 16-byte slot)
+    rows: int
+    cols: int
+
+    @staticmethod
+    def empty(rows: int, cols: int, device="cuda") -> "NVFP4Tensor":
+        torch = _torch()
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+        scales = torch.empty(int(_lib.nvfp4_scales_bytes(rows, cols)), dtype=torch.uint8,
+                             device=device)
+        g = torch.zeros(4, dtype=torch.float32, device=device)
+        return NVFP4Tensor(codes, scales, g, rows, cols)
+
+    def c(self) -> CTensor:
+        return CTensor(self.codes.data_ptr(), self.scales.data_ptr(),
+                       self.tensor_scale.data_ptr(), self.rows, self.cols)
+
+
+def codes_bytes(rows: int, cols: int) -> int:
+    return int(_lib.nvfp4_codes_bytes(rows, cols))
+
+
+def scales_bytes(rows: int, cols: int) -> int:
+    return int(_lib.nvfp4_scales_bytes(rows, cols))
+
+
+def workspace_bytes(op: int, M: int, N: int, K: int) -> int:
+    return int(_lib.nvfp4_workspace_bytes(op, M, N, K))
+
+
+def workspace(op: int, M: int, N: int, K: int, device="cuda"):
+    """A zero-filled workspace for ``op`` at this shape."""
+    torch = _torch()
+    return torch.zeros(workspace_bytes(op, M, N, K), dtype=torch.uint8, device=device)
+
+
+def nvfp4_quantize(x, out: NVFP4Tensor, ws, stream=None) -> NVFP4Tensor:
+    """Quantize a 2-D bf16/fp32 CUDA tensor (row pitch x.stride(0)) into out."""
+    assert x.dim() == 2 and x.stride(1) == 1
+    ct = out.c()
+    st = _lib.nvfp4_quantize(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], x.stride(0),
+                             ctypes.byref(ct), ws.data_ptr(), ws.numel(), _stream(stream))
+    _check(st, "nvfp4_quantize")
+    return out
+
+
+def nvfp4_dequantize(q: NVFP4Tensor, y, stream=None):
+    assert y.dim() == 2 and y.stride(1) == 1
+    ct = q.c()
+    st = _lib.nvfp4_dequantize(ctypes.byref(ct), y.data_ptr(), _dtype_code(y), y.stride(0),
+                               _stream(stream))
+    _check(st, "nvfp4_dequantize")
+    return y
+
+
+def nvfp4_gemm(a: NVFP4Tensor, b: NVFP4Tensor, y, ws, stream=None):
+    """y[M][N] = (a . b^T) * ga * gb."""
+    assert y.dim() == 2 and y.stride(1) == 1
+    ca, cb = a.c(), b.c()
+    st = _lib.nvfp4_gemm(ctypes.byref(ca), ctypes.byref(cb), y.data_ptr(), _dtype_code(y),
+                         y.stride(0), ws.data_ptr(), ws.numel(), _stream(stream))
+    _check(st, "nvfp4_gemm")
+    return y
+
+
+def nvfp4_linear_fused(x, w: NVFP4Tensor, ws, epilogue: int = EPI_STORE, y=None,
+                       w_up: NVFP4Tensor | None = None, y_q: NVFP4Tensor | None = None,
+                       x_q: NVFP4Tensor | None = None, stream=None):
+    """Quantize x on the device and run the W4A4 linear layer (see nvfp4.h)."""
+    assert x.dim() == 2 and x.stride(1) == 1
+    cw = w.c()
+    cwu = w_up.c() if w_up is not None else None
+    cyq = y_q.c() if y_q is not None else None
+    cxq = x_q.c() if x_q is not None else None
+    yt = _dtype_code(y) if y is not None else F32
+    ldy = y.stride(0) if y is not None else 0
+    st = _lib.nvfp4_linear_fused(
+        x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], x.stride(0), ctypes.byref(cw),
+        ctypes.byref(cwu) if cwu is not None else None, epilogue, _ptr(y), yt, ldy,
+        ctypes.byref(cyq) if cyq is not None else None,
+        ctypes.byref(cxq) if cxq is not None else None, ws.data_ptr(), ws.numel(),
+        _stream(stream))
+    _check(st, "nvfp4_linear_fused")
+    return y
+
+
+def nvfp4_get_device_status(ws, stream=None) -> int:
+    return int(_lib.nvfp4_get_device_status(ws.data_ptr(), _stream(stream)))
+
+
+def nvfp4_selftest_bounded_wait(ws, timeout_us: int, stream=None) -> None:
+    _check(_lib.nvfp4_selftest_bounded_wait(ws.data_ptr(), int(timeout_us), _stream(stream)),
+           "nvfp4_selftest_bounded_wait")
+
+
+def nvfp4_set_wait_timeout_us(timeout_us: int) -> int:
+    return int(_lib.nvfp4_set_wait_timeout_us(int(timeout_us)))
+
+
+# convenience -----------------------------------------------------------------
+
+def quantize(x, ws=None, stream=None) -> NVFP4Tensor:
+    """Allocate an NVFP4Tensor and quantize x into it."""
+    out = NVFP4Tensor.empty(x.shape[0], x.shape[1], device=x.device)
+    if ws is None:
+        ws = workspace(OP_QUANTIZE, x.shape[0], 0, x.shape[1], device=x.device)
+    return nvfp4_quantize(x, out, ws, stream)

@@ -1,0 +1,312 @@
+// api.cu -- the extern "C" boundary declared in include/nvfp4.h: argument
+// validation (synchronous, no launch on error), workspace carving and the
+// kernel launches.  No allocation, no synchronisation except in
+// nvfp4_get_device_status.
+#include <atomic>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "nvfp4.h"
+
+using namespace nvfp4;
+
+namespace {
+
+std::atomic<uint32_t> g_wait_timeout_us{2000000u};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Device properties of the current device, cached per device ordinal.
+struct DevInfo {
+    int sms = 0;
+    int major = 0;
+    int minor = 0;
+};
+
+nvfp4_status current_device(DevInfo *out) {
+    static DevInfo cache[64];
+    static std::atomic<bool> have[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return NVFP4_ERR_CUDA;
+    if (dev < 64 && have[dev].load(std::memory_order_acquire)) {
+        *out = cache[dev];
+    } else {
+        DevInfo d;
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        if (dev < 64) {
+            cache[dev] = d;
+            have[dev].store(true, std::memory_order_release);
+        }
+        *out = d;
+    }
+    if (out->major != 10 || out->minor != 0) return NVFP4_ERR_ARCH;
+    return NVFP4_OK;
+}
+
+nvfp4_status check_tensor(const nvfp4_tensor *t, int64_t rows, int64_t cols) {
+    if (!t || !t->codes || !t->scales || !t->tensor_scale) return NVFP4_ERR_INVALID_ARG;
+    if (t->rows != rows || t->cols != cols || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+    if (cols % kBlock) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(t->codes) || !aligned16(t->scales) || !aligned16(t->tensor_scale))
+        return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+nvfp4_status check_ws(void *ws, size_t ws_bytes, size_t need) {
+    if (!ws || ws_bytes < need) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+uint8_t *ws_at(void *ws, size_t off) { return static_cast<uint8_t *>(ws) + off; }
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Workspace carving (offsets in bytes).
+constexpr size_t kPartialsOff = kWsStatusBytes;
+constexpr size_t kPartialsBytes = kMaxAmaxPartials * sizeof(float);
+constexpr size_t kQuantizeWs = kPartialsOff + kPartialsBytes;
+
+size_t quantized_bytes(int64_t rows, int64_t cols) {
+    return align256(static_cast<size_t>(rows * cols / 2)) +
+           align256(static_cast<size_t>(round_up(rows, 128) * kb4_of(cols))) + 256;
+}
+
+uint64_t timeout_ns() { return static_cast<uint64_t>(g_wait_timeout_us.load()) * 1000ull; }
+
+nvfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t nvfp4_codes_bytes(int64_t rows, int64_t cols) {
+    if (rows < 0 || cols < 0) return 0;
+    return static_cast<size_t>(rows * cols / 2);
+}
+
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols) {
+    if (rows < 0 || cols < 0) return 0;
+    return static_cast<size_t>(round_up(rows, 128) * kb4_of(cols));
+}
+
+size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K) {
+    if (M < 0 || N < 0 || K < 0) return 0;
+    switch (op) {
+    case NVFP4_OP_QUANTIZE:
+        return kQuantizeWs;
+    case NVFP4_OP_DEQUANTIZE:
+    case NVFP4_OP_GEMM:
+        return kWsStatusBytes;
+    case NVFP4_OP_LINEAR_FUSED: {
+        // partials | x_q (codes, scales, g) | gate, up, h (fp32 [M][N] each)
+        size_t b = kQuantizeWs + quantized_bytes(M, K);
+        b += 3 * align256(static_cast<size_t>(M * N) * sizeof(float));
+        return b;
+    }
+    }
+    return 0;
+}
+
+nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                            const nvfp4_tensor *out, void *ws, size_t ws_bytes,
+                            nvfp4_stream_t stream) {
+    if (!x || (xt != NVFP4_F32 && xt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_tensor(out, rows, cols);
+    if (st != NVFP4_OK) return st;
+    const int eb = xt == NVFP4_BF16 ? 2 : 4;
+    if (!aligned16(x) || (ld * eb) % 16) return NVFP4_ERR_MISALIGNED;
+    if ((st = check_ws(ws, ws_bytes, kQuantizeWs)) != NVFP4_OK) return st;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    return from_cuda(launch_quantize(x, xt == NVFP4_BF16, rows, cols, ld, out->codes, out->scales,
+                                     out->tensor_scale,
+                                     reinterpret_cast<float *>(ws_at(ws, kPartialsOff)), dev.sms,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_dequantize(const nvfp4_tensor *q, void *y, nvfp4_dtype yt, int64_t ldy,
+                              nvfp4_stream_t stream) {
+    if (!q || !y || (yt != NVFP4_F32 && yt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_tensor(q, q->rows, q->cols);
+    if (st != NVFP4_OK) return st;
+    const int eb = yt == NVFP4_BF16 ? 2 : 4;
+    if (ldy < q->cols) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(y) || (ldy * eb) % 16) return NVFP4_ERR_MISALIGNED;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    if (q->rows == 0 || q->cols == 0) return NVFP4_OK;
+    return from_cuda(launch_dequantize(q->codes, q->scales, q->tensor_scale, q->rows, q->cols, y,
+                                       yt == NVFP4_BF16, ldy, dev.sms,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static nvfp4_status check_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y,
+                               nvfp4_dtype yt, int64_t ldy) {
+    if (!a || !b || !y || (yt != NVFP4_F32 && yt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if (a->cols != b->cols) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_tensor(a, a->rows, a->cols);
+    if (st != NVFP4_OK) return st;
+    if ((st = check_tensor(b, b->rows, b->cols)) != NVFP4_OK) return st;
+    if (a->cols % 64) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (a->rows > INT32_MAX / 2 || b->rows > INT32_MAX / 2) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ldy < b->rows) return NVFP4_ERR_INVALID_ARG;
+    const int eb = yt == NVFP4_BF16 ? 2 : 4;
+    if (!aligned16(y) || (ldy * eb) % 16) return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+static nvfp4_status gemm_impl(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y,
+                              nvfp4_dtype yt, int64_t ldy, uint32_t *status, int num_sms,
+                              cudaStream_t stream) {
+    if (a->rows == 0 || b->rows == 0) return NVFP4_OK;
+    if (a->cols == 0)   // empty reduction: y = 0
+        return from_cuda(cudaMemset2DAsync(y, ldy * (yt == NVFP4_BF16 ? 2 : 4), 0,
+                                           b->rows * (yt == NVFP4_BF16 ? 2 : 4), a->rows, stream));
+    Operand act{a->codes, a->scales, a->tensor_scale, a->rows};
+    Operand wgt{b->codes, b->scales, b->tensor_scale, b->rows};
+    return from_cuda(launch_gemm(act, wgt, a->cols, y, yt == NVFP4_BF16, ldy, status, timeout_ns(),
+                                 num_sms, stream));
+}
+
+nvfp4_status nvfp4_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y, nvfp4_dtype yt,
+                        int64_t ldy, void *ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    nvfp4_status st = check_gemm(a, b, y, yt, ldy);
+    if (st != NVFP4_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, kWsStatusBytes)) != NVFP4_OK) return st;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    return gemm_impl(a, b, y, yt, ldy, static_cast<uint32_t *>(ws), dev.sms,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                const nvfp4_tensor *w, const nvfp4_tensor *w_up,
+                                nvfp4_epilogue epilogue, void *y, nvfp4_dtype yt, int64_t ldy,
+                                const nvfp4_tensor *y_q, const nvfp4_tensor *x_q, void *ws,
+                                size_t ws_bytes, nvfp4_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!x || !w || (xt != NVFP4_F32 && xt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if (M < 0 || K < 0 || ldx < K) return NVFP4_ERR_INVALID_ARG;
+    if (epilogue != NVFP4_EPI_STORE && epilogue != NVFP4_EPI_SILU_MUL_REQUANT)
+        return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_tensor(w, w->rows, K);
+    if (st != NVFP4_OK) return st;
+    if (K % 64) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const int xeb = xt == NVFP4_BF16 ? 2 : 4;
+    if (!aligned16(x) || (ldx * xeb) % 16) return NVFP4_ERR_MISALIGNED;
+    const int64_t N = w->rows;
+    if (epilogue == NVFP4_EPI_STORE) {
+        if (!y || (yt != NVFP4_F32 && yt != NVFP4_BF16) || ldy < N) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(y) || (ldy * (yt == NVFP4_BF16 ? 2 : 4)) % 16) return NVFP4_ERR_MISALIGNED;
+    } else {
+        if (!w_up || (st = check_tensor(w_up, N, K)) != NVFP4_OK)
+            return st != NVFP4_OK ? st : NVFP4_ERR_INVALID_ARG;
+        if ((st = check_tensor(y_q, M, N)) != NVFP4_OK) return st;
+        if (y && (yt != NVFP4_F32 || ldy < N)) return NVFP4_ERR_INVALID_ARG;
+        if (y && (!aligned16(y) || (ldy * 4) % 16)) return NVFP4_ERR_MISALIGNED;
+    }
+    if (x_q && (st = check_tensor(x_q, M, K)) != NVFP4_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, nvfp4_workspace_bytes(NVFP4_OP_LINEAR_FUSED, M, N, K))) != NVFP4_OK)
+        return st;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    if (M == 0) return NVFP4_OK;
+
+    // Quantized activations: caller's buffers or carved from the workspace.
+    size_t off = kQuantizeWs;
+    nvfp4_tensor xq;
+    if (x_q) {
+        xq = *x_q;
+    } else {
+        xq.codes = ws_at(ws, off);
+        off += align256(static_cast<size_t>(M * K / 2));
+        xq.scales = ws_at(ws, off);
+        off += align256(nvfp4_scales_bytes(M, K));
+        xq.tensor_scale = reinterpret_cast<float *>(ws_at(ws, off));
+        off += 256;
+        xq.rows = M;
+        xq.cols = K;
+    }
+    if (!x_q) off = kQuantizeWs + quantized_bytes(M, K);
+    cudaError_t e = launch_quantize(x, xt == NVFP4_BF16, M, K, ldx, xq.codes, xq.scales,
+                                    xq.tensor_scale, reinterpret_cast<float *>(ws_at(ws, kPartialsOff)),
+                                    dev.sms, stream);
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    uint32_t *status = static_cast<uint32_t *>(ws);
+    if (epilogue == NVFP4_EPI_STORE)
+        return gemm_impl(&xq, w, y, yt, ldy, status, dev.sms, stream);
+
+    // SiLU(gate) * up, then re-quantize h for the down projection.
+    const size_t mn = align256(static_cast<size_t>(M * N) * sizeof(float));
+    float *gate = reinterpret_cast<float *>(ws_at(ws, off));
+    float *up = reinterpret_cast<float *>(ws_at(ws, off + mn));
+    float *h = y ? static_cast<float *>(y) : reinterpret_cast<float *>(ws_at(ws, off + 2 * mn));
+    const int64_t ldh = y ? ldy : N;
+    if ((st = gemm_impl(&xq, w, gate, NVFP4_F32, N, status, dev.sms, stream)) != NVFP4_OK) return st;
+    if ((st = gemm_impl(&xq, w_up, up, NVFP4_F32, N, status, dev.sms, stream)) != NVFP4_OK) return st;
+    if (ldh == N) {
+        if (launch_silu_mul(gate, up, h, M * N, dev.sms, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
+    } else {
+        for (int64_t r = 0; r < M; ++r)
+            if (launch_silu_mul(gate + r * N, up + r * N, h + r * ldh, N, dev.sms, stream) != cudaSuccess)
+                return NVFP4_ERR_CUDA;
+    }
+    return from_cuda(launch_quantize(h, false, M, N, ldh, y_q->codes, y_q->scales,
+                                     y_q->tensor_scale,
+                                     reinterpret_cast<float *>(ws_at(ws, kPartialsOff)), dev.sms,
+                                     stream));
+}
+
+nvfp4_status nvfp4_get_device_status(void *ws, nvfp4_stream_t stream) {
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, ws, sizeof word, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (word) {
+        if (cudaMemsetAsync(ws, 0, sizeof word, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    }
+    for (int code = 1; code < 32; ++code)
+        if (word & (1u << code)) return static_cast<nvfp4_status>(code);
+    return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_selftest_bounded_wait(void *ws, uint32_t timeout_us, nvfp4_stream_t stream) {
+    nvfp4_status st = check_ws(ws, kWsStatusBytes, kWsStatusBytes);
+    if (st != NVFP4_OK) return st;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    return from_cuda(launch_wait_selftest(static_cast<uint32_t *>(ws),
+                                          static_cast<uint64_t>(timeout_us) * 1000ull,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+uint32_t nvfp4_set_wait_timeout_us(uint32_t timeout_us) {
+    return g_wait_timeout_us.exchange(timeout_us == 0 ? 1u : timeout_us);
+}
+
+const char *nvfp4_status_string(nvfp4_status s) {
+    switch (s) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case NVFP4_ERR_MISALIGNED: return "misaligned pointer or pitch";
+    case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_TIMEOUT: return "device-side wait timed out";
+    case NVFP4_ERR_ARCH: return "device is not sm_100";
+    }
+    return "unknown status";
+}
+
+int nvfp4_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,37 @@
+// common.cuh -- shapes, the tiled scale layout and small helpers shared by the
+// CUDA kernels of the library (never by the CPU oracle).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+constexpr int kBlock = 16;           // values per microblock (NVFP4 wiki page, "技術原理")
+constexpr float kTensorScaleDiv = 2688.0f;   // 6 (E2M1 max) * 448 (E4M3 max)
+
+__host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ __forceinline__ int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+// Number of 16-element blocks per row, padded to a multiple of 4 (one 32-bit
+// scale word per 64 columns).
+__host__ __device__ __forceinline__ int64_t kb4_of(int64_t cols) { return round_up(cols / kBlock, 4); }
+
+// Byte offset of the scale of block kb of row r in the tiled layout: 128-row x
+// 4-block atoms of 512 bytes, row r%32 at 16*(r%32), row quarter (r/32)%4 at
+// 4*((r/32)%4), block kb%4 at kb%4.  This is the order in which tcgen05.cp
+// (32x128b, replicated to four lane quarters) places scales where the
+// block-scaled MMA reads them: lane r%32 of every quarter, column (r/32)%4,
+// byte kb%4.
+__host__ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t kb, int64_t kb4) {
+    int64_t tile = (r >> 7) * (kb4 >> 2) + (kb >> 2);
+    return tile * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3);
+}
+
+// Workspace layout: [0,16) status words, [256, ...) scratch.
+constexpr size_t kWsStatusBytes = 256;
+constexpr int kMaxAmaxPartials = 4096;
+
+}  // namespace nvfp4

@@ -1,0 +1,434 @@
+// gemm.cu -- W4A4 block-scaled FP4 GEMM on the sm_100a tensor cores.
+//
+// The linear layer consumes NVFP4 weights and NVFP4 activations directly on
+// the FP4 tensor cores, with no dequantize-to-16-bit step (aixq.cc article on
+// Unsloth Dynamic NVFP4, section "核心差异：W4A4 vs W4A16"); the tensor cores
+// apply the per-16-element E4M3 block scales themselves, and the FP32 tensor
+// scales are applied once in the epilogue (NVFP4 wiki page, section "技術原理":
+// a second-level FP32 scale over the whole tensor).
+//
+// Design (one persistent CTA per SM, 6 warps):
+//   warp 0      TMA producer: for every 256-element K slab, a 128-row tile of
+//               the MMA's A operand and a BN-row tile of its B operand (packed
+//               E2M1, 128-byte swizzle) plus their 512-byte scale atoms (bulk
+//               copies) into a STAGES-deep shared-memory ring (mbarriers).
+//   warp 1      TMEM allocator and MMA issuer: copies the scale atoms into
+//               tensor memory (tcgen05.cp 32x128b, replicated to the 4 lane
+//               quarters) and issues tcgen05.mma kind::mxf4nvf4 (M=128,
+//               N=BN, K=64) into an fp32 accumulator in tensor memory.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator, y = acc * (gA*gB),
+//               RNE to bf16 (or fp32), and the store.
+// Small M (decode) runs "swapped": the weights ride the MMA's M = 128 and the
+// few activation rows ride N = BN, so the weight stream spreads over all SMs.
+// Every wait is bounded; a timeout sets the status word and winds the CTA
+// down without leaving tensor memory allocated.
+#include "common.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+struct GemmArgs {
+    const uint8_t *sfa;      // tiled scales of the MMA A operand (P rows)
+    const uint8_t *sfb;      // tiled scales of the MMA B operand (Q rows)
+    const float *ga;
+    const float *gb;
+    void *y;
+    int64_t ldy;
+    int32_t P, Q;            // rows of the A and B operands
+    int32_t num_k_steps;     // K / 64
+    int32_t num_p_tiles, num_q_tiles;
+    int32_t q_row_tiles;     // ceil(Q / 128): 128-row scale tiles of B
+    uint32_t *status;
+    uint64_t timeout_ns;
+};
+
+template <int BN>
+struct GemmCfg {
+    static constexpr int kNQT = (BN + 127) / 128;              // 128-row scale tiles per B tile
+    static constexpr int kAStage = 128 * 128;                  // bytes of A per stage
+    static constexpr int kBStage = BN * 128;
+    static constexpr int kSfaStage = 4 * 512;                  // 4 K-steps x one 512 B atom
+    static constexpr int kSfbStage = kNQT * 4 * 512;
+    static constexpr int kStageBytes = kAStage + kBStage + kSfaStage + kSfbStage;
+    static constexpr int kStages = (BN == 256) ? 4 : (BN == 128 ? 6 : (BN == 64 ? 7 : 8));
+    static constexpr int kSfCols = 16 + 16 * kNQT;             // TMEM columns for scales
+    static constexpr int kAccStages = (2 * BN + kSfCols <= 512) ? 2 : 1;
+    static constexpr int kSfaCol = kAccStages * BN;
+    static constexpr int kSfbCol = kSfaCol + 16;
+    static constexpr int kColsUsed = kSfbCol + 16 * kNQT;
+    static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
+                                   : kColsUsed <= 256 ? 256 : 512;
+    static constexpr int kBarBytes = 8 * (2 * kStages + 4) + 16;
+    static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;   // + alignment slack
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+};
+
+template <int BN, bool SWAP, typename OutT>
+__global__ void __launch_bounds__(192, 1)
+gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ GemmArgs args) {
+    using C = GemmCfg<BN>;
+    constexpr int STAGES = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = sA + STAGES * C::kAStage;
+    uint8_t *sSfa = sB + STAGES * C::kBStage;
+    uint8_t *sSfb = sSfa + STAGES * C::kSfaStage;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sSfb + STAGES * C::kSfbStage);
+    uint64_t *empty = full + STAGES;
+    uint64_t *tfull = empty + STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tempty + 2);
+    volatile uint32_t *abort_flag = tmem_holder + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&tfull[s], 1);
+            mbar_init(&tempty[s], 128);
+        }
+        *abort_flag = 0u;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_holder, C::kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    // Operands may come from the kernel launched just before (the quantizer).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    const int num_tiles = args.num_p_tiles * args.num_q_tiles;
+    const int num_kstages = (args.num_k_steps + 3) / 4;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------------------ producer
+        const uint64_t pol_a = SWAP ? policy_evict_first() : policy_evict_normal();
+        const uint64_t pol_b = SWAP ? policy_evict_last() : policy_evict_normal();
+        uint32_t stage = 0, phase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            const int pt = tile % args.num_p_tiles;
+            const int qt = tile / args.num_p_tiles;
+            bool ok = true;
+            for (int ks = 0; ks < num_kstages; ++ks) {
+                if (!mbar_wait(&empty[stage], phase ^ 1u, args.timeout_ns, abort_flag, args.status)) {
+                    ok = false;
+                    break;
+                }
+                const int nk = min(4, args.num_k_steps - 4 * ks);
+                int nq_loaded = 0;
+                for (int q = 0; q < C::kNQT; ++q) nq_loaded += (qt * C::kNQT + q < args.q_row_tiles);
+                const uint32_t bytes = C::kAStage + C::kBStage + nk * 512 * (1 + nq_loaded);
+                mbar_arrive_expect_tx(&full[stage], bytes);
+                tma_load_2d(sA + stage * C::kAStage, &tmA, &full[stage], ks * 128, pt * 128, pol_a);
+                tma_load_2d(sB + stage * C::kBStage, &tmB, &full[stage], ks * 128, qt * BN, pol_b);
+                bulk_load(sSfa + stage * C::kSfaStage,
+                          args.sfa + (static_cast<int64_t>(pt) * args.num_k_steps + 4 * ks) * 512,
+                          nk * 512, &full[stage], pol_a);
+                for (int q = 0; q < C::kNQT; ++q) {
+                    const int rt = qt * C::kNQT + q;
+                    if (rt < args.q_row_tiles)
+                        bulk_load(sSfb + stage * C::kSfbStage + q * 2048,
+                                  args.sfb + (static_cast<int64_t>(rt) * args.num_k_steps + 4 * ks) * 512,
+                                  nk * 512, &full[stage], pol_b);
+                }
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = make_idesc_nvf4(BN);
+        const uint32_t a_base = smem_addr(sA), b_base = smem_addr(sB);
+        const uint32_t sfa_base = smem_addr(sSfa), sfb_base = smem_addr(sSfb);
+        uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.timeout_ns, abort_flag, args.status)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + acc * BN;
+            bool ok = true;
+            for (int ks = 0; ks < num_kstages; ++ks) {
+                if (!mbar_wait(&full[stage], phase, args.timeout_ns, abort_flag, args.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int nk = min(4, args.num_k_steps - 4 * ks);
+                for (int j = 0; j < nk; ++j) {
+                    tc_cp_32x128b_warpx4(tmem_base + C::kSfaCol + 4 * j,
+                                         make_sf_desc(sfa_base + stage * C::kSfaStage + j * 512));
+#pragma unroll
+                    for (int q = 0; q < C::kNQT; ++q)
+                        tc_cp_32x128b_warpx4(tmem_base + C::kSfbCol + 4 * (j * C::kNQT + q),
+                                             make_sf_desc(sfb_base + stage * C::kSfbStage + q * 2048 + j * 512));
+                }
+                for (int j = 0; j < nk; ++j) {
+                    const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage + 32 * j);
+                    const uint64_t bdesc = make_operand_desc(b_base + stage * C::kBStage + 32 * j);
+                    mma_nvf4(d_tmem, adesc, bdesc, idesc, tmem_base + C::kSfaCol + 4 * j,
+                             tmem_base + C::kSfbCol + 4 * C::kNQT * j, (ks | j) != 0 ? 1u : 0u);
+                }
+                tc_commit(&empty[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            tc_commit(&tfull[acc]);
+            if (C::kAccStages == 2) {
+                acc ^= 1u;
+                if (acc == 0) acc_phase ^= 1u;
+            } else {
+                acc_phase ^= 1u;
+            }
+        }
+    } else if (warp >= 2) {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;               // TMEM lane quarter this warp may read
+        const int row = quarter * 32 + lane;        // accumulator row (MMA M index)
+        const float alpha = __fmul_rn(*args.ga, *args.gb);
+        constexpr int CH = BN < 32 ? BN : 32;
+        uint32_t acc = 0, acc_phase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            const int pt = tile % args.num_p_tiles;
+            const int qt = tile / args.num_p_tiles;
+            // The decision must be warp-uniform: tcgen05.ld below is .sync.aligned.
+            const bool ok = mbar_wait(&tfull[acc], acc_phase, args.timeout_ns, abort_flag, args.status);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const int p = pt * 128 + row;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += CH) {
+                uint32_t r[CH];
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN + c0;
+                if constexpr (CH == 32)
+                    tmem_ld_32x32b_x32(taddr, reinterpret_cast<uint32_t(&)[32]>(r));
+                else
+                    tmem_ld_32x32b_x16(taddr, reinterpret_cast<uint32_t(&)[16]>(r));
+                tmem_ld_wait();
+                float v[CH];
+#pragma unroll
+                for (int i = 0; i < CH; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+                const int q0 = qt * BN + c0;
+                if constexpr (SWAP) {
+                    // y[q][p]: for each i the warp writes 32 consecutive p
+                    if (p < args.P) {
+                        OutT *y = static_cast<OutT *>(args.y);
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) {
+                            const int q = q0 + i;
+                            if (q < args.Q) {
+                                if constexpr (sizeof(OutT) == 2)
+                                    y[static_cast<int64_t>(q) * args.ldy + p] = __float2bfloat16_rn(v[i]);
+                                else
+                                    y[static_cast<int64_t>(q) * args.ldy + p] = v[i];
+                            }
+                        }
+                    }
+                } else {
+                    // y[p][q0 .. q0+CH): one contiguous run per thread
+                    if (p < args.P) {
+                        OutT *yrow = static_cast<OutT *>(args.y) + static_cast<int64_t>(p) * args.ldy;
+                        if (q0 + CH <= args.Q) {
+                            if constexpr (sizeof(OutT) == 2) {
+#pragma unroll
+                                for (int i = 0; i < CH; i += 8) {
+                                    uint4 pk;
+                                    uint32_t *w = reinterpret_cast<uint32_t *>(&pk);
+#pragma unroll
+                                    for (int k = 0; k < 4; ++k) {
+                                        __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * k], v[i + 2 * k + 1]);
+                                        w[k] = *reinterpret_cast<uint32_t *>(&b2);
+                                    }
+                                    *reinterpret_cast<uint4 *>(yrow + q0 + i) = pk;
+                                }
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < CH; i += 4)
+                                    *reinterpret_cast<float4 *>(yrow + q0 + i) =
+                                        make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < CH; ++i) {
+                                if (q0 + i < args.Q) {
+                                    if constexpr (sizeof(OutT) == 2)
+                                        yrow[q0 + i] = __float2bfloat16_rn(v[i]);
+                                    else
+                                        yrow[q0 + i] = v[i];
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            if (C::kAccStages == 2) {
+                acc ^= 1u;
+                if (acc == 0) acc_phase ^= 1u;
+            } else {
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+CUresult encode_tensor_map_u8(CUtensorMap *map, const void *base, uint64_t inner_bytes,
+                              uint64_t rows, uint32_t box_inner, uint32_t box_rows) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return CUDA_ERROR_NOT_FOUND;
+    cuuint64_t dims[2] = {inner_bytes, rows};
+    cuuint64_t strides[1] = {inner_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+template <int BN, bool SWAP, typename OutT>
+static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, void *y, int64_t ldy,
+                            uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t stream) {
+    using C = GemmCfg<BN>;
+    CUtensorMap tmA, tmB;
+    if (encode_tensor_map_u8(&tmA, pa.codes, K / 2, pa.rows, 128, 128) != CUDA_SUCCESS ||
+        encode_tensor_map_u8(&tmB, qb.codes, K / 2, qb.rows, 128, BN) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    GemmArgs a;
+    a.sfa = pa.scales;
+    a.sfb = qb.scales;
+    a.ga = pa.g;
+    a.gb = qb.g;
+    a.y = y;
+    a.ldy = ldy;
+    a.P = static_cast<int32_t>(pa.rows);
+    a.Q = static_cast<int32_t>(qb.rows);
+    a.num_k_steps = static_cast<int32_t>(K / 64);
+    a.num_p_tiles = static_cast<int32_t>(ceil_div(pa.rows, 128));
+    a.num_q_tiles = static_cast<int32_t>(ceil_div(qb.rows, BN));
+    a.q_row_tiles = static_cast<int32_t>(ceil_div(qb.rows, 128));
+    a.status = status;
+    a.timeout_ns = timeout_ns;
+    const int tiles = a.num_p_tiles * a.num_q_tiles;
+    auto kern = gemm_nvf4_kernel<BN, SWAP, OutT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(tiles < num_sms ? tiles : num_sms);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
+}
+
+cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
+                        int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
+                        cudaStream_t stream) {
+    const int64_t M = act.rows, N = wgt.rows;
+    if (M <= 64) {
+        // weights on the MMA's M side, activations on N; y[m][n] = acc[n][m]
+        const int bn = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+#define NVFP4_SWAPPED(BNV)                                                                          \
+    return y_bf16 ? run_gemm<BNV, true, __nv_bfloat16>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, stream) \
+                  : run_gemm<BNV, true, float>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, stream);
+        if (bn == 16) { NVFP4_SWAPPED(16) }
+        if (bn == 32) { NVFP4_SWAPPED(32) }
+        NVFP4_SWAPPED(64)
+#undef NVFP4_SWAPPED
+    }
+    const int64_t ptiles = ceil_div(M, 128);
+    const bool wide = ptiles * ceil_div(N, 256) >= 2 * num_sms;
+    if (wide)
+        return y_bf16 ? run_gemm<256, false, __nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, stream)
+                      : run_gemm<256, false, float>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, stream);
+    return y_bf16 ? run_gemm<128, false, __nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, stream)
+                  : run_gemm<128, false, float>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Elementwise SiLU(gate) * up (fp32), SiLU(z) = z / (1 + exp(-z)).
+// ---------------------------------------------------------------------------
+__global__ void silu_mul_kernel(const float *__restrict__ gate, const float *__restrict__ up,
+                                float *__restrict__ h, int64_t n) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float z = gate[i];
+        h[i] = __fmul_rn(__fdiv_rn(z, __fadd_rn(1.0f, expf(-z))), up[i]);
+    }
+}
+
+cudaError_t launch_silu_mul(const float *gate, const float *up, float *h, int64_t n, int num_sms,
+                            cudaStream_t stream) {
+    int64_t blocks = ceil_div(n, 256);
+    const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+    blocks = blocks < 1 ? 1 : (blocks < cap ? blocks : cap);
+    silu_mul_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(gate, up, h, n);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Bounded-wait self test: one thread waits on a barrier nothing completes.
+// ---------------------------------------------------------------------------
+__global__ void wait_selftest_kernel(uint32_t *status, uint64_t timeout_ns) {
+    __shared__ uint64_t bar;
+    __shared__ uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0u;
+        fence_mbar_init();
+        // Phase 0 never completes: nobody arrives on the barrier.
+        mbar_wait(&bar, 0u, timeout_ns, &abort_flag, status);
+    }
+}
+
+cudaError_t launch_wait_selftest(uint32_t *status, uint64_t timeout_ns, cudaStream_t stream) {
+    wait_selftest_kernel<<<1, 32, 0, stream>>>(status, timeout_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,41 @@
+// kernels.cuh -- host launchers of the CUDA kernels (internal to the library).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld,
+                            uint8_t *codes, uint8_t *scales, float *g_out, float *partials,
+                            int num_sms, cudaStream_t stream);
+
+cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scales, const float *g,
+                              int64_t rows, int64_t cols, void *y, bool bf16, int64_t ldy,
+                              int num_sms, cudaStream_t stream);
+
+// One GEMM operand as the GEMM kernel reads it.
+struct Operand {
+    const uint8_t *codes;    // [rows][K/2]
+    const uint8_t *scales;   // tiled layout
+    const float *g;          // tensor scale (device)
+    int64_t rows;
+};
+
+// y[M][N] = (A . B^T) * gA * gB, A = act [M][K], B = wgt [N][K].
+cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
+                        int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
+                        cudaStream_t stream);
+
+// h = SiLU(gate) * up elementwise in fp32 (n values).
+cudaError_t launch_silu_mul(const float *gate, const float *up, float *h, int64_t n, int num_sms,
+                            cudaStream_t stream);
+
+cudaError_t launch_wait_selftest(uint32_t *status, uint64_t timeout_ns, cudaStream_t stream);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+CUresult encode_tensor_map_u8(CUtensorMap *map, const void *base, uint64_t inner_bytes,
+                              uint64_t rows, uint32_t box_inner, uint32_t box_rows);
+
+}  // namespace nvfp4

@@ -1,0 +1,108 @@
+"""CPU-side checks of the C ABI: the library loads, exports every function the
+header declares, reports sizes, and rejects bad arguments synchronously
+without touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_block_scaled_21_b200 as nv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "nvfp4.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_four_entry_points():
+    names = declared_functions()
+    for n in ("nvfp4_quantize", "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_linear_fused"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = nv.lib()
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(nv.EXPORTED) == set(declared_functions())
+
+
+def test_sizes():
+    assert nv.codes_bytes(8192, 5120) == 8192 * 5120 // 2
+    assert nv.scales_bytes(8192, 5120) == 8192 * 320
+    assert nv.scales_bytes(8, 5120) == 128 * 320          # rows padded to 128
+    assert nv.scales_bytes(1, 16) == 128 * 4              # blocks padded to 4
+    assert nv.scales_bytes(130, 80) == 256 * 8
+    assert nv.workspace_bytes(nv.OP_GEMM, 1, 1, 64) >= 256
+    assert nv.workspace_bytes(nv.OP_QUANTIZE, 10, 0, 16) >= 256 + 4 * 1184
+    assert nv.version() >= 100
+
+
+def test_status_strings():
+    assert nv.status_string(nv.OK) == "ok"
+    assert "timed out" in nv.status_string(nv.ERR_TIMEOUT)
+    assert nv.status_string(99) == "unknown status"
+
+
+def _t(codes=16, scales=16, g=16, rows=4, cols=64):
+    return nv.CTensor(codes, scales, g, rows, cols)
+
+
+def test_quantize_rejects_bad_arguments_without_launch():
+    lib = nv.lib()
+    ws = 4096
+    out = _t()
+    q = lambda x, xt, r, c, ld, o, w, wb: lib.nvfp4_quantize(x, xt, r, c, ld, ctypes.byref(o) if o else None, w, wb, None)
+    assert q(None, nv.BF16, 4, 64, 64, out, ws, 1 << 20) == nv.ERR_INVALID_ARG
+    assert q(16, 7, 4, 64, 64, out, ws, 1 << 20) == nv.ERR_INVALID_ARG
+    assert q(16, nv.BF16, 4, 64, 32, out, ws, 1 << 20) == nv.ERR_INVALID_ARG      # ld < cols
+    assert q(16, nv.BF16, 4, 64, 64, None, ws, 1 << 20) == nv.ERR_INVALID_ARG
+    assert q(16, nv.BF16, 4, 64, 64, _t(rows=5), ws, 1 << 20) == nv.ERR_INVALID_ARG
+    assert q(16, nv.BF16, 4, 24, 24, _t(cols=24), ws, 1 << 20) == nv.ERR_UNSUPPORTED_SHAPE
+    assert q(18, nv.BF16, 4, 64, 64, out, ws, 1 << 20) == nv.ERR_MISALIGNED
+    assert q(16, nv.BF16, 4, 64, 68, out, ws, 1 << 20) == nv.ERR_MISALIGNED       # row pitch
+    assert q(16, nv.BF16, 4, 64, 64, _t(codes=24), ws, 1 << 20) == nv.ERR_MISALIGNED
+    assert q(16, nv.BF16, 4, 64, 64, out, None, 1 << 20) == nv.ERR_WORKSPACE
+    assert q(16, nv.BF16, 4, 64, 64, out, ws, 100) == nv.ERR_WORKSPACE
+
+
+def test_gemm_rejects_bad_arguments_without_launch():
+    lib = nv.lib()
+    a, b = _t(rows=8, cols=128), _t(rows=32, cols=128)
+    g = lambda a, b, y, yt, ldy, ws, wb: lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), y, yt, ldy, ws, wb, None)
+    assert g(a, b, None, nv.BF16, 32, 4096, 256) == nv.ERR_INVALID_ARG
+    assert g(a, _t(rows=32, cols=64), 16, nv.BF16, 32, 4096, 256) == nv.ERR_INVALID_ARG   # K mismatch
+    assert g(_t(rows=8, cols=96), _t(rows=32, cols=96), 16, nv.BF16, 32, 4096, 256) == nv.ERR_UNSUPPORTED_SHAPE
+    assert g(a, b, 16, nv.BF16, 16, 4096, 256) == nv.ERR_INVALID_ARG                       # ldy < N
+    assert g(a, b, 16, nv.BF16, 36, 4096, 256) == nv.ERR_MISALIGNED                        # pitch
+    assert g(a, b, 16, nv.BF16, 32, 4096, 8) == nv.ERR_WORKSPACE
+
+
+def test_linear_fused_rejects_bad_arguments_without_launch():
+    lib = nv.lib()
+    w = _t(rows=32, cols=128)
+    f = lambda epi, wu, yq, y: lib.nvfp4_linear_fused(16, nv.BF16, 8, 128, 128, ctypes.byref(w),
+                                                      ctypes.byref(wu) if wu else None, epi, y,
+                                                      nv.BF16, 32, ctypes.byref(yq) if yq else None,
+                                                      None, 4096, 1 << 30, None)
+    assert f(nv.EPI_STORE, None, None, None) == nv.ERR_INVALID_ARG                  # y missing
+    assert f(5, None, None, 16) == nv.ERR_INVALID_ARG
+    assert f(nv.EPI_SILU_MUL_REQUANT, None, _t(rows=8, cols=32), None) == nv.ERR_INVALID_ARG
+    assert f(nv.EPI_SILU_MUL_REQUANT, _t(rows=16, cols=128), _t(rows=8, cols=32), None) == nv.ERR_INVALID_ARG
+
+
+def test_package_fails_loudly_without_library(tmp_path):
+    """The binding refuses to import when libnvfp4.so is absent: no CPU fallback."""
+    import subprocess
+    import sys
+    import shutil
+    pkg = tmp_path / "nvfp4_block_scaled_21_b200"
+    shutil.copytree(os.path.join(ROOT, "nvfp4_block_scaled_21_b200"), pkg,
+                    ignore=shutil.ignore_patterns("*.so", "csrc", "__pycache__"))
+    r = subprocess.run([sys.executable, "-c", "import nvfp4_block_scaled_21_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libnvfp4.so is missing" in r.stderr

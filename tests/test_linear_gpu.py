@@ -1,0 +1,104 @@
+"""GPU parity of the fused linear layer (activation quantize + W4A4 GEMM) and
+of the MLP step SiLU(gate)*up re-quantized to NVFP4, then the down GEMM.
+
+The MLP check has three parts, since the GPU's fp32 h is not bit-equal to the
+oracle's fp64 h: (i) GPU h against fp64 SiLU(gate)*up within the propagated
+GEMM tolerance; (ii) GPU h_q bit-exact against the oracle quantizer fed the
+GPU's own h; (iii) the down projection against the fp64 GEMM of that h_q."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import (assert_gemm_close, assert_quantized_equal, bf16_tensor, f32_tensor,
+                         gemm_tolerance, to_numpy_f64)
+from nvfp4_block_scaled_21_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import nvfp4_block_scaled_21_b200 as nv
+    return nv
+
+
+def quantize_gpu(nv, x):
+    out = nv.NVFP4Tensor.empty(*x.shape)
+    nv.nvfp4_quantize(x, out, nv.workspace(nv.OP_QUANTIZE, x.shape[0], 0, x.shape[1]))
+    return out
+
+
+def norms(q):
+    return np.linalg.norm(oracle.dequantize_f64(q), axis=1)
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 512, 1024), (96, 384, 640), (300, 256, 256)])
+def test_linear_store(nv, M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[rng.random(x.shape) < 1e-3] *= 50
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    xbits = xb.view(torch.int16).numpy().view(np.uint16)
+    wt = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    xq_o, wq_o = oracle.quantize(xbits), oracle.quantize(wt)
+    wq = quantize_gpu(nv, f32_tensor(wt))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    x_q = nv.NVFP4Tensor.empty(M, K)
+    ws = nv.workspace(nv.OP_LINEAR_FUSED, M, N, K)
+    nv.nvfp4_linear_fused(xb.cuda(), wq, ws, nv.EPI_STORE, y=y, x_q=x_q)
+    assert nv.nvfp4_get_device_status(ws) == nv.OK
+    assert_quantized_equal(x_q, xq_o)
+    ref = oracle.gemm_f64(xq_o, wq_o)
+    assert_gemm_close(to_numpy_f64(y), ref, norms(xq_o)[:, None], norms(wq_o)[None, :], K, True, "linear")
+
+
+def _silu(z):
+    return z / (1.0 + np.exp(-z))
+
+
+def check_mlp(nv, X, Wg, Wu, Wd, M, K, N):
+    """X bf16 bits [M][K]; Wg, Wu [N][K]; Wd [K][N] (bf16 bits)."""
+    xq_o = oracle.quantize(X)
+    wg_o, wu_o, wd_o = oracle.quantize(Wg), oracle.quantize(Wu), oracle.quantize(Wd)
+    wg, wu, wd = (quantize_gpu(nv, bf16_tensor(a)) for a in (Wg, Wu, Wd))
+    h = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    h_q = nv.NVFP4Tensor.empty(M, N)
+    ws = nv.workspace(nv.OP_LINEAR_FUSED, M, N, K)
+    nv.nvfp4_linear_fused(bf16_tensor(X), wg, ws, nv.EPI_SILU_MUL_REQUANT, y=h, w_up=wu, y_q=h_q)
+    y = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    nv.nvfp4_gemm(h_q, wd, y, nv.workspace(nv.OP_GEMM, M, K, N))
+    assert nv.nvfp4_get_device_status(ws) == nv.OK
+
+    # (i) h against fp64 SiLU(gate) * up with the GEMM tolerance propagated
+    gate = oracle.gemm_f64(xq_o, wg_o)
+    up = oracle.gemm_f64(xq_o, wu_o)
+    h_ref = oracle.silu_mul_f64(gate, up)
+    nx = norms(xq_o)[:, None]
+    tg = gemm_tolerance(gate, nx, norms(wg_o)[None, :], K, False)
+    tu = gemm_tolerance(up, nx, norms(wu_o)[None, :], K, False)
+    dsilu_max = 1.1   # |d/dz z*sigmoid(z)| <= 1.0998
+    tol_h = dsilu_max * (np.abs(up) + tu) * tg + np.abs(_silu(gate)) * tu + 1e-6 * np.abs(h_ref)
+    hc = h.cpu().numpy().astype(np.float64)
+    err = np.abs(hc - h_ref)
+    assert (err <= tol_h).all(), f"h: max err/tol {(err / tol_h).max():.3f}"
+
+    # (ii) h_q bit-exact against the oracle quantizer fed the GPU's h
+    hq_o = oracle.quantize(h.cpu().numpy())
+    assert_quantized_equal(h_q, hq_o)
+
+    # (iii) the down projection against the fp64 GEMM of that h_q
+    ref = oracle.gemm_f64(hq_o, wd_o)
+    assert_gemm_close(to_numpy_f64(y), ref, norms(hq_o)[:, None], norms(wd_o)[None, :], N, True, "down")
+
+
+def test_mlp_small(nv):
+    M, K, N = 32, 512, 384
+    w = workloads.make("mlp", M=M, K=K, N=N, seed=40)
+    check_mlp(nv, w["X"], w["Wg"], w["Wu"], w["Wd"], M, K, N)
+
+
+def test_mlp_workload_full(nv):
+    """The fused MLP workload at full size: M=128, K=5120, N=17408 (seed 4)."""
+    w = workloads.make("mlp")
+    check_mlp(nv, w["X"], w["Wg"], w["Wu"], w["Wd"], 128, 5120, 17408)

@@ -1,0 +1,154 @@
+"""GPU parity of the quantizer and dequantizer against the CPU oracle:
+packed codes, tiled scales (padding included) and the tensor scale must be
+bit-exact."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import (assert_quantized_equal, bf16_tensor, f32_tensor, tiled_scales)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import nvfp4_block_scaled_21_b200 as nv
+    return nv
+
+
+def quantize_gpu(nv, x_dev, ld=None):
+    rows, cols = x_dev.shape
+    if ld is not None and ld != cols:
+        buf = torch.zeros((rows, ld), dtype=x_dev.dtype, device=x_dev.device)
+        buf[:, :cols] = x_dev
+        x_dev = buf[:, :cols]
+    out = nv.NVFP4Tensor.empty(rows, cols)
+    ws = nv.workspace(nv.OP_QUANTIZE, rows, 0, cols)
+    nv.nvfp4_quantize(x_dev, out, ws)
+    return out
+
+
+def test_worked_example(nv, golden_dir):
+    with open(os.path.join(golden_dir, "worked_example_1x32.json")) as f:
+        ex = json.load(f)
+    x = np.array([float(v) for v in ex["x"]], np.float32).reshape(1, 32)
+    out = quantize_gpu(nv, f32_tensor(x))
+    torch.cuda.synchronize()
+    assert [f"{b:02x}" for b in out.codes.cpu().numpy()[0]] == ex["packed_bytes_hex"]
+    sc = out.scales.cpu().numpy()
+    assert [f"{sc[0]:02x}", f"{sc[1]:02x}"] == ex["scales_hex"]
+    assert out.tensor_scale[0].item() == float(ex["g"])
+    assert_quantized_equal(out, oracle.quantize(x))
+
+
+@pytest.mark.parametrize("k", [0, -20, 30])
+def test_round_trip_every_representable_value(nv, k):
+    """Every positive finite E4M3 scale with all 16 codes (same construction
+    as the oracle pin) gives the same bytes on the GPU."""
+    rows = [np.zeros(16, np.float32)]
+    rows[0][0] = np.float32(2688.0 * 2.0 ** k)
+    order = [7] + [c for c in range(16) if c != 7]
+    for s in range(1, 0x7F):
+        ds = oracle.e4m3_value(s)
+        rows.append(np.array([oracle.e2m1_value(c) * ds * 2.0 ** k for c in order], np.float32))
+    x = np.stack(rows)
+    assert_quantized_equal(quantize_gpu(nv, f32_tensor(x)), oracle.quantize(x))
+    # the bf16 path sees the same values (all of them are exact in bf16)
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    assert torch.equal(xb.float(), torch.from_numpy(x))
+    assert_quantized_equal(quantize_gpu(nv, xb.cuda()), oracle.quantize(x))
+
+
+def _rand(rows, cols, seed, outliers=True):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, cols)).astype(np.float32)
+    if outliers:
+        m = rng.random(x.shape) < 1e-3
+        x[m] = (rng.standard_normal(m.sum()) * 50).astype(np.float32)
+    return x
+
+
+SHAPES = [(1, 16), (2, 48), (3, 80), (17, 1040), (129, 64), (300, 640), (257, 5120)]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_quantize_parity(nv, shape, dtype):
+    x = _rand(*shape, seed=shape[0] * 7 + shape[1])
+    if dtype == "bf16":
+        xt = torch.from_numpy(x).to(torch.bfloat16)
+        bits = xt.view(torch.int16).numpy().view(np.uint16)
+        q = oracle.quantize(bits)
+        xd = xt.cuda()
+    else:
+        q = oracle.quantize(x)
+        xd = f32_tensor(x)
+    assert_quantized_equal(quantize_gpu(nv, xd), q)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_quantize_row_pitch(nv, dtype):
+    x = _rand(37, 96, seed=5)
+    xd = f32_tensor(x) if dtype == "f32" else f32_tensor(x).to(torch.bfloat16)
+    ref = oracle.quantize(x if dtype == "f32" else xd.cpu().view(torch.int16).numpy().view(np.uint16))
+    assert_quantized_equal(quantize_gpu(nv, xd, ld=160), ref)
+
+
+def test_quantize_edge_cases(nv):
+    # all zeros, including a negative zero
+    z = np.zeros((5, 32), np.float32)
+    z[2, 3] = -0.0
+    assert_quantized_equal(quantize_gpu(nv, f32_tensor(z)), oracle.quantize(z))
+    # zero-scale blocks next to normal ones; tiny amax
+    t = np.zeros((3, 48), np.float32)
+    t[0, 0] = np.float32(2688 * 2.0 ** -120)
+    t[0, 16] = np.float32(2.0 ** -134)
+    t[1, 0] = np.float32(-3.0 * 2.0 ** -130)
+    t[2, 5] = np.float32(-1e-38)
+    assert_quantized_equal(quantize_gpu(nv, f32_tensor(t)), oracle.quantize(t))
+    # negative values that round to zero keep their sign; exact E2M1 ties
+    s = np.zeros((1, 32), np.float32)
+    s[0, :16] = [6, -0.1, -0.0, 0.1, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, -5, -0.25, 7, -7, 0]
+    s[0, 16:] = np.linspace(-3, 3, 16)
+    assert_quantized_equal(quantize_gpu(nv, f32_tensor(s)), oracle.quantize(s))
+    # a single huge value: every other block's scale underflows towards zero
+    h = _rand(4, 64, seed=9, outliers=False)
+    h[0, 0] = 3e38
+    assert_quantized_equal(quantize_gpu(nv, f32_tensor(h)), oracle.quantize(h))
+
+
+def test_quantize_empty(nv):
+    out = quantize_gpu(nv, torch.zeros((0, 64), device="cuda"))
+    torch.cuda.synchronize()
+    assert out.tensor_scale[0].item() == 0.0
+
+
+def test_quantize_full_size_quantize_workload(nv):
+    """The 8192x5120 bf16 quantize workload (seed 1), launched exactly as the
+    benchmark launches it, bit-exact over the whole tensor."""
+    from nvfp4_block_scaled_21_b200 import workloads
+    w = workloads.make("quantize")
+    q = oracle.quantize(w["X"])
+    assert_quantized_equal(quantize_gpu(nv, bf16_tensor(w["X"])), q)
+
+
+@pytest.mark.parametrize("shape", [(1, 16), (7, 96), (130, 320)])
+def test_dequantize_parity(nv, shape):
+    x = _rand(*shape, seed=11)
+    q = oracle.quantize(x)
+    ref = oracle.dequantize(q)
+    t = nv.NVFP4Tensor.empty(*shape)
+    t.codes.copy_(torch.from_numpy(q.codes))
+    t.scales.copy_(torch.from_numpy(tiled_scales(q.scales)))
+    t.tensor_scale[0] = float(q.g)
+    y = torch.empty(shape, dtype=torch.float32, device="cuda")
+    nv.nvfp4_dequantize(t, y)
+    got = y.cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    yb = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    nv.nvfp4_dequantize(t, yb)
+    assert torch.equal(yb.cpu(), torch.from_numpy(ref).to(torch.bfloat16))
