@@ -1,0 +1,592 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 hot path on B200: activation quantize + W4A4
+block-scaled GEMM (prefill, decode), the standalone quantizer, and the fused
+MLP step.  Prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill|decode|quantize|mlp]
+
+A step is one pass of the hot path over one batch of synthetic input already
+resident in HBM.  The headline workload (default: prefill, M=4096 N=17408
+K=5120) is timed over exactly K steps bracketed by a barrier and a device
+synchronize; the other workloads are measured the same way and reported under
+"workloads".  L2 (126 MB) is defeated by rotating enough input copies that
+each step's operands were evicted by the steps before it.  Multi-GPU runs are
+independent batches per rank (weak scaling, no data-path collective); the
+time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP4_PER_BF16 = 4.0          # dense FP4 : dense BF16 on B200 (9 : 2.25 PFLOP/s nominal)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML)
+# ---------------------------------------------------------------------------
+_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def _reasons_now(self):
+        n = self.nvml
+        f = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(n, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return f(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                self.reasons |= int(self._reasons_now())
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": [name for bit, name in _REASONS.items() if self.reasons & bit],
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+
+class Timer:
+    """CUDA events around one kernel inside each step, on the launching stream."""
+
+    def __init__(self, torch, n):
+        self.ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(n)]
+        self.i = 0
+
+    def begin(self):
+        self.ev[self.i][0].record()
+
+    def end(self):
+        self.ev[self.i][1].record()
+        self.i += 1
+
+    def mean_us(self):
+        ts = [a.elapsed_time(b) * 1e3 for a, b in self.ev[:self.i]]
+        return sum(ts) / len(ts) if ts else float("nan")
+
+
+def _copies(t, n):
+    return [t] + [t.clone() for _ in range(n - 1)]
+
+
+def _clone_q(nv, q, n):
+    out = [q]
+    for _ in range(n - 1):
+        out.append(nv.NVFP4Tensor(q.codes.clone(), q.scales.clone(), q.tensor_scale.clone(),
+                                  q.rows, q.cols))
+    return out
+
+
+def _gen(name):
+    from nvfp4_block_scaled_21_b200 import workloads
+    return workloads.make(name)
+
+
+def _bf16(torch, bits):
+    import numpy as np
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+class Prefill:
+    name = "prefill"
+    metric = "NVFP4 GEMM TFLOPS (prefill)"
+    unit = "TFLOP/s"
+
+    def __init__(self, nv, torch, data=None):
+        w = data or _gen("prefill")
+        self.M, self.K, self.N = w["M"], w["K"], w["N"]
+        W = _bf16(torch, w["W"])
+        wq = nv.quantize(W)
+        del W
+        X = _bf16(torch, w["X"])
+        per_step = X.numel() * 2 + wq.codes.numel() + wq.scales.numel()
+        self.R = max(2, -(-2 * L2_BYTES // per_step))
+        self.X = _copies(X, self.R)
+        self.Wq = _clone_q(nv, wq, self.R)
+        self.xq = [nv.NVFP4Tensor.empty(self.M, self.K) for _ in range(self.R)]
+        self.y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device="cuda")
+        self.wsq = nv.workspace(nv.OP_QUANTIZE, self.M, 0, self.K)
+        self.wsg = nv.workspace(nv.OP_GEMM, self.M, self.N, self.K)
+        self.wsl = nv.workspace(nv.OP_LINEAR_FUSED, self.M, self.N, self.K)
+        self.nv, self.torch = nv, torch
+        self.flops = 2.0 * self.M * self.N * self.K
+        self.units = self.flops / 1e12          # TFLOP per step
+        self.launches = 3                       # amax, encode, GEMM
+        self.dominant = {"kernel": "gemm_nvf4_kernel (128x256 tiles)", "bound": "tensor",
+                         "algorithmic": self.flops, "unit": "TFLOP/s"}
+        self.config = {"workload": f"prefill W4A4 linear: quantize X bf16 {self.M}x{self.K} per call, "
+                                   f"GEMM with pre-quantized W {self.N}x{self.K}, bf16 out",
+                       "M": self.M, "N": self.N, "K": self.K,
+                       "l2": f"{self.R} rotating copies of X and W_q ({self.R * per_step / 2**20:.0f} MiB) > 126 MB L2"}
+
+    def step(self, i, timer=None):
+        r = i % self.R
+        self.nv.nvfp4_quantize(self.X[r], self.xq[r], self.wsq)
+        if timer: timer.begin()
+        self.nv.nvfp4_gemm(self.xq[r], self.Wq[r], self.y, self.wsg)
+        if timer: timer.end()
+
+    def e2e_setup(self):
+        self.x_host = self.X[0].cpu().pin_memory()
+        self.y_host = torch_empty_pinned(self.torch, self.y)
+        self.h2d = self.x_host.numel() * 2
+        self.d2h = self.y.numel() * 2
+
+    def e2e_step(self, i):
+        r = i % self.R
+        self.X[r].copy_(self.x_host, non_blocking=True)
+        self.nv.nvfp4_linear_fused(self.X[r], self.Wq[r], self.wsl, self.nv.EPI_STORE, y=self.y)
+        self.y_host.copy_(self.y, non_blocking=True)
+
+    def value(self, seconds_per_step):
+        return self.units / seconds_per_step
+
+
+class Decode(Prefill):
+    name = "decode"
+    metric = "NVFP4 GEMM GB/s (decode)"
+    unit = "GB/s"
+
+    def __init__(self, nv, torch):
+        super().__init__(nv, torch, _gen("decode"))
+        M, N, K = self.M, self.N, self.K
+        w_bytes = N * K // 2 + N * K // 16
+        # algorithmic bytes of the step: W codes + W scales, X bf16 in, Y bf16 out
+        self.bytes = w_bytes + M * K * 2 + M * N * 2
+        self.units = self.bytes / 1e9
+        gemm_bytes = w_bytes + M * K // 2 + M * K // 16 + M * N * 2
+        self.dominant = {"kernel": "gemm_nvf4_kernel (swapped, 128x16 tiles)", "bound": "hbm",
+                         "algorithmic": gemm_bytes, "unit": "GB/s"}
+        self.config["workload"] = (f"decode W4A4 linear: quantize X bf16 {M}x{K} per call, GEMM with "
+                                   f"pre-quantized W {N}x{K}, bf16 out")
+        self.config["algorithmic_bytes_per_step"] = self.bytes
+
+
+class Quantize:
+    name = "quantize"
+    metric = "NVFP4 quantize GB/s"
+    unit = "GB/s"
+
+    def __init__(self, nv, torch):
+        w = _gen("quantize")
+        self.M, self.K = w["M"], w["K"]
+        X = _bf16(torch, w["X"])
+        self.R = max(2, -(-2 * L2_BYTES // (X.numel() * 2)))
+        self.X = _copies(X, self.R)
+        self.q = [nv.NVFP4Tensor.empty(self.M, self.K) for _ in range(self.R)]
+        self.ws = nv.workspace(nv.OP_QUANTIZE, self.M, 0, self.K)
+        self.nv, self.torch = nv, torch
+        n = self.M * self.K
+        # one read of x plus the writes (codes, scales, tensor scale)
+        self.bytes = n * 2 + n // 2 + n // 16 + 4
+        self.bytes_two_pass = self.bytes + n * 2
+        self.units = self.bytes / 1e9
+        self.launches = 2
+        self.dominant = {"kernel": "amax_partials_kernel + encode_kernel", "bound": "hbm",
+                         "algorithmic": self.bytes, "unit": "GB/s"}
+        self.config = {"workload": f"quantize bf16 {self.M}x{self.K} to NVFP4 (codes, tiled E4M3 scales, fp32 tensor scale)",
+                       "rows": self.M, "cols": self.K,
+                       "algorithmic_bytes_per_step": self.bytes,
+                       "two_pass_bytes_per_step": self.bytes_two_pass,
+                       "l2": f"{self.R} rotating copies of x ({self.R * n * 2 / 2**20:.0f} MiB) > 126 MB L2"}
+
+    def step(self, i, timer=None):
+        r = i % self.R
+        if timer: timer.begin()
+        self.nv.nvfp4_quantize(self.X[r], self.q[r], self.ws)
+        if timer: timer.end()
+
+    def e2e_setup(self):
+        self.x_host = self.X[0].cpu().pin_memory()
+        self.c_host = torch_empty_pinned(self.torch, self.q[0].codes)
+        self.h2d = self.x_host.numel() * 2
+        self.d2h = self.q[0].codes.numel() + self.q[0].scales.numel() + 4
+        self.s_host = torch_empty_pinned(self.torch, self.q[0].scales)
+        self.g_host = torch_empty_pinned(self.torch, self.q[0].tensor_scale)
+
+    def e2e_step(self, i):
+        r = i % self.R
+        self.X[r].copy_(self.x_host, non_blocking=True)
+        self.nv.nvfp4_quantize(self.X[r], self.q[r], self.ws)
+        self.c_host.copy_(self.q[r].codes, non_blocking=True)
+        self.s_host.copy_(self.q[r].scales, non_blocking=True)
+        self.g_host.copy_(self.q[r].tensor_scale, non_blocking=True)
+
+    def value(self, seconds_per_step):
+        return self.units / seconds_per_step
+
+
+class Mlp:
+    name = "mlp"
+    metric = "NVFP4 fused MLP GB/s (M=128)"
+    unit = "GB/s"
+
+    def __init__(self, nv, torch):
+        w = _gen("mlp")
+        self.M, self.K, self.N = w["M"], w["K"], w["N"]
+        M, K, N = self.M, self.K, self.N
+        wg, wu, wd = (nv.quantize(_bf16(torch, w[k])) for k in ("Wg", "Wu", "Wd"))
+        X = _bf16(torch, w["X"])
+        per_step = 3 * (N * K // 2 + N * K // 16)
+        self.R = max(2, -(-2 * L2_BYTES // per_step))
+        self.X = _copies(X, self.R)
+        self.wg, self.wu, self.wd = (_clone_q(nv, q, self.R) for q in (wg, wu, wd))
+        self.hq = nv.NVFP4Tensor.empty(M, N)
+        self.y = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+        self.wsl = nv.workspace(nv.OP_LINEAR_FUSED_SILU, M, N, K)
+        self.wsg = nv.workspace(nv.OP_GEMM, M, K, N)
+        self.nv, self.torch = nv, torch
+        hq_bytes = M * N // 2 + M * N // 16
+        self.bytes = per_step + M * K * 2 + M * K * 2 + 2 * hq_bytes
+        self.units = self.bytes / 1e9
+        self.launches = 8
+        self.dominant = {"kernel": "gemm_nvf4_kernel (down projection, K=17408)", "bound": "hbm",
+                         "algorithmic": N * K // 2 + N * K // 16 + hq_bytes + M * K * 2,
+                         "unit": "GB/s"}
+        self.config = {"workload": f"fused MLP M={M}: quantize X, gate/up K={K} N={N}, SiLU(gate)*up "
+                                   f"re-quantized to NVFP4, down K={N} N={K}, bf16 out",
+                       "M": M, "K": K, "N": N, "algorithmic_bytes_per_step": self.bytes,
+                       "flops_per_step": 2.0 * M * N * K * 3,
+                       "l2": f"{self.R} rotating copies of the three weight matrices > 126 MB L2"}
+
+    def step(self, i, timer=None):
+        r = i % self.R
+        nv = self.nv
+        nv.nvfp4_linear_fused(self.X[r], self.wg[r], self.wsl, nv.EPI_SILU_MUL_REQUANT,
+                              w_up=self.wu[r], y_q=self.hq)
+        if timer: timer.begin()
+        nv.nvfp4_gemm(self.hq, self.wd[r], self.y, self.wsg)
+        if timer: timer.end()
+
+    def e2e_setup(self):
+        self.x_host = self.X[0].cpu().pin_memory()
+        self.y_host = torch_empty_pinned(self.torch, self.y)
+        self.h2d = self.x_host.numel() * 2
+        self.d2h = self.y.numel() * 2
+
+    def e2e_step(self, i):
+        r = i % self.R
+        self.X[r].copy_(self.x_host, non_blocking=True)
+        self.step(i)
+        self.y_host.copy_(self.y, non_blocking=True)
+
+    def value(self, seconds_per_step):
+        return self.units / seconds_per_step
+
+
+WORKLOADS = {"prefill": Prefill, "decode": Decode, "quantize": Quantize, "mlp": Mlp}
+
+
+def torch_empty_pinned(torch, like):
+    return torch.empty(like.shape, dtype=like.dtype, pin_memory=True)
+
+
+# ---------------------------------------------------------------------------
+# measurement
+# ---------------------------------------------------------------------------
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measure(wl, torch, K, W, world, local, sample_clocks=False):
+    for i in range(W):
+        wl.step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    timer = Timer(torch, K)
+    sampler = ClockSampler(local) if sample_clocks else None
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ctx = sampler if sampler else _Null()
+    with ctx:
+        start.record()
+        for i in range(K):
+            wl.step(W + i, timer)
+        end.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    elapsed = max_over_ranks(world, start.elapsed_time(end) / 1e3)
+    kern_us = max_over_ranks(world, timer.mean_us())
+    return elapsed, kern_us, (sampler.summary() if sampler else None)
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def measure_e2e(wl, torch, K, world):
+    wl.e2e_setup()
+    for i in range(2):
+        wl.e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(K):
+        wl.e2e_step(i)
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(world, start.elapsed_time(end) / 1e3)
+
+
+def roofline(wl, kern_us, peaks):
+    d = wl.dominant
+    if d["bound"] == "tensor":
+        achieved = d["algorithmic"] / (kern_us * 1e-6) / 1e12
+        peak = peaks["bf16_tflops"] * FP4_PER_BF16
+        unit = "TFLOP/s"
+        peak_note = (f"dense FP4 = {FP4_PER_BF16:g} x {peaks['source']} bf16 burst "
+                     f"{peaks['bf16_tflops']:.1f} TFLOP/s")
+    else:
+        achieved = d["algorithmic"] / (kern_us * 1e-6) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+        peak_note = f"{peaks['source']} HBM copy bandwidth"
+    return {"bound": d["bound"], "achieved": round(achieved, 1), "peak": round(peak, 1),
+            "unit": unit, "frac": round(achieved / peak, 4), "traffic": None,
+            "kernel": d["kernel"], "kernel_us": round(kern_us, 2),
+            "algorithmic_per_launch": d["algorithmic"], "peak_source": peak_note}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands, on a bounded sample
+# ---------------------------------------------------------------------------
+
+def cpu_oracle_prefill(rows: int):
+    """Oracle time for quantizing `rows` activation rows and their fp64 GEMM
+    against the whole pre-quantized weight (prefill workload, seed 3)."""
+    import numpy as np
+    import oracle
+    w = _gen("prefill")
+    wq = oracle.quantize(w["W"])                     # pre-quantized weights: untimed
+    xs = w["X"][:rows]
+    t0 = time.perf_counter()
+    xq = oracle.quantize(xs)
+    oracle.gemm_f64(xq, wq)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * rows * w["N"] * w["K"]
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": f"prefill workload: oracle quantize of {rows} of 4096 X rows + fp64 GEMM of "
+                      f"those rows against all 17408 pre-quantized W rows (K=5120), "
+                      f"{os.cpu_count()} threads"}
+
+
+def reference_arm(args):
+    """--impl reference: the CPU oracle timed on this host, K steps of a
+    bounded sample of the headline workload."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    w = _gen(args.workload if args.workload in ("prefill", "decode") else "prefill")
+    wq = oracle.quantize(w["W"])
+    rows = 2
+    times = []
+    for i in range(args.warmup + args.steps):
+        r0 = (i * rows) % w["M"]
+        t0 = time.perf_counter()
+        xq = oracle.quantize(w["X"][r0:r0 + rows])
+        oracle.gemm_f64(xq, wq)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    per_step = sum(times) / len(times)
+    flops = 2.0 * rows * w["N"] * w["K"]
+    v = flops / per_step / 1e12
+    line = {"impl": "reference", "metric": "NVFP4 GEMM TFLOPS (prefill)", "value": v,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
+            "config": {"workload": f"{w['name']} W4A4 linear, CPU oracle: each step quantizes "
+                                   f"{rows} X rows and runs their fp64 GEMM against all "
+                                   f"{w['N']} pre-quantized W rows (K={w['K']})"},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(),
+                             "kind": "oracle", "sample": f"{rows} X rows per step"},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def _build_library():
+    """Compile libnvfp4.so in-tree if it is missing or stale (nvcc)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_nvfp4_build", os.path.join(ROOT, "nvfp4_block_scaled_21_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="prefill")
+    ap.add_argument("--only", action="store_true", help="measure the headline workload only")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=64)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    world, rank, local = dist_setup(args)
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}; using {world}", file=sys.stderr)
+    import torch
+    torch.cuda.set_device(local)
+    _build_library()
+    import nvfp4_block_scaled_21_b200 as nv
+
+    peaks = load_peaks()
+    names = [args.workload] + ([] if args.only else [n for n in WORKLOADS if n != args.workload])
+    results = {}
+    head = None
+    for n in names:
+        wl = WORKLOADS[n](nv, torch)
+        is_head = n == args.workload
+        elapsed, kern_us, clocks = measure(wl, torch, args.steps, args.warmup, world, local,
+                                           sample_clocks=is_head)
+        sps = elapsed / args.steps
+        value = wl.value(sps) * world
+        e2e_steps = min(args.steps, 20)
+        e2e_elapsed = measure_e2e(wl, torch, e2e_steps, world)
+        e2e_value = wl.value(e2e_elapsed / e2e_steps) * world
+        res = {"metric": wl.metric, "value": round(value, 2), "unit": wl.unit,
+               "ms_per_step": round(sps * 1e3, 4), "config": wl.config,
+               "roofline": roofline(wl, kern_us, peaks),
+               "e2e": {"value": round(e2e_value, 3), "unit": wl.unit,
+                       "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h},
+               "gpu_launches": wl.launches * args.steps}
+        if is_head:
+            head = res
+            head["clocks"] = clocks
+        else:
+            results[n] = res
+        del wl
+        torch.cuda.empty_cache()
+
+    line = {"metric": head["metric"], "value": head["value"], "unit": head["unit"],
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4",
+            "data": "synthetic (seeded numpy PCG64: N(0,1) activations with 0.1% x50 outliers, "
+                    "N(0,0.02) weights, bf16)",
+            "config": dict(head["config"], parallelism=f"independent batch per GPU x{world}"),
+            "roofline": head["roofline"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+            "clocks": head["clocks"], "workloads": results,
+            "peaks": peaks}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "prefill":
+        line["cpu_baseline"] = cpu_oracle_prefill(args.cpu_rows)
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

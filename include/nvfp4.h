@@ -80,7 +80,8 @@ typedef enum {
     NVFP4_OP_QUANTIZE = 0,
     NVFP4_OP_DEQUANTIZE = 1,
     NVFP4_OP_GEMM = 2,
-    NVFP4_OP_LINEAR_FUSED = 3
+    NVFP4_OP_LINEAR_FUSED = 3,           /* nvfp4_linear_fused with NVFP4_EPI_STORE */
+    NVFP4_OP_LINEAR_FUSED_SILU = 4       /* nvfp4_linear_fused with NVFP4_EPI_SILU_MUL_REQUANT */
 } nvfp4_op;
 
 typedef enum {

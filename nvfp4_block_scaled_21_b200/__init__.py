@@ -26,7 +26,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_WORKSPACE, ERR_CUDA, \
     ERR_TIMEOUT, ERR_ARCH = range(8)
 F32, BF16 = 0, 1
-OP_QUANTIZE, OP_DEQUANTIZE, OP_GEMM, OP_LINEAR_FUSED = range(4)
+OP_QUANTIZE, OP_DEQUANTIZE, OP_GEMM, OP_LINEAR_FUSED, OP_LINEAR_FUSED_SILU = range(5)
 EPI_STORE, EPI_SILU_MUL_REQUANT = 0, 1
 
 EXPORTED = (

@@ -48,8 +48,10 @@ nvfp4_status current_device(DevInfo *out) {
 }
 
 nvfp4_status check_tensor(const nvfp4_tensor *t, int64_t rows, int64_t cols) {
-    if (!t || !t->codes || !t->scales || !t->tensor_scale) return NVFP4_ERR_INVALID_ARG;
+    if (!t || !t->tensor_scale) return NVFP4_ERR_INVALID_ARG;
     if (t->rows != rows || t->cols != cols || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+    // an empty tensor may have NULL codes and scales (nothing is read or written)
+    if (rows * cols != 0 && (!t->codes || !t->scales)) return NVFP4_ERR_INVALID_ARG;
     if (cols % kBlock) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(t->codes) || !aligned16(t->scales) || !aligned16(t->tensor_scale))
         return NVFP4_ERR_MISALIGNED;
@@ -102,12 +104,13 @@ size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K) {
     case NVFP4_OP_DEQUANTIZE:
     case NVFP4_OP_GEMM:
         return kWsStatusBytes;
-    case NVFP4_OP_LINEAR_FUSED: {
-        // partials | x_q (codes, scales, g) | gate, up, h (fp32 [M][N] each)
-        size_t b = kQuantizeWs + quantized_bytes(M, K);
-        b += 3 * align256(static_cast<size_t>(M * N) * sizeof(float));
-        return b;
-    }
+    case NVFP4_OP_LINEAR_FUSED:
+        // partials | x_q (codes, scales, g)
+        return kQuantizeWs + quantized_bytes(M, K);
+    case NVFP4_OP_LINEAR_FUSED_SILU:
+        // partials | x_q | gate, up, h (fp32 [M][N] each)
+        return kQuantizeWs + quantized_bytes(M, K) +
+               3 * align256(static_cast<size_t>(M * N) * sizeof(float));
     }
     return 0;
 }
@@ -115,7 +118,7 @@ size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K) {
 nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype xt, int64_t rows, int64_t cols, int64_t ld,
                             const nvfp4_tensor *out, void *ws, size_t ws_bytes,
                             nvfp4_stream_t stream) {
-    if (!x || (xt != NVFP4_F32 && xt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if ((!x && rows * cols != 0) || (xt != NVFP4_F32 && xt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
     if (rows < 0 || cols < 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
     nvfp4_status st = check_tensor(out, rows, cols);
     if (st != NVFP4_OK) return st;
@@ -212,8 +215,8 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
         if (y && (!aligned16(y) || (ldy * 4) % 16)) return NVFP4_ERR_MISALIGNED;
     }
     if (x_q && (st = check_tensor(x_q, M, K)) != NVFP4_OK) return st;
-    if ((st = check_ws(ws, ws_bytes, nvfp4_workspace_bytes(NVFP4_OP_LINEAR_FUSED, M, N, K))) != NVFP4_OK)
-        return st;
+    const nvfp4_op op = epilogue == NVFP4_EPI_STORE ? NVFP4_OP_LINEAR_FUSED : NVFP4_OP_LINEAR_FUSED_SILU;
+    if ((st = check_ws(ws, ws_bytes, nvfp4_workspace_bytes(op, M, N, K))) != NVFP4_OK) return st;
     DevInfo dev;
     if ((st = current_device(&dev)) != NVFP4_OK) return st;
     if (M == 0) return NVFP4_OK;

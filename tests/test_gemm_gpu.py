@@ -31,10 +31,15 @@ def quantize_gpu(nv, x):
 
 
 def run_gemm(nv, a, b, out_dtype):
-    y = torch.full((a.rows, b.rows), float("nan"), dtype=out_dtype, device="cuda")
+    # rows of y must start on 16-byte boundaries: pad the pitch, then slice
+    per16 = 16 // torch.empty((), dtype=out_dtype).element_size()
+    ldy = -(-b.rows // per16) * per16
+    buf = torch.full((a.rows, ldy), float("nan"), dtype=out_dtype, device="cuda")
+    y = buf[:, :b.rows]
     ws = nv.workspace(nv.OP_GEMM, a.rows, b.rows, a.cols)
     nv.nvfp4_gemm(a, b, y, ws)
     assert nv.nvfp4_get_device_status(ws) == nv.OK
+    assert torch.isnan(buf[:, b.rows:].float()).all()      # nothing written past N
     return y
 
 

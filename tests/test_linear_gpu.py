@@ -64,7 +64,7 @@ def check_mlp(nv, X, Wg, Wu, Wd, M, K, N):
     wg, wu, wd = (quantize_gpu(nv, bf16_tensor(a)) for a in (Wg, Wu, Wd))
     h = torch.empty((M, N), dtype=torch.float32, device="cuda")
     h_q = nv.NVFP4Tensor.empty(M, N)
-    ws = nv.workspace(nv.OP_LINEAR_FUSED, M, N, K)
+    ws = nv.workspace(nv.OP_LINEAR_FUSED_SILU, M, N, K)
     nv.nvfp4_linear_fused(bf16_tensor(X), wg, ws, nv.EPI_SILU_MUL_REQUANT, y=h, w_up=wu, y_q=h_q)
     y = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
     nv.nvfp4_gemm(h_q, wd, y, nv.workspace(nv.OP_GEMM, M, K, N))
