@@ -177,6 +177,37 @@ NVFP4_API nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t
                                 void *ws, size_t ws_bytes, nvfp4_stream_t stream);
 
 /*
+ * nvfp4_linear_noalloc: the same W4A4 linear layer as nvfp4_linear_fused with
+ * NVFP4_EPI_STORE (quantize x on the device, then y = x_q . w^T * gx * gw),
+ * for callers that cannot allocate device memory and so cannot pass a
+ * workspace: a plugin whose host framework's caching allocator owns every
+ * device byte and forbids raw cudaMalloc, a runtime whose memory plan is fixed
+ * before it runs, a latency-critical loop that must not risk the implicit
+ * device synchronisation of cudaMalloc/cudaFree, or a foreign-language caller
+ * that only holds pointers it was given.  The pages have no counterpart: this
+ * is an interface convenience, not part of the method.
+ *   Scratch: one 4 MiB file-scope __device__ array inside the library, held on
+ *   every GPU that loads the library until the process exits.  It carries the
+ *   status word, the quantizer's partial maxima and the quantized activations,
+ *   so M * K/2 + roundup(M,128) * roundup(K/16,4) must stay within about
+ *   4 MiB - 17 KiB (about 1.3k rows at K = 5120); larger shapes are rejected
+ *   with NVFP4_ERR_UNSUPPORTED_SHAPE and nothing is launched.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Every call shares the one array and finds the previous call's contents in
+ *   it: calls that overlap on the GPU race on it.  Each call clears the status
+ *   word first and rewrites everything else.  Device-side waits give up after
+ *   2 s; there is no status readback for this entry point (use
+ *   nvfp4_linear_fused with a workspace to observe one).
+ *   Other arguments, layouts and errors as nvfp4_linear_fused; allocates
+ *   nothing (no cudaMalloc, cudaFree or allocating library routine).
+ */
+NVFP4_API nvfp4_status nvfp4_linear_noalloc(const void *x, nvfp4_dtype xt, int64_t M, int64_t K,
+                                            int64_t ldx, const nvfp4_tensor *w, void *y,
+                                            nvfp4_dtype yt, int64_t ldy, nvfp4_stream_t stream);
+
+/*
  * Synchronise `stream`, read the sticky device status word in ws, clear it,
  * and return it (NVFP4_OK when no device-side wait gave up since the last
  * read).  Also returns NVFP4_ERR_CUDA if the stream reports an error.

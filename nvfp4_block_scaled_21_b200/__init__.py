@@ -33,7 +33,7 @@ EXPORTED = (
     "nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize",
     "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_linear_fused", "nvfp4_get_device_status",
     "nvfp4_selftest_bounded_wait", "nvfp4_set_wait_timeout_us", "nvfp4_status_string",
-    "nvfp4_version",
+    "nvfp4_version", "nvfp4_linear_noalloc",
 )
 
 
@@ -62,6 +62,8 @@ _lib.nvfp4_gemm.restype = _I
 _lib.nvfp4_linear_fused.argtypes = [_P, _I, _I64, _I64, _I64, _T, _T, _I, _P, _I, _I64, _T, _T,
                                     _P, _SZ, _P]
 _lib.nvfp4_linear_fused.restype = _I
+_lib.nvfp4_linear_noalloc.argtypes = [_P, _I, _I64, _I64, _I64, _T, _P, _I, _I64, _P]
+_lib.nvfp4_linear_noalloc.restype = _I
 _lib.nvfp4_get_device_status.argtypes = [_P, _P]
 _lib.nvfp4_get_device_status.restype = _I
 _lib.nvfp4_selftest_bounded_wait.argtypes = [_P, ctypes.c_uint32, _P]
@@ -214,6 +216,20 @@ def nvfp4_linear_fused(x, w: NVFP4Tensor, ws, epilogue: int = EPI_STORE, y=None,
         ctypes.byref(cxq) if cxq is not None else None, ws.data_ptr(), ws.numel(),
         _stream(stream))
     _check(st, "nvfp4_linear_fused")
+    return y
+
+
+def nvfp4_linear_noalloc(x, w: NVFP4Tensor, y, stream=None):
+    """W4A4 linear layer (quantize x, GEMM with w) using the library's own
+    static scratch instead of a caller workspace; for callers that cannot
+    allocate device memory.  See nvfp4_linear_noalloc in nvfp4.h for the size
+    limit and the rule that calls must not overlap on the GPU."""
+    assert x.dim() == 2 and x.stride(1) == 1 and y.dim() == 2 and y.stride(1) == 1
+    cw = w.c()
+    st = _lib.nvfp4_linear_noalloc(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1],
+                                   x.stride(0), ctypes.byref(cw), y.data_ptr(), _dtype_code(y),
+                                   y.stride(0), _stream(stream))
+    _check(st, "nvfp4_linear_noalloc")
     return y
 
 
