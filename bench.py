@@ -8,7 +8,8 @@ MLP step.  Prints ONE JSON line (rank 0).
 
 A step is one pass of the hot path over one batch of synthetic input already
 resident in HBM.  The headline workload (default: prefill, M=4096 N=17408
-K=5120) is timed over exactly K steps bracketed by a barrier and a device
+K=5120) is timed over exactly K steps (CUDA-graph replays, one step each)
+bracketed by a barrier and a device
 synchronize; the other workloads are measured the same way and reported under
 "workloads".  L2 (126 MB) is defeated by rotating enough input copies that
 each step's operands were evicted by the steps before it.  Multi-GPU runs are
@@ -110,26 +111,6 @@ class ClockSampler:
 # workloads
 # ---------------------------------------------------------------------------
 
-class Timer:
-    """CUDA events around one kernel inside each step, on the launching stream."""
-
-    def __init__(self, torch, n):
-        self.ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(n)]
-        self.i = 0
-
-    def begin(self):
-        self.ev[self.i][0].record()
-
-    def end(self):
-        self.ev[self.i][1].record()
-        self.i += 1
-
-    def mean_us(self):
-        ts = [a.elapsed_time(b) * 1e3 for a, b in self.ev[:self.i]]
-        return sum(ts) / len(ts) if ts else float("nan")
-
-
 def _copies(t, n):
     return [t] + [t.clone() for _ in range(n - 1)]
 
@@ -184,12 +165,14 @@ class Prefill:
                        "M": self.M, "N": self.N, "K": self.K,
                        "l2": f"{self.R} rotating copies of X and W_q ({self.R * per_step / 2**20:.0f} MiB) > 126 MB L2"}
 
-    def step(self, i, timer=None):
+    def step(self, i):
         r = i % self.R
         self.nv.nvfp4_quantize(self.X[r], self.xq[r], self.wsq)
-        if timer: timer.begin()
         self.nv.nvfp4_gemm(self.xq[r], self.Wq[r], self.y, self.wsg)
-        if timer: timer.end()
+
+    def dominant_call(self, i):
+        r = i % self.R
+        self.nv.nvfp4_gemm(self.xq[r], self.Wq[r], self.y, self.wsg)
 
     def e2e_setup(self):
         self.x_host = self.X[0].cpu().pin_memory()
@@ -255,11 +238,11 @@ class Quantize:
                        "two_pass_bytes_per_step": self.bytes_two_pass,
                        "l2": f"{self.R} rotating copies of x ({self.R * n * 2 / 2**20:.0f} MiB) > 126 MB L2"}
 
-    def step(self, i, timer=None):
+    def step(self, i):
         r = i % self.R
-        if timer: timer.begin()
         self.nv.nvfp4_quantize(self.X[r], self.q[r], self.ws)
-        if timer: timer.end()
+
+    dominant_call = step
 
     def e2e_setup(self):
         self.x_host = self.X[0].cpu().pin_memory()
@@ -314,14 +297,16 @@ class Mlp:
                        "flops_per_step": 2.0 * M * N * K * 3,
                        "l2": f"{self.R} rotating copies of the three weight matrices > 126 MB L2"}
 
-    def step(self, i, timer=None):
+    def step(self, i):
         r = i % self.R
         nv = self.nv
         nv.nvfp4_linear_fused(self.X[r], self.wg[r], self.wsl, nv.EPI_SILU_MUL_REQUANT,
                               w_up=self.wu[r], y_q=self.hq)
-        if timer: timer.begin()
         nv.nvfp4_gemm(self.hq, self.wd[r], self.y, self.wsg)
-        if timer: timer.end()
+
+    def dominant_call(self, i):
+        r = i % self.R
+        self.nv.nvfp4_gemm(self.hq, self.wd[r], self.y, self.wsg)
 
     def e2e_setup(self):
         self.x_host = self.X[0].cpu().pin_memory()
@@ -380,26 +365,54 @@ def max_over_ranks(world, value):
     return float(t.item())
 
 
+def _capture(torch, fn, n):
+    """One CUDA graph per rotation slot, each holding one call of fn(slot)."""
+    graphs = []
+    for r in range(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn(r)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    return graphs
+
+
 def measure(wl, torch, K, W, world, local, sample_clocks=False):
-    for i in range(W):
+    """Device time of exactly K steps (CUDA-graph replays, one step per
+    replay, rotating input slots), bracketed by barrier + synchronize; then the
+    dominant kernel alone over K launches on the same slots."""
+    for i in range(W):                       # eager warm-up (also resolves lazy set-up)
         wl.step(i)
+    torch.cuda.synchronize()
+    steps = _capture(torch, wl.step, wl.R)
+    kern = _capture(torch, wl.dominant_call, wl.R)
+    for i in range(W):
+        steps[i % wl.R].replay()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    timer = Timer(torch, K)
     sampler = ClockSampler(local) if sample_clocks else None
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ctx = sampler if sampler else _Null()
-    with ctx:
+    with (sampler if sampler else _Null()):
         start.record()
         for i in range(K):
-            wl.step(W + i, timer)
+            steps[(W + i) % wl.R].replay()
         end.record()
         torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     elapsed = max_over_ranks(world, start.elapsed_time(end) / 1e3)
-    kern_us = max_over_ranks(world, timer.mean_us())
+    for i in range(W):
+        kern[i % wl.R].replay()
+    torch.cuda.synchronize()
+    ks, ke = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ks.record()
+    for i in range(K):
+        kern[(W + i) % wl.R].replay()
+    ke.record()
+    torch.cuda.synchronize()
+    kern_us = max_over_ranks(world, ks.elapsed_time(ke) * 1e3 / K)
+    del steps, kern
     return elapsed, kern_us, (sampler.summary() if sampler else None)
 
 
