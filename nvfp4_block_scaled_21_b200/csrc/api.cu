@@ -164,9 +164,12 @@ static nvfp4_status check_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, voi
     return NVFP4_OK;
 }
 
+// weights_ready: b was not written by the kernel launched just before (true
+// inside nvfp4_linear_fused, whose first kernel is launched without a
+// programmatic dependency, so every earlier writer of b has finished).
 static nvfp4_status gemm_impl(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y,
                               nvfp4_dtype yt, int64_t ldy, uint32_t *status, int num_sms,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, bool weights_ready = false) {
     if (a->rows == 0 || b->rows == 0) return NVFP4_OK;
     if (a->cols == 0)   // empty reduction: y = 0
         return from_cuda(cudaMemset2DAsync(y, ldy * (yt == NVFP4_BF16 ? 2 : 4), 0,
@@ -174,7 +177,7 @@ static nvfp4_status gemm_impl(const nvfp4_tensor *a, const nvfp4_tensor *b, void
     Operand act{a->codes, a->scales, a->tensor_scale, a->rows};
     Operand wgt{b->codes, b->scales, b->tensor_scale, b->rows};
     return from_cuda(launch_gemm(act, wgt, a->cols, y, yt == NVFP4_BF16, ldy, status, timeout_ns(),
-                                 num_sms, stream));
+                                 num_sms, stream, weights_ready));
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y, nvfp4_dtype yt,
@@ -243,7 +246,7 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     uint32_t *status = static_cast<uint32_t *>(ws);
     if (epilogue == NVFP4_EPI_STORE)
-        return gemm_impl(&xq, w, y, yt, ldy, status, dev.sms, stream);
+        return gemm_impl(&xq, w, y, yt, ldy, status, dev.sms, stream, true);
 
     // SiLU(gate) * up, then re-quantize h for the down projection.
     const size_t mn = align256(static_cast<size_t>(M * N) * sizeof(float));
@@ -251,8 +254,8 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
     float *up = reinterpret_cast<float *>(ws_at(ws, off + mn));
     float *h = y ? static_cast<float *>(y) : reinterpret_cast<float *>(ws_at(ws, off + 2 * mn));
     const int64_t ldh = y ? ldy : N;
-    if ((st = gemm_impl(&xq, w, gate, NVFP4_F32, N, status, dev.sms, stream)) != NVFP4_OK) return st;
-    if ((st = gemm_impl(&xq, w_up, up, NVFP4_F32, N, status, dev.sms, stream)) != NVFP4_OK) return st;
+    if ((st = gemm_impl(&xq, w, gate, NVFP4_F32, N, status, dev.sms, stream, true)) != NVFP4_OK) return st;
+    if ((st = gemm_impl(&xq, w_up, up, NVFP4_F32, N, status, dev.sms, stream, true)) != NVFP4_OK) return st;
     if (ldh == N) {
         if (launch_silu_mul(gate, up, h, M * N, dev.sms, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
     } else {

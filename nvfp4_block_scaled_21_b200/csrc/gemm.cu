@@ -7,19 +7,30 @@
 // scales are applied once in the epilogue (NVFP4 wiki page, section "技術原理":
 // a second-level FP32 scale over the whole tensor).
 //
-// Design (one persistent CTA per SM, 6 warps):
+// Design (one persistent CTA per SM, 10 warps):
 //   warp 0      TMA producer: for every 256-element K slab, a 128-row tile of
 //               the MMA's A operand and a BN-row tile of its B operand (packed
 //               E2M1, 128-byte swizzle) plus their 512-byte scale atoms (bulk
 //               copies) into a STAGES-deep shared-memory ring (mbarriers).
-//   warp 1      TMEM allocator and MMA issuer: copies the scale atoms into
-//               tensor memory (tcgen05.cp 32x128b, replicated to the 4 lane
-//               quarters) and issues tcgen05.mma kind::mxf4nvf4 (M=128,
-//               N=BN, K=64) into an fp32 accumulator in tensor memory.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator, y = acc * (gA*gB),
-//               RNE to bf16 (or fp32), and the store.
+//   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::mxf4nvf4
+//               (M=128, N=BN, K=64) into an fp32 accumulator in tensor memory;
+//               a stage is released by tcgen05.commit when its MMAs are done.
+//   warps 2..5  scale warps: each copies the stage's scale atoms from shared
+//               memory into its own 32-lane quarter of tensor memory with
+//               tcgen05.st (the four quarters hold the same scales, which is the
+//               replicated layout the block-scaled MMA reads), into a TMEM scale
+//               slot owned by the stage.  This keeps scale movement off the
+//               tensor pipe, where a tcgen05.cp per 512-byte atom would cost
+//               about as much tensor-pipe time as the MMAs themselves.
+//   warps 6..9  epilogue: tcgen05.ld of the accumulator (next chunk in flight
+//               while the current one is stored), y = acc * (gA*gB), RNE to
+//               bf16 (or fp32), and the store.
 // Small M (decode) runs "swapped": the weights ride the MMA's M = 128 and the
 // few activation rows ride N = BN, so the weight stream spreads over all SMs.
+// When the weights are known not to come from the kernel launched just before
+// (inside nvfp4_linear_fused), the producer starts streaming them before the
+// programmatic-dependent-launch wait, hiding the pipeline fill behind the
+// activation quantizer.
 // Every wait is bounded; a timeout sets the status word and winds the CTA
 // down without leaving tensor memory allocated.
 #include "common.cuh"
@@ -39,6 +50,8 @@ struct GemmArgs {
     int32_t num_k_steps;     // K / 64
     int32_t num_p_tiles, num_q_tiles;
     int32_t q_row_tiles;     // ceil(Q / 128): 128-row scale tiles of B
+    int32_t preload;         // stages of the weight operand loaded before the PDL wait
+    int32_t weights_are_a;   // 1: the weights are the MMA A operand (swapped)
     uint32_t *status;
     uint64_t timeout_ns;
 };
@@ -52,21 +65,22 @@ struct GemmCfg {
     static constexpr int kSfbStage = kNQT * 4 * 512;
     static constexpr int kStageBytes = kAStage + kBStage + kSfaStage + kSfbStage;
     static constexpr int kStages = (BN == 256) ? 4 : (BN == 128 ? 6 : (BN == 64 ? 7 : 8));
-    static constexpr int kSfCols = 16 + 16 * kNQT;             // TMEM columns for scales
-    static constexpr int kAccStages = (2 * BN + kSfCols <= 512) ? 2 : 1;
-    static constexpr int kSfaCol = kAccStages * BN;
-    static constexpr int kSfbCol = kSfaCol + 16;
-    static constexpr int kColsUsed = kSfbCol + 16 * kNQT;
+    static constexpr int kSfCols = 16 + 16 * kNQT;             // TMEM scale columns per stage
+    static constexpr int kAccStages = (2 * BN + kStages * kSfCols <= 512) ? 2 : 1;
+    static constexpr int kSfBase = kAccStages * BN;            // first scale column
+    static constexpr int kColsUsed = kSfBase + kStages * kSfCols;
     static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
-    static constexpr int kBarBytes = 8 * (2 * kStages + 4) + 16;
+    static constexpr int kBarBytes = 8 * (3 * kStages + 4) + 16;
     static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;   // + alignment slack
+    static constexpr int kThreads = 320;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kColsUsed <= 512, "tensor memory budget");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
 };
 
 template <int BN, bool SWAP, typename OutT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ GemmArgs args) {
     using C = GemmCfg<BN>;
@@ -78,7 +92,8 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     uint8_t *sSfa = sB + STAGES * C::kBStage;
     uint8_t *sSfb = sSfa + STAGES * C::kSfaStage;
     uint64_t *full = reinterpret_cast<uint64_t *>(sSfb + STAGES * C::kSfbStage);
-    uint64_t *empty = full + STAGES;
+    uint64_t *sf_full = full + STAGES;
+    uint64_t *empty = sf_full + STAGES;
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tempty + 2);
@@ -92,6 +107,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         prefetch_tensormap(&tmB);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&sf_full[s], 128);
             mbar_init(&empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -107,97 +123,190 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
-    // Operands may come from the kernel launched just before (the quantizer).
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-
     const int num_tiles = args.num_p_tiles * args.num_q_tiles;
     const int num_kstages = (args.num_k_steps + 3) / 4;
 
-    if (warp == 0 && lane == 0) {
-        // ------------------------------------------------------------ producer
-        const uint64_t pol_a = SWAP ? policy_evict_first() : policy_evict_normal();
-        const uint64_t pol_b = SWAP ? policy_evict_last() : policy_evict_normal();
-        uint32_t stage = 0, phase = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            const int pt = tile % args.num_p_tiles;
-            const int qt = tile / args.num_p_tiles;
-            bool ok = true;
-            for (int ks = 0; ks < num_kstages; ++ks) {
-                if (!mbar_wait(&empty[stage], phase ^ 1u, args.timeout_ns, abort_flag, args.status)) {
-                    ok = false;
-                    break;
-                }
-                const int nk = min(4, args.num_k_steps - 4 * ks);
+    if (warp == 0) {
+        if (lane == 0) {
+            // -------------------------------------------------------- producer
+            const uint64_t pol_a = SWAP ? policy_evict_first() : policy_evict_normal();
+            const uint64_t pol_b = SWAP ? policy_evict_last() : policy_evict_normal();
+            // The weights may be streamed before the dependent-launch wait for
+            // the first `pre` stages of this CTA's first tile.
+            const int pre = (static_cast<int>(blockIdx.x) < num_tiles) ? min(args.preload, min(STAGES, num_kstages)) : 0;
+            uint32_t stage = 0, phase = 0;
+            bool waited = (pre == 0);
+            if (waited) asm volatile("griddepcontrol.wait;" ::: "memory");
+            int it = 0;   // stage index within this CTA's work
+            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+                const int pt = tile % args.num_p_tiles;
+                const int qt = tile / args.num_p_tiles;
+                bool ok = true;
                 int nq_loaded = 0;
                 for (int q = 0; q < C::kNQT; ++q) nq_loaded += (qt * C::kNQT + q < args.q_row_tiles);
-                const uint32_t bytes = C::kAStage + C::kBStage + nk * 512 * (1 + nq_loaded);
-                mbar_arrive_expect_tx(&full[stage], bytes);
-                tma_load_2d(sA + stage * C::kAStage, &tmA, &full[stage], ks * 128, pt * 128, pol_a);
-                tma_load_2d(sB + stage * C::kBStage, &tmB, &full[stage], ks * 128, qt * BN, pol_b);
-                bulk_load(sSfa + stage * C::kSfaStage,
-                          args.sfa + (static_cast<int64_t>(pt) * args.num_k_steps + 4 * ks) * 512,
-                          nk * 512, &full[stage], pol_a);
-                for (int q = 0; q < C::kNQT; ++q) {
-                    const int rt = qt * C::kNQT + q;
-                    if (rt < args.q_row_tiles)
-                        bulk_load(sSfb + stage * C::kSfbStage + q * 2048,
-                                  args.sfb + (static_cast<int64_t>(rt) * args.num_k_steps + 4 * ks) * 512,
-                                  nk * 512, &full[stage], pol_b);
+                for (int ks = 0; ks < num_kstages; ++ks, ++it) {
+                    const int nk = min(4, args.num_k_steps - 4 * ks);
+                    const uint32_t bytes = C::kAStage + C::kBStage + nk * 512 * (1 + nq_loaded);
+                    auto load_a = [&]() {
+                        tma_load_2d(sA + stage * C::kAStage, &tmA, &full[stage], ks * 128, pt * 128, pol_a);
+                        bulk_load(sSfa + stage * C::kSfaStage,
+                                  args.sfa + (static_cast<int64_t>(pt) * args.num_k_steps + 4 * ks) * 512,
+                                  nk * 512, &full[stage], pol_a);
+                    };
+                    auto load_b = [&]() {
+                        tma_load_2d(sB + stage * C::kBStage, &tmB, &full[stage], ks * 128, qt * BN, pol_b);
+                        for (int q = 0; q < C::kNQT; ++q) {
+                            const int rt = qt * C::kNQT + q;
+                            if (rt < args.q_row_tiles)
+                                bulk_load(sSfb + stage * C::kSfbStage + q * 2048,
+                                          args.sfb + (static_cast<int64_t>(rt) * args.num_k_steps + 4 * ks) * 512,
+                                          nk * 512, &full[stage], pol_b);
+                        }
+                    };
+                    if (it < pre) {
+                        // fresh stage (first pass over the ring): no empty wait needed
+                        mbar_arrive_expect_tx(&full[stage], bytes);
+                        if (args.weights_are_a) load_a(); else load_b();
+                    } else {
+                        if (!waited) {
+                            // finish the preloaded stages with the dependent operand
+                            asm volatile("griddepcontrol.wait;" ::: "memory");
+                            waited = true;
+                            for (int p = 0; p < pre; ++p) {
+                                // the preloaded stages are stages 0..pre-1 of the first tile
+                                const int ks0 = p;
+                                const int nk0 = min(4, args.num_k_steps - 4 * ks0);
+                                const int pt0 = static_cast<int>(blockIdx.x) % args.num_p_tiles;
+                                const int qt0 = static_cast<int>(blockIdx.x) / args.num_p_tiles;
+                                if (args.weights_are_a) {
+                                    tma_load_2d(sB + p * C::kBStage, &tmB, &full[p], ks0 * 128, qt0 * BN, pol_b);
+                                    for (int q = 0; q < C::kNQT; ++q) {
+                                        const int rt = qt0 * C::kNQT + q;
+                                        if (rt < args.q_row_tiles)
+                                            bulk_load(sSfb + p * C::kSfbStage + q * 2048,
+                                                      args.sfb + (static_cast<int64_t>(rt) * args.num_k_steps + 4 * ks0) * 512,
+                                                      nk0 * 512, &full[p], pol_b);
+                                    }
+                                } else {
+                                    tma_load_2d(sA + p * C::kAStage, &tmA, &full[p], ks0 * 128, pt0 * 128, pol_a);
+                                    bulk_load(sSfa + p * C::kSfaStage,
+                                              args.sfa + (static_cast<int64_t>(pt0) * args.num_k_steps + 4 * ks0) * 512,
+                                              nk0 * 512, &full[p], pol_a);
+                                }
+                            }
+                        }
+                        if (!mbar_wait(&empty[stage], phase ^ 1u, args.timeout_ns, abort_flag, args.status)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&full[stage], bytes);
+                        load_a();
+                        load_b();
+                    }
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                if (!ok) break;
             }
-            if (!ok) break;
+            if (!waited) {
+                // everything fit in the preload: issue the dependent halves now
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                for (int p = 0; p < pre; ++p) {
+                    const int nk0 = min(4, args.num_k_steps - 4 * p);
+                    const int pt0 = static_cast<int>(blockIdx.x) % args.num_p_tiles;
+                    const int qt0 = static_cast<int>(blockIdx.x) / args.num_p_tiles;
+                    if (args.weights_are_a) {
+                        tma_load_2d(sB + p * C::kBStage, &tmB, &full[p], p * 128, qt0 * BN, pol_b);
+                        for (int q = 0; q < C::kNQT; ++q) {
+                            const int rt = qt0 * C::kNQT + q;
+                            if (rt < args.q_row_tiles)
+                                bulk_load(sSfb + p * C::kSfbStage + q * 2048,
+                                          args.sfb + (static_cast<int64_t>(rt) * args.num_k_steps + 4 * p) * 512,
+                                          nk0 * 512, &full[p], pol_b);
+                        }
+                    } else {
+                        tma_load_2d(sA + p * C::kAStage, &tmA, &full[p], p * 128, pt0 * 128, pol_a);
+                        bulk_load(sSfa + p * C::kSfaStage,
+                                  args.sfa + (static_cast<int64_t>(pt0) * args.num_k_steps + 4 * p) * 512,
+                                  nk0 * 512, &full[p], pol_a);
+                    }
+                }
+            }
         }
-    } else if (warp == 1 && lane == 0) {
-        // ------------------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = make_idesc_nvf4(BN);
-        const uint32_t a_base = smem_addr(sA), b_base = smem_addr(sB);
-        const uint32_t sfa_base = smem_addr(sSfa), sfb_base = smem_addr(sSfb);
-        uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // -------------------------------------------------------- MMA issuer
+            constexpr uint32_t idesc = make_idesc_nvf4(BN);
+            const uint32_t a_base = smem_addr(sA), b_base = smem_addr(sB);
+            uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.timeout_ns, abort_flag, args.status)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                bool ok = true;
+                for (int ks = 0; ks < num_kstages; ++ks) {
+                    if (!mbar_wait(&full[stage], phase, args.timeout_ns, abort_flag, args.status) ||
+                        !mbar_wait(&sf_full[stage], phase, args.timeout_ns, abort_flag, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nk = min(4, args.num_k_steps - 4 * ks);
+                    const uint32_t sf = tmem_base + C::kSfBase + stage * C::kSfCols;
+                    for (int j = 0; j < nk; ++j) {
+                        const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage + 32 * j);
+                        const uint64_t bdesc = make_operand_desc(b_base + stage * C::kBStage + 32 * j);
+                        mma_nvf4(d_tmem, adesc, bdesc, idesc, sf + 4 * j, sf + 16 + 4 * C::kNQT * j,
+                                 (ks | j) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(&tfull[acc]);
+                if (C::kAccStages == 2) {
+                    acc ^= 1u;
+                    if (acc == 0) acc_phase ^= 1u;
+                } else {
+                    acc_phase ^= 1u;
+                }
+            }
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ scale warps
+        // Lane l of every quarter receives the 16 bytes at l*16 of each 512-byte
+        // atom: columns c = 0..3 hold rows 32c + l, bytes = the 4 K-blocks.
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        uint32_t stage = 0, phase = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.timeout_ns, abort_flag, args.status)) break;
-            tc_fence_after();
-            const uint32_t d_tmem = tmem_base + acc * BN;
             bool ok = true;
             for (int ks = 0; ks < num_kstages; ++ks) {
-                if (!mbar_wait(&full[stage], phase, args.timeout_ns, abort_flag, args.status)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
+                const bool got = mbar_wait(&full[stage], phase, args.timeout_ns, abort_flag, args.status);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 const int nk = min(4, args.num_k_steps - 4 * ks);
+                const uint32_t sf = tmem_base + lane_off + C::kSfBase + stage * C::kSfCols;
+                const uint8_t *a_src = sSfa + stage * C::kSfaStage + lane * 16;
+                const uint8_t *b_src = sSfb + stage * C::kSfbStage + lane * 16;
                 for (int j = 0; j < nk; ++j) {
-                    tc_cp_32x128b_warpx4(tmem_base + C::kSfaCol + 4 * j,
-                                         make_sf_desc(sfa_base + stage * C::kSfaStage + j * 512));
+                    tmem_st_32x32b_x4(sf + 4 * j, ld_shared_v4(a_src + j * 512));
 #pragma unroll
                     for (int q = 0; q < C::kNQT; ++q)
-                        tc_cp_32x128b_warpx4(tmem_base + C::kSfbCol + 4 * (j * C::kNQT + q),
-                                             make_sf_desc(sfb_base + stage * C::kSfbStage + q * 2048 + j * 512));
+                        tmem_st_32x32b_x4(sf + 16 + 4 * (j * C::kNQT + q), ld_shared_v4(b_src + q * 2048 + j * 512));
                 }
-                for (int j = 0; j < nk; ++j) {
-                    const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage + 32 * j);
-                    const uint64_t bdesc = make_operand_desc(b_base + stage * C::kBStage + 32 * j);
-                    mma_nvf4(d_tmem, adesc, bdesc, idesc, tmem_base + C::kSfaCol + 4 * j,
-                             tmem_base + C::kSfbCol + 4 * C::kNQT * j, (ks | j) != 0 ? 1u : 0u);
-                }
-                tc_commit(&empty[stage]);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&sf_full[stage]);
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
-            tc_commit(&tfull[acc]);
-            if (C::kAccStages == 2) {
-                acc ^= 1u;
-                if (acc == 0) acc_phase ^= 1u;
-            } else {
-                acc_phase ^= 1u;
-            }
         }
-    } else if (warp >= 2) {
+    } else {
         // ------------------------------------------------------------ epilogue
+        asm volatile("griddepcontrol.wait;" ::: "memory");   // tensor scales may be fresh
         const int quarter = warp & 3;               // TMEM lane quarter this warp may read
         const int row = quarter * 32 + lane;        // accumulator row (MMA M index)
         const float alpha = __fmul_rn(*args.ga, *args.gb);
         constexpr int CH = BN < 32 ? BN : 32;
+        constexpr int NCH = BN / CH;
         uint32_t acc = 0, acc_phase = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             const int pt = tile % args.num_p_tiles;
@@ -207,19 +316,23 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const int p = pt * 128 + row;
-#pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += CH) {
-                uint32_t r[CH];
-                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN + c0;
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
+            uint32_t r[2][CH];
+            auto ld = [&](int c, uint32_t (&dst)[CH]) {
                 if constexpr (CH == 32)
-                    tmem_ld_32x32b_x32(taddr, reinterpret_cast<uint32_t(&)[32]>(r));
+                    tmem_ld_32x32b_x32(tbase + c * CH, reinterpret_cast<uint32_t(&)[32]>(dst));
                 else
-                    tmem_ld_32x32b_x16(taddr, reinterpret_cast<uint32_t(&)[16]>(r));
-                tmem_ld_wait();
+                    tmem_ld_32x32b_x16(tbase + c * CH, reinterpret_cast<uint32_t(&)[16]>(dst));
+            };
+            ld(0, r[0]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+                if (c + 1 < NCH) ld(c + 1, r[(c + 1) & 1]);       // next chunk in flight
                 float v[CH];
 #pragma unroll
-                for (int i = 0; i < CH; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
-                const int q0 = qt * BN + c0;
+                for (int i = 0; i < CH; ++i) v[i] = __fmul_rn(__uint_as_float(r[c & 1][i]), alpha);
+                const int q0 = qt * BN + c * CH;
                 if constexpr (SWAP) {
                     // y[q][p]: for each i the warp writes 32 consecutive p
                     if (p < args.P) {
@@ -271,6 +384,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         }
                     }
                 }
+                if (c + 1 < NCH) tmem_ld_wait();
             }
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
@@ -328,7 +442,8 @@ CUresult encode_tensor_map_u8(CUtensorMap *map, const void *base, uint64_t inner
 
 template <int BN, bool SWAP, typename OutT>
 static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, void *y, int64_t ldy,
-                            uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t stream) {
+                            uint32_t *status, uint64_t timeout_ns, int num_sms, int preload,
+                            cudaStream_t stream) {
     using C = GemmCfg<BN>;
     CUtensorMap tmA, tmB;
     if (encode_tensor_map_u8(&tmA, pa.codes, K / 2, pa.rows, 128, 128) != CUDA_SUCCESS ||
@@ -347,6 +462,8 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     a.num_p_tiles = static_cast<int32_t>(ceil_div(pa.rows, 128));
     a.num_q_tiles = static_cast<int32_t>(ceil_div(qb.rows, BN));
     a.q_row_tiles = static_cast<int32_t>(ceil_div(qb.rows, 128));
+    a.preload = preload;
+    a.weights_are_a = SWAP ? 1 : 0;
     a.status = status;
     a.timeout_ns = timeout_ns;
     const int tiles = a.num_p_tiles * a.num_q_tiles;
@@ -355,7 +472,7 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles < num_sms ? tiles : num_sms);
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -368,14 +485,17 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
 
 cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
                         int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, bool weights_ready) {
+    // weights_ready: the weights were not written by the kernel launched just
+    // before this one, so they may be streamed before the dependent-launch wait.
+    const int preload = weights_ready ? 8 : 0;
     const int64_t M = act.rows, N = wgt.rows;
     if (M <= 64) {
         // weights on the MMA's M side, activations on N; y[m][n] = acc[n][m]
         const int bn = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
 #define NVFP4_SWAPPED(BNV)                                                                          \
-    return y_bf16 ? run_gemm<BNV, true, __nv_bfloat16>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, stream) \
-                  : run_gemm<BNV, true, float>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, stream);
+    return y_bf16 ? run_gemm<BNV, true, __nv_bfloat16>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, stream) \
+                  : run_gemm<BNV, true, float>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, stream);
         if (bn == 16) { NVFP4_SWAPPED(16) }
         if (bn == 32) { NVFP4_SWAPPED(32) }
         NVFP4_SWAPPED(64)
@@ -384,10 +504,10 @@ cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void 
     const int64_t ptiles = ceil_div(M, 128);
     const bool wide = ptiles * ceil_div(N, 256) >= 2 * num_sms;
     if (wide)
-        return y_bf16 ? run_gemm<256, false, __nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, stream)
-                      : run_gemm<256, false, float>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, stream);
-    return y_bf16 ? run_gemm<128, false, __nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, stream)
-                  : run_gemm<128, false, float>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, stream);
+        return y_bf16 ? run_gemm<256, false, __nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, stream)
+                      : run_gemm<256, false, float>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, stream);
+    return y_bf16 ? run_gemm<128, false, __nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, stream)
+                  : run_gemm<128, false, float>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, stream);
 }
 
 // ---------------------------------------------------------------------------

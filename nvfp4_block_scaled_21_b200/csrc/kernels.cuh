@@ -24,9 +24,11 @@ struct Operand {
 };
 
 // y[M][N] = (A . B^T) * gA * gB, A = act [M][K], B = wgt [N][K].
+// weights_ready: the weights were not written by the kernel launched just
+// before (they may be streamed before the programmatic-dependent-launch wait).
 cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
                         int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
-                        cudaStream_t stream);
+                        cudaStream_t stream, bool weights_ready = false);
 
 // h = SiLU(gate) * up elementwise in fp32 (n values).
 cudaError_t launch_silu_mul(const float *gate, const float *up, float *h, int64_t n, int num_sms,

@@ -10,10 +10,9 @@
 // Pass 2 (encode_kernel): every CTA reduces the partial maxima (a few KB from
 //   L2), derives g = amax/2688 on the device, and encodes the tensor, walking
 //   the windows in the reverse order of pass 1 so that the tail pass 1 read
-//   last is still in L2.  A 16-element block is held by 2 (bf16) or 4 (fp32)
-//   adjacent lanes; its amax is one or two shuffles; the E4M3 scale and the
-//   E2M1 codes come from the hardware RNE-satfinite conversions; codes go out
-//   as coalesced 32-bit (bf16) or 16-bit (fp32) stores and scales as one
+//   last is still in L2.  One thread owns one 16-element block; the E4M3
+//   scale and the E2M1 codes come from the hardware RNE-satfinite
+//   conversions; codes go out as one 8-byte store per block and scales as one
 //   32-bit word per four blocks in the tiled layout the tensor cores read.
 #include "common.cuh"
 #include "kernels.cuh"
@@ -129,47 +128,6 @@ __device__ __forceinline__ float e4m3_value(uint32_t s) {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xffffu)));
 }
 
-// Four bytes of packed E2M1 codes from eight values: element 2k in the low
-// nibble of byte k, element 2k+1 in the high nibble.
-__device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
-    uint32_t out;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-        : "=r"(out)
-        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
-    return out;
-}
-__device__ __forceinline__ uint32_t e2m1x4(const float (&v)[4]) {
-    uint32_t out;
-    asm("{\n\t.reg .b8 b0, b1;\n\t.reg .b16 h;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "mov.b16 h, {b0, b1};\n\t"
-        "cvt.u32.u16 %0, h;\n\t}"
-        : "=r"(out)
-        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]));
-    return out;
-}
-
-__device__ __forceinline__ void unpack(const uint4 &v, float (&x)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        x[2 * k] = __uint_as_float(w[k] << 16);
-        x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-    }
-}
-__device__ __forceinline__ void unpack(const uint4 &v, float (&x)[4]) {
-    x[0] = __uint_as_float(v.x);
-    x[1] = __uint_as_float(v.y);
-    x[2] = __uint_as_float(v.z);
-    x[3] = __uint_as_float(v.w);
-}
-
 // Reduce the pass-1 partial maxima (every CTA does it; it is a few KB of L2).
 __device__ __forceinline__ float reduce_partials(const float *__restrict__ partials, int n) {
     float m = 0.0f;
@@ -191,8 +149,69 @@ __device__ __forceinline__ float reduce_partials(const float *__restrict__ parti
 }
 
 // ---------------------------------------------------------------------------
-// Pass 2: encode.
+// Pass 2: encode.  One thread owns one 16-value block: its amax needs no
+// shuffle, the scale arithmetic runs once per block, the 16 products are 8
+// packed f32x2 multiplies (per-lane IEEE round-to-nearest, identical to 16
+// scalar ones), and the 8 code bytes leave as one 8-byte store.  Four
+// neighbouring lanes hold the four blocks of a 64-column group; their scale
+// bytes are gathered into one 32-bit word in the tiled layout.
 // ---------------------------------------------------------------------------
+
+// 16 values of one block as fp32 pairs, from 2 (bf16) or 4 (fp32) 16-byte loads.
+__device__ __forceinline__ void load_block(const __nv_bfloat16 *p, uint32_t (&w)[8]) {
+    const uint4 a = load_item(p), b = load_item(p + 8);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+}
+__device__ __forceinline__ float block_absmax(const uint32_t (&w)[8], __nv_bfloat16 *) {
+    uint32_t m = __vmaxu2(__vmaxu2(w[0] & 0x7fff7fffu, w[1] & 0x7fff7fffu),
+                          __vmaxu2(w[2] & 0x7fff7fffu, w[3] & 0x7fff7fffu));
+    m = __vmaxu2(m, __vmaxu2(__vmaxu2(w[4] & 0x7fff7fffu, w[5] & 0x7fff7fffu),
+                             __vmaxu2(w[6] & 0x7fff7fffu, w[7] & 0x7fff7fffu)));
+    return __uint_as_float(max(m & 0xffffu, m >> 16) << 16);
+}
+// element pair k of a bf16 block as a packed (lo, hi) fp32 pair
+__device__ __forceinline__ uint64_t pair_f32(const uint32_t (&w)[8], int k, __nv_bfloat16 *) {
+    return static_cast<uint64_t>(w[k] << 16) | (static_cast<uint64_t>(w[k] & 0xffff0000u) << 32);
+}
+
+__device__ __forceinline__ void load_block(const float *p, uint32_t (&w)[16]) {
+    const uint4 a = load_item(p), b = load_item(p + 4), c = load_item(p + 8), d = load_item(p + 12);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    w[8] = c.x; w[9] = c.y; w[10] = c.z; w[11] = c.w;
+    w[12] = d.x; w[13] = d.y; w[14] = d.z; w[15] = d.w;
+}
+__device__ __forceinline__ float block_absmax(const uint32_t (&w)[16], float *) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) m = max(m, w[k] & 0x7fffffffu);
+    return __uint_as_float(m);
+}
+__device__ __forceinline__ uint64_t pair_f32(const uint32_t (&w)[16], int k, float *) {
+    return static_cast<uint64_t>(w[2 * k]) | (static_cast<uint64_t>(w[2 * k + 1]) << 32);
+}
+
+// (lo, hi) * (r, r), each lane rounded to nearest even.
+__device__ __forceinline__ uint64_t mul_pair(uint64_t v, uint64_t rr) {
+    uint64_t o;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(o) : "l"(v), "l"(rr));
+    return o;
+}
+
+// one code byte from a packed (lo, hi) pair: lo -> low nibble, hi -> high nibble
+__device__ __forceinline__ uint32_t e2m1_pair(uint64_t v) {
+    uint32_t out;
+    const float lo = __uint_as_float(static_cast<uint32_t>(v));
+    const float hi = __uint_as_float(static_cast<uint32_t>(v >> 32));
+    asm("{\n\t.reg .b8 b;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\t"
+        "cvt.u32.u8 %0, b;\n\t}"
+        : "=r"(out)
+        : "f"(lo), "f"(hi));
+    return out;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, int64_t rows,
                                                      int64_t cols, int64_t ld,
@@ -200,11 +219,9 @@ __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, in
                                                      int num_partials, uint8_t *__restrict__ codes,
                                                      uint8_t *__restrict__ scales,
                                                      float *__restrict__ g_out) {
-    constexpr int EPI = Elem<T>::kPerItem;      // values per item
-    constexpr int IPB = kBlock / EPI;           // items (lanes) per 16-value block
-    constexpr int GROUP = 4 * IPB;              // lanes per 32-bit scale word
-    const int64_t ipr = cols / EPI;
-    const int64_t total = rows * ipr;
+    constexpr int W = sizeof(T) == 2 ? 8 : 16;        // 32-bit words per block
+    const int64_t bpr = cols / kBlock;                  // blocks per row
+    const int64_t total = rows * bpr;
     const int64_t kb4 = kb4_of(cols);
     const int64_t S = static_cast<int64_t>(gridDim.x) * blockDim.x;
     const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -217,57 +234,57 @@ __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, in
     const float six_g = __fmul_rn(6.0f, g);
     if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
 
+    // Walk the windows of S blocks from the last one back to the first: the
+    // tail of x that pass 1 read last is the part most likely still in L2.
     const int64_t nwin = ceil_div(total, S);
-    const int64_t dr = S / ipr, dj = S - dr * ipr;
+    const int64_t dr = S / bpr, dj = S - dr * bpr;
     ItemCursor c;
-    c.set((nwin - 1) * S + t, ipr);
+    c.set((nwin - 1) * S + t, bpr);
     constexpr int U = 2;
     for (int64_t w = nwin - 1; w >= 0; w -= U) {
-        uint4 v[U];
+        uint32_t v[U][W];
         ItemCursor cu[U];
         bool valid[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             cu[u] = c;
-            const int64_t i = (w - u) * S + t;
-            valid[u] = (w - u) >= 0 && i < total;
-            v[u] = valid[u] ? load_item(x + c.r * ld + c.j * EPI) : make_uint4(0, 0, 0, 0);
-            c.retreat(dr, dj, ipr);
+            valid[u] = (w - u) >= 0 && (w - u) * S + t < total;
+            if (valid[u]) {
+                load_block(x + c.r * ld + c.j * kBlock, v[u]);
+            } else {
+#pragma unroll
+                for (int k = 0; k < W; ++k) v[u][k] = 0u;
+            }
+            c.retreat(dr, dj, bpr);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            float bamax = item_absmax(v[u], static_cast<T *>(nullptr));
-#pragma unroll
-            for (int o = 1; o < IPB; o <<= 1) bamax = fmaxf(bamax, __shfl_xor_sync(0xffffffffu, bamax, o));
+            const float bamax = block_absmax(v[u], static_cast<T *>(nullptr));
             const float tb = g > 0.0f ? __fdiv_rn(bamax, six_g) : 0.0f;
             const uint32_t s = e4m3_of(tb);
             const float d = __fmul_rn(e4m3_value(s), g);
             const float rcp = __frcp_rn(d);
             const bool zero_block = (d == 0.0f) || isinf(rcp);
-            float xv[EPI];
-            unpack(v[u], xv);
+            const uint64_t rr = static_cast<uint64_t>(__float_as_uint(rcp)) * 0x100000001ull;
+            uint32_t lo = 0, hi = 0;
 #pragma unroll
-            for (int k = 0; k < EPI; ++k) xv[k] = __fmul_rn(xv[k], rcp);
-            uint32_t packed = (EPI == 8) ? e2m1x8(reinterpret_cast<float(&)[8]>(xv))
-                                         : e2m1x4(reinterpret_cast<float(&)[4]>(xv));
-            if (zero_block) packed = 0;
-            // gather the four block scales of a 64-column group into one word
+            for (int k = 0; k < 4; ++k)
+                lo |= e2m1_pair(mul_pair(pair_f32(v[u], k, static_cast<T *>(nullptr)), rr)) << (8 * k);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                hi |= e2m1_pair(mul_pair(pair_f32(v[u], 4 + k, static_cast<T *>(nullptr)), rr)) << (8 * k);
+            if (zero_block) lo = hi = 0u;
             uint32_t word = s;
-            word |= __shfl_down_sync(0xffffffffu, s, IPB) << 8;
-            word |= __shfl_down_sync(0xffffffffu, s, 2 * IPB) << 16;
-            word |= __shfl_down_sync(0xffffffffu, s, 3 * IPB) << 24;
+            word |= __shfl_down_sync(0xffffffffu, s, 1) << 8;
+            word |= __shfl_down_sync(0xffffffffu, s, 2) << 16;
+            word |= __shfl_down_sync(0xffffffffu, s, 3) << 24;
             if (valid[u]) {
-                const int64_t r = cu[u].r, j = cu[u].j;
-                if (EPI == 8)
-                    *reinterpret_cast<uint32_t *>(codes + r * (cols / 2) + j * 4) = packed;
-                else
-                    *reinterpret_cast<uint16_t *>(codes + r * (cols / 2) + j * 2) =
-                        static_cast<uint16_t>(packed);
-                const int64_t kb = j / IPB;
+                const int64_t r = cu[u].r, kb = cu[u].j;
+                *reinterpret_cast<uint2 *>(codes + r * (cols / 2) + kb * 8) = make_uint2(lo, hi);
                 if (word_scales) {
-                    if ((lane % GROUP) == 0)
+                    if ((lane & 3) == 0)
                         *reinterpret_cast<uint32_t *>(scales + scale_offset(r, kb, kb4)) = word;
-                } else if ((lane % IPB) == 0) {
+                } else {
                     scales[scale_offset(r, kb, kb4)] = static_cast<uint8_t>(s);
                 }
             }
@@ -276,12 +293,11 @@ __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, in
 
     // Zero the padding of the scale layout: blocks kb in [cols/16, kb4) of
     // real rows, and every block of rows in [rows, roundup(rows, 128)).
-    const int64_t kb = cols / kBlock;
-    const int64_t pad_a = rows * (kb4 - kb);
+    const int64_t pad_a = rows * (kb4 - bpr);
     const int64_t r128 = round_up(rows, 128);
     const int64_t pad_b_words = (r128 - rows) * (kb4 / 4);
     for (int64_t i = t; i < pad_a; i += S) {
-        const int64_t r = i / (kb4 - kb), q = kb + (i - r * (kb4 - kb));
+        const int64_t r = i / (kb4 - bpr), q = bpr + (i - r * (kb4 - bpr));
         scales[scale_offset(r, q, kb4)] = 0;
     }
     for (int64_t i = t; i < pad_b_words; i += S) {
@@ -360,7 +376,8 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
                             int num_sms, cudaStream_t stream) {
     const int eb = bf16 ? 2 : 4;
     int g1 = quantize_grid(rows, cols, eb, num_sms, 4);
-    int g2 = quantize_grid(rows, cols, eb, num_sms, 8);
+    // pass 2 runs one thread per 16-value block
+    const int g2 = quantize_grid(rows, cols, 1, num_sms, 4);
     if (g1 > kMaxAmaxPartials) g1 = kMaxAmaxPartials;
     if (bf16)
         amax_partials_kernel<__nv_bfloat16><<<g1, 256, 0, stream>>>(
