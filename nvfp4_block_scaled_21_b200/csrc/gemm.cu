@@ -22,9 +22,11 @@
 //               slot owned by the stage.  This keeps scale movement off the
 //               tensor pipe, where a tcgen05.cp per 512-byte atom would cost
 //               about as much tensor-pipe time as the MMAs themselves.
-//   warps 6..9  epilogue: tcgen05.ld of the accumulator (next chunk in flight
-//               while the current one is stored), y = acc * (gA*gB), RNE to
-//               bf16 (or fp32), and the store.
+//   warps 6..13 epilogue, two warps per TMEM lane quarter, each owning half
+//               of the tile's columns (bf16 output, tiles >= 64 wide):
+//               tcgen05.ld of the accumulator with the next chunk in flight,
+//               y = acc * (gA*gB), RNE to bf16, store; the accumulator is
+//               released to the MMA warp as soon as both halves are read.
 // Small M (decode) runs "swapped": the weights ride the MMA's M = 128 and the
 // few activation rows ride N = BN, so the weight stream spreads over all SMs.
 // When the weights are known not to come from the kernel launched just before
@@ -73,14 +75,14 @@ struct GemmCfg {
                                    : kColsUsed <= 256 ? 256 : 512;
     static constexpr int kBarBytes = 8 * (3 * kStages + 4) + 16;
     static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;   // + alignment slack
-    static constexpr int kThreads = 320;
+    static constexpr int kThreads = 448;                       // 14 warps
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kColsUsed <= 512, "tensor memory budget");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
 };
 
 template <int BN, bool SWAP, typename OutT>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
 gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ GemmArgs args) {
     using C = GemmCfg<BN>;
@@ -112,7 +114,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&tfull[s], 1);
-            mbar_init(&tempty[s], 128);
+            mbar_init(&tempty[s], 256);
         }
         *abort_flag = 0u;
         fence_mbar_init();
@@ -303,10 +305,10 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // ------------------------------------------------------------ epilogue
         asm volatile("griddepcontrol.wait;" ::: "memory");   // tensor scales may be fresh
         const int quarter = warp & 3;               // TMEM lane quarter this warp may read
+        const int half = (warp - 6) >> 2;           // column half of the tile (fast drain)
         const int row = quarter * 32 + lane;        // accumulator row (MMA M index)
         const float alpha = __fmul_rn(*args.ga, *args.gb);
-        constexpr int CH = BN < 32 ? BN : 32;
-        constexpr int NCH = BN / CH;
+        constexpr bool kFastDrain = !SWAP && sizeof(OutT) == 2 && BN >= 64;
         uint32_t acc = 0, acc_phase = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             const int pt = tile % args.num_p_tiles;
@@ -317,77 +319,124 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             tc_fence_after();
             const int p = pt * 128 + row;
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
-            uint32_t r[2][CH];
-            auto ld = [&](int c, uint32_t (&dst)[CH]) {
-                if constexpr (CH == 32)
-                    tmem_ld_32x32b_x32(tbase + c * CH, reinterpret_cast<uint32_t(&)[32]>(dst));
-                else
-                    tmem_ld_32x32b_x16(tbase + c * CH, reinterpret_cast<uint32_t(&)[16]>(dst));
-            };
-            ld(0, r[0]);
-            tmem_ld_wait();
+            if constexpr (kFastDrain) {
+                // each warp drains and stores its half of the columns, the next
+                // 32-column chunk in flight while the current one is stored
+                constexpr int HC = BN / 2;
+                constexpr int NCH = HC / 32;
+                uint32_t r[2][32];
+                const uint32_t tb = tbase + half * HC;
+                tmem_ld_32x32b_x32(tb, r[0]);
+                tmem_ld_wait();
+                OutT *yrow = static_cast<OutT *>(args.y) + static_cast<int64_t>(p) * args.ldy;
 #pragma unroll
-            for (int c = 0; c < NCH; ++c) {
-                if (c + 1 < NCH) ld(c + 1, r[(c + 1) & 1]);       // next chunk in flight
-                float v[CH];
+                for (int c = 0; c < NCH; ++c) {
+                    if (c + 1 < NCH) tmem_ld_32x32b_x32(tb + (c + 1) * 32, r[(c + 1) & 1]);
+                    uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < CH; ++i) v[i] = __fmul_rn(__uint_as_float(r[c & 1][i]), alpha);
-                const int q0 = qt * BN + c * CH;
-                if constexpr (SWAP) {
-                    // y[q][p]: for each i the warp writes 32 consecutive p
-                    if (p < args.P) {
-                        OutT *y = static_cast<OutT *>(args.y);
-#pragma unroll
-                        for (int i = 0; i < CH; ++i) {
-                            const int q = q0 + i;
-                            if (q < args.Q) {
-                                if constexpr (sizeof(OutT) == 2)
-                                    y[static_cast<int64_t>(q) * args.ldy + p] = __float2bfloat16_rn(v[i]);
-                                else
-                                    y[static_cast<int64_t>(q) * args.ldy + p] = v[i];
-                            }
-                        }
+                    for (int k = 0; k < 16; ++k) {
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[c & 1][2 * k]), alpha),
+                                                                  __fmul_rn(__uint_as_float(r[c & 1][2 * k + 1]), alpha));
+                        pk[k] = *reinterpret_cast<uint32_t *>(&b2);
                     }
-                } else {
-                    // y[p][q0 .. q0+CH): one contiguous run per thread
+                    const int q0 = qt * BN + half * HC + c * 32;
                     if (p < args.P) {
-                        OutT *yrow = static_cast<OutT *>(args.y) + static_cast<int64_t>(p) * args.ldy;
-                        if (q0 + CH <= args.Q) {
-                            if constexpr (sizeof(OutT) == 2) {
+                        if (q0 + 32 <= args.Q) {
 #pragma unroll
-                                for (int i = 0; i < CH; i += 8) {
-                                    uint4 pk;
-                                    uint32_t *w = reinterpret_cast<uint32_t *>(&pk);
-#pragma unroll
-                                    for (int k = 0; k < 4; ++k) {
-                                        __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * k], v[i + 2 * k + 1]);
-                                        w[k] = *reinterpret_cast<uint32_t *>(&b2);
-                                    }
-                                    *reinterpret_cast<uint4 *>(yrow + q0 + i) = pk;
-                                }
-                            } else {
-#pragma unroll
-                                for (int i = 0; i < CH; i += 4)
-                                    *reinterpret_cast<float4 *>(yrow + q0 + i) =
-                                        make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                            }
+                            for (int i = 0; i < 4; ++i)
+                                *reinterpret_cast<uint4 *>(yrow + q0 + 8 * i) =
+                                    make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                         } else {
 #pragma unroll
-                            for (int i = 0; i < CH; ++i) {
-                                if (q0 + i < args.Q) {
-                                    if constexpr (sizeof(OutT) == 2)
-                                        yrow[q0 + i] = __float2bfloat16_rn(v[i]);
-                                    else
-                                        yrow[q0 + i] = v[i];
-                                }
+                            for (int i = 0; i < 16; ++i) {
+                                if (q0 + 2 * i < args.Q)
+                                    reinterpret_cast<unsigned short *>(yrow)[q0 + 2 * i] = static_cast<unsigned short>(pk[i] & 0xffffu);
+                                if (q0 + 2 * i + 1 < args.Q)
+                                    reinterpret_cast<unsigned short *>(yrow)[q0 + 2 * i + 1] = static_cast<unsigned short>(pk[i] >> 16);
                             }
                         }
                     }
+                    if (c + 1 < NCH) tmem_ld_wait();
                 }
-                if (c + 1 < NCH) tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&tempty[acc]);
+            } else {
+                if (half == 0) {
+                    constexpr int CH = BN < 32 ? BN : 32;
+                    constexpr int NCH = BN / CH;
+                    uint32_t r[2][CH];
+                    auto ld = [&](int c, uint32_t (&dst)[CH]) {
+                        if constexpr (CH == 32)
+                            tmem_ld_32x32b_x32(tbase + c * CH, reinterpret_cast<uint32_t(&)[32]>(dst));
+                        else
+                            tmem_ld_32x32b_x16(tbase + c * CH, reinterpret_cast<uint32_t(&)[16]>(dst));
+                    };
+                    ld(0, r[0]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < NCH; ++c) {
+                        if (c + 1 < NCH) ld(c + 1, r[(c + 1) & 1]);       // next chunk in flight
+                        float v[CH];
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) v[i] = __fmul_rn(__uint_as_float(r[c & 1][i]), alpha);
+                        const int q0 = qt * BN + c * CH;
+                        if constexpr (SWAP) {
+                            // y[q][p]: for each i the warp writes 32 consecutive p
+                            if (p < args.P) {
+                                OutT *y = static_cast<OutT *>(args.y);
+#pragma unroll
+                                for (int i = 0; i < CH; ++i) {
+                                    const int q = q0 + i;
+                                    if (q < args.Q) {
+                                        if constexpr (sizeof(OutT) == 2)
+                                            y[static_cast<int64_t>(q) * args.ldy + p] = __float2bfloat16_rn(v[i]);
+                                        else
+                                            y[static_cast<int64_t>(q) * args.ldy + p] = v[i];
+                                    }
+                                }
+                            }
+                        } else {
+                            // y[p][q0 .. q0+CH): one contiguous run per thread
+                            if (p < args.P) {
+                                OutT *yrow = static_cast<OutT *>(args.y) + static_cast<int64_t>(p) * args.ldy;
+                                if (q0 + CH <= args.Q) {
+                                    if constexpr (sizeof(OutT) == 2) {
+#pragma unroll
+                                        for (int i = 0; i < CH; i += 8) {
+                                            uint4 pk;
+                                            uint32_t *w = reinterpret_cast<uint32_t *>(&pk);
+#pragma unroll
+                                            for (int k = 0; k < 4; ++k) {
+                                                __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * k], v[i + 2 * k + 1]);
+                                                w[k] = *reinterpret_cast<uint32_t *>(&b2);
+                                            }
+                                            *reinterpret_cast<uint4 *>(yrow + q0 + i) = pk;
+                                        }
+                                    } else {
+#pragma unroll
+                                        for (int i = 0; i < CH; i += 4)
+                                            *reinterpret_cast<float4 *>(yrow + q0 + i) =
+                                                make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                                    }
+                                } else {
+#pragma unroll
+                                    for (int i = 0; i < CH; ++i) {
+                                        if (q0 + i < args.Q) {
+                                            if constexpr (sizeof(OutT) == 2)
+                                                yrow[q0 + i] = __float2bfloat16_rn(v[i]);
+                                            else
+                                                yrow[q0 + i] = v[i];
+                                        }
+                                    }
+                                }
+                            }
+                        }
+                        if (c + 1 < NCH) tmem_ld_wait();
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&tempty[acc]);
             }
-            tc_fence_before();
-            mbar_arrive(&tempty[acc]);
             if (C::kAccStages == 2) {
                 acc ^= 1u;
                 if (acc == 0) acc_phase ^= 1u;

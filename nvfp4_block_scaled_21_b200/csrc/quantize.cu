@@ -9,8 +9,8 @@
 //   workspace (no atomics, nothing to reset between calls).
 // Pass 2 (encode_kernel): every CTA reduces the partial maxima (a few KB from
 //   L2), derives g = amax/2688 on the device, and encodes the tensor, walking
-//   the windows in the reverse order of pass 1 so that the tail pass 1 read
-//   last is still in L2.  One thread owns one 16-element block; the E4M3
+//   the windows in the same order as pass 1 (on B200 a second forward sweep
+//   finds part of x in L2).  One thread owns one 16-element block; the E4M3
 //   scale and the E2M1 codes come from the hardware RNE-satfinite
 //   conversions; codes go out as one 8-byte store per block and scales as one
 //   32-bit word per four blocks in the tiled layout the tensor cores read.
@@ -70,29 +70,48 @@ __global__ void __launch_bounds__(256) amax_partials_kernel(const T *__restrict_
                                                             int64_t cols, int64_t ld,
                                                             float *__restrict__ partials) {
     constexpr int EPI = Elem<T>::kPerItem;
-    const int64_t ipr = cols / EPI;
-    const int64_t total = rows * ipr;
-    const int64_t S = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t dr = S / ipr, dj = S - dr * ipr;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // let the encode pass queue up
     float m = 0.0f;
-    ItemCursor c;
-    c.set(t, ipr);
-    constexpr int U = 4;
-    for (int64_t i = t; i < total; i += U * S) {
-        uint4 v[U];
-        ItemCursor cu = c;
+    if (ld == cols && rows * cols / EPI < (int64_t(1) << 31)) {
+        // contiguous: one flat stream of 16-byte vectors, 32-bit indices,
+        // 8 loads in flight per thread
+        const uint32_t total = static_cast<uint32_t>(rows * cols / EPI);
+        const uint32_t S = gridDim.x * blockDim.x;
+        const uint4 *v16 = reinterpret_cast<const uint4 *>(x);
+        constexpr int U = 8;
+        uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+        for (; i + (U - 1) * S < total; i += U * S) {
+            uint4 v[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            if (i + u * S < total)
-                v[u] = load_item(x + cu.r * ld + cu.j * EPI);
-            else
-                v[u] = make_uint4(0, 0, 0, 0);
-            cu.advance(dr, dj, ipr);
+            for (int u = 0; u < U; ++u) v[u] = __ldg(v16 + i + u * S);
+#pragma unroll
+            for (int u = 0; u < U; ++u) m = fmaxf(m, item_absmax(v[u], static_cast<T *>(nullptr)));
         }
+        for (; i < total; i += S) m = fmaxf(m, item_absmax(__ldg(v16 + i), static_cast<T *>(nullptr)));
+    } else {
+        const int64_t ipr = cols / EPI;
+        const int64_t total = rows * ipr;
+        const int64_t S = static_cast<int64_t>(gridDim.x) * blockDim.x;
+        const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+        const int64_t dr = S / ipr, dj = S - dr * ipr;
+        ItemCursor c;
+        c.set(t, ipr);
+        constexpr int U = 4;
+        for (int64_t i = t; i < total; i += U * S) {
+            uint4 v[U];
+            ItemCursor cu = c;
 #pragma unroll
-        for (int u = 0; u < U; ++u) m = fmaxf(m, item_absmax(v[u], static_cast<T *>(nullptr)));
-        c = cu;
+            for (int u = 0; u < U; ++u) {
+                if (i + u * S < total)
+                    v[u] = load_item(x + cu.r * ld + cu.j * EPI);
+                else
+                    v[u] = make_uint4(0, 0, 0, 0);
+                cu.advance(dr, dj, ipr);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) m = fmaxf(m, item_absmax(v[u], static_cast<T *>(nullptr)));
+            c = cu;
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -105,8 +124,6 @@ __global__ void __launch_bounds__(256) amax_partials_kernel(const T *__restrict_
         for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
         if (threadIdx.x == 0) partials[blockIdx.x] = v;
     }
-    // Let a dependent launch (the encode pass) start its prologue.
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -199,17 +216,54 @@ __device__ __forceinline__ uint64_t mul_pair(uint64_t v, uint64_t rr) {
     return o;
 }
 
-// one code byte from a packed (lo, hi) pair: lo -> low nibble, hi -> high nibble
-__device__ __forceinline__ uint32_t e2m1_pair(uint64_t v) {
+// four code bytes from four packed (lo, hi) pairs: pair k -> byte k, lo in
+// the low nibble, hi in the high nibble
+__device__ __forceinline__ uint32_t e2m1_x8(uint64_t p0, uint64_t p1, uint64_t p2, uint64_t p3) {
     uint32_t out;
-    const float lo = __uint_as_float(static_cast<uint32_t>(v));
-    const float hi = __uint_as_float(static_cast<uint32_t>(v >> 32));
-    asm("{\n\t.reg .b8 b;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\t"
-        "cvt.u32.u8 %0, b;\n\t}"
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
         : "=r"(out)
-        : "f"(lo), "f"(hi));
+        : "f"(__uint_as_float(static_cast<uint32_t>(p0))), "f"(__uint_as_float(static_cast<uint32_t>(p0 >> 32))),
+          "f"(__uint_as_float(static_cast<uint32_t>(p1))), "f"(__uint_as_float(static_cast<uint32_t>(p1 >> 32))),
+          "f"(__uint_as_float(static_cast<uint32_t>(p2))), "f"(__uint_as_float(static_cast<uint32_t>(p2 >> 32))),
+          "f"(__uint_as_float(static_cast<uint32_t>(p3))), "f"(__uint_as_float(static_cast<uint32_t>(p3 >> 32))));
     return out;
+}
+
+// E4M3 scale byte of one block: s = RNE_E4M3(fl32(bamax / six_g)).
+// The quotient only feeds the E4M3 rounding, so it is first formed as
+// tq = fl32(bamax * fl32(1 / six_g)), which is within 1.5 ulp of the correctly
+// rounded quotient.  If rounding tq scaled by (1 - 2^-20) and by (1 + 2^-20)
+// gives the same E4M3 byte, no E4M3 rounding boundary (and no tie) lies within
+// that interval, which contains the exact quotient's rounding, so the byte is
+// the one the correctly rounded division would give.  Otherwise (a boundary
+// is near, probability about 3e-5) the division is done exactly.
+__device__ __forceinline__ uint32_t block_scale_byte(float bamax, float six_g, float inv6g,
+                                                     bool exact_only) {
+    if (!exact_only) {
+        const float tq = __fmul_rn(bamax, inv6g);
+        const uint32_t lo = e4m3_of(__fmul_rn(tq, 0.99999904632568359375f));   // 1 - 2^-20
+        const uint32_t hi = e4m3_of(__fmul_rn(tq, 1.00000095367431640625f));   // 1 + 2^-20
+        if (lo == hi) return lo;
+    }
+    return e4m3_of(six_g > 0.0f ? __fdiv_rn(bamax, six_g) : 0.0f);
+}
+
+// Codes of one block: 8 bytes, element 2k in the low nibble of byte k.
+template <typename T, int W>
+__device__ __forceinline__ uint2 block_codes(const uint32_t (&v)[W], float rcp) {
+    const uint64_t rr = static_cast<uint64_t>(__float_as_uint(rcp)) * 0x100000001ull;
+    T *tag = nullptr;
+    const uint32_t lo = e2m1_x8(mul_pair(pair_f32(v, 0, tag), rr), mul_pair(pair_f32(v, 1, tag), rr),
+                                mul_pair(pair_f32(v, 2, tag), rr), mul_pair(pair_f32(v, 3, tag), rr));
+    const uint32_t hi = e2m1_x8(mul_pair(pair_f32(v, 4, tag), rr), mul_pair(pair_f32(v, 5, tag), rr),
+                                mul_pair(pair_f32(v, 6, tag), rr), mul_pair(pair_f32(v, 7, tag), rr));
+    // rcp == 0 marks a zero-scale block: all of its codes are 0
+    return rcp == 0.0f ? make_uint2(0u, 0u) : make_uint2(lo, hi);
 }
 
 template <typename T>
@@ -228,66 +282,102 @@ __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, in
     const int lane = threadIdx.x & 31;
     const bool word_scales = (cols % 64) == 0;
 
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // let the GEMM queue up
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const float amax = reduce_partials(partials, num_partials);
     const float g = __fdiv_rn(amax, kTensorScaleDiv);
     const float six_g = __fmul_rn(6.0f, g);
     if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    // Reciprocal of every possible block scale: fl32(1 / fl32(dec(s) * g)),
+    // 0 marking a zero-scale block (d == 0 or 1/d overflows).
+    __shared__ float rcp_table[128];
+    if (threadIdx.x < 128) {
+        const float d = __fmul_rn(e4m3_value(threadIdx.x), g);
+        const float r = __frcp_rn(d);
+        rcp_table[threadIdx.x] = (d == 0.0f || isinf(r)) ? 0.0f : r;
+    }
+    const float inv6g = __frcp_rn(six_g);
+    const bool exact_only = !(six_g > 0.0f) || isinf(inv6g);
+    __syncthreads();
 
-    // Walk the windows of S blocks from the last one back to the first: the
-    // tail of x that pass 1 read last is the part most likely still in L2.
-    const int64_t nwin = ceil_div(total, S);
-    const int64_t dr = S / bpr, dj = S - dr * bpr;
-    ItemCursor c;
-    c.set((nwin - 1) * S + t, bpr);
     constexpr int U = 2;
-    for (int64_t w = nwin - 1; w >= 0; w -= U) {
-        uint32_t v[U][W];
-        ItemCursor cu[U];
-        bool valid[U];
+    const bool flat32 = (ld == cols) && total < (int64_t(1) << 31) &&
+                        round_up(rows, 128) * kb4 < (int64_t(1) << 31);
+    if (flat32) {
+        // contiguous tensor: block b at element 16 b, codes at byte 8 b;
+        // (row, block-in-row) tracked incrementally in 32 bits
+        const uint32_t total32 = static_cast<uint32_t>(total), S32 = static_cast<uint32_t>(S);
+        const uint32_t bpr32 = static_cast<uint32_t>(bpr), kb4q = static_cast<uint32_t>(kb4 >> 2);
+        const uint32_t dr = S32 / bpr32, dj = S32 - dr * bpr32;
+        uint32_t r = static_cast<uint32_t>(t) / bpr32, kb = static_cast<uint32_t>(t) - r * bpr32;
+        for (uint32_t b0 = static_cast<uint32_t>(t); b0 < total32; b0 += U * S32) {
+            uint32_t v[U][W];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            cu[u] = c;
-            valid[u] = (w - u) >= 0 && (w - u) * S + t < total;
-            if (valid[u]) {
-                load_block(x + c.r * ld + c.j * kBlock, v[u]);
-            } else {
-#pragma unroll
-                for (int k = 0; k < W; ++k) v[u][k] = 0u;
-            }
-            c.retreat(dr, dj, bpr);
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const float bamax = block_absmax(v[u], static_cast<T *>(nullptr));
-            const float tb = g > 0.0f ? __fdiv_rn(bamax, six_g) : 0.0f;
-            const uint32_t s = e4m3_of(tb);
-            const float d = __fmul_rn(e4m3_value(s), g);
-            const float rcp = __frcp_rn(d);
-            const bool zero_block = (d == 0.0f) || isinf(rcp);
-            const uint64_t rr = static_cast<uint64_t>(__float_as_uint(rcp)) * 0x100000001ull;
-            uint32_t lo = 0, hi = 0;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                lo |= e2m1_pair(mul_pair(pair_f32(v[u], k, static_cast<T *>(nullptr)), rr)) << (8 * k);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                hi |= e2m1_pair(mul_pair(pair_f32(v[u], 4 + k, static_cast<T *>(nullptr)), rr)) << (8 * k);
-            if (zero_block) lo = hi = 0u;
-            uint32_t word = s;
-            word |= __shfl_down_sync(0xffffffffu, s, 1) << 8;
-            word |= __shfl_down_sync(0xffffffffu, s, 2) << 16;
-            word |= __shfl_down_sync(0xffffffffu, s, 3) << 24;
-            if (valid[u]) {
-                const int64_t r = cu[u].r, kb = cu[u].j;
-                *reinterpret_cast<uint2 *>(codes + r * (cols / 2) + kb * 8) = make_uint2(lo, hi);
-                if (word_scales) {
-                    if ((lane & 3) == 0)
-                        *reinterpret_cast<uint32_t *>(scales + scale_offset(r, kb, kb4)) = word;
+            for (int u = 0; u < U; ++u) {
+                const uint32_t b = b0 + u * S32;
+                if (b < total32) {
+                    load_block(x + static_cast<size_t>(b) * kBlock, v[u]);
                 } else {
-                    scales[scale_offset(r, kb, kb4)] = static_cast<uint8_t>(s);
+#pragma unroll
+                    for (int k = 0; k < W; ++k) v[u][k] = 0u;
                 }
             }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const uint32_t b = b0 + u * S32;
+                const float bamax = block_absmax(v[u], static_cast<T *>(nullptr));
+                const uint32_t sb = block_scale_byte(bamax, six_g, inv6g, exact_only);
+                const uint2 cw = block_codes<T, W>(v[u], rcp_table[sb]);
+                uint32_t word = sb;
+                word |= __shfl_down_sync(0xffffffffu, sb, 1) << 8;
+                word |= __shfl_down_sync(0xffffffffu, sb, 2) << 16;
+                word |= __shfl_down_sync(0xffffffffu, sb, 3) << 24;
+                if (b < total32) {
+                    *reinterpret_cast<uint2 *>(codes + static_cast<size_t>(b) * 8) = cw;
+                    const uint32_t off = ((r >> 7) * kb4q + (kb >> 2)) * 512u + (r & 31u) * 16u +
+                                         ((r >> 5) & 3u) * 4u + (kb & 3u);
+                    if (word_scales) {
+                        if ((lane & 3) == 0) *reinterpret_cast<uint32_t *>(scales + off) = word;
+                    } else {
+                        scales[off] = static_cast<uint8_t>(sb);
+                    }
+                }
+                r += dr;
+                kb += dj;
+                if (kb >= bpr32) { kb -= bpr32; ++r; }
+            }
+        }
+    } else {
+        const int64_t nwin = ceil_div(total, S);
+        const int64_t dr = S / bpr, dj = S - dr * bpr;
+        ItemCursor c;
+        c.set(t, bpr);
+        for (int64_t w = 0; w < nwin; ++w) {
+            uint32_t v[W];
+            const bool valid = w * S + t < total;
+            if (valid) {
+                load_block(x + c.r * ld + c.j * kBlock, v);
+            } else {
+#pragma unroll
+                for (int k = 0; k < W; ++k) v[k] = 0u;
+            }
+            const float bamax = block_absmax(v, static_cast<T *>(nullptr));
+            const uint32_t sb = block_scale_byte(bamax, six_g, inv6g, exact_only);
+            const uint2 cw = block_codes<T, W>(v, rcp_table[sb]);
+            uint32_t word = sb;
+            word |= __shfl_down_sync(0xffffffffu, sb, 1) << 8;
+            word |= __shfl_down_sync(0xffffffffu, sb, 2) << 16;
+            word |= __shfl_down_sync(0xffffffffu, sb, 3) << 24;
+            if (valid) {
+                *reinterpret_cast<uint2 *>(codes + c.r * (cols / 2) + c.j * 8) = cw;
+                if (word_scales) {
+                    if ((lane & 3) == 0)
+                        *reinterpret_cast<uint32_t *>(scales + scale_offset(c.r, c.j, kb4)) = word;
+                } else {
+                    scales[scale_offset(c.r, c.j, kb4)] = static_cast<uint8_t>(sb);
+                }
+            }
+            c.advance(dr, dj, bpr);
         }
     }
 
@@ -304,7 +394,6 @@ __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, in
         const int64_t r = rows + i / (kb4 / 4), q = 4 * (i % (kb4 / 4));
         *reinterpret_cast<uint32_t *>(scales + scale_offset(r, q, kb4)) = 0u;
     }
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -371,13 +460,26 @@ int quantize_grid(int64_t rows, int64_t cols, int elem_bytes, int num_sms, int p
     return static_cast<int>(blocks < cap ? blocks : cap);
 }
 
+// Resident 256-thread CTAs per SM of a kernel (looked up once).
+template <typename K>
+static int resident_ctas(K kernel) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 256, 0) != cudaSuccess || n < 1)
+        n = 1;
+    return n;
+}
+
 cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld,
                             uint8_t *codes, uint8_t *scales, float *g_out, float *partials,
                             int num_sms, cudaStream_t stream) {
     const int eb = bf16 ? 2 : 4;
-    int g1 = quantize_grid(rows, cols, eb, num_sms, 4);
+    static const int occ_amax[2] = {resident_ctas(amax_partials_kernel<float>),
+                                    resident_ctas(amax_partials_kernel<__nv_bfloat16>)};
+    static const int occ_encode[2] = {resident_ctas(encode_kernel<float>),
+                                      resident_ctas(encode_kernel<__nv_bfloat16>)};
+    int g1 = quantize_grid(rows, cols, eb, num_sms, occ_amax[bf16]);
     // pass 2 runs one thread per 16-value block
-    const int g2 = quantize_grid(rows, cols, 1, num_sms, 4);
+    const int g2 = quantize_grid(rows, cols, 1, num_sms, occ_encode[bf16]);
     if (g1 > kMaxAmaxPartials) g1 = kMaxAmaxPartials;
     if (bf16)
         amax_partials_kernel<__nv_bfloat16><<<g1, 256, 0, stream>>>(

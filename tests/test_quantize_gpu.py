@@ -121,6 +121,29 @@ def test_quantize_edge_cases(nv):
     assert_quantized_equal(quantize_gpu(nv, f32_tensor(h)), oracle.quantize(h))
 
 
+def test_block_scale_ties_and_boundaries(nv):
+    """Blocks whose quotient bamax/(6g) lands exactly on an E4M3 rounding
+    midpoint (ties to even), one ulp either side of it, and on E4M3 values:
+    the kernel's fast scale path must hand these to its exact division."""
+    vals = [oracle.e4m3_value(c) for c in range(0x7F)]
+    mids = [(a + b) / 2 for a, b in zip(vals[:-1], vals[1:])]
+    rows = [np.zeros(16, np.float32)]
+    rows[0][0] = np.float32(2688.0)                        # g = 1 exactly
+    for m in mids + vals[1:]:
+        for nudge in (0, -1, 1):
+            t = np.float32(m)
+            if nudge:
+                t = np.nextafter(t, np.float32(nudge * 1e9))
+            bamax = np.float32(np.float64(t) * 6.0)        # 6 t is exact in fp32 for these t
+            if np.float64(bamax) != np.float64(t) * 6.0 or t > 448:
+                continue                                   # keep the tensor amax at 2688
+            row = np.linspace(-1, 1, 16).astype(np.float32) * bamax
+            row[3] = bamax
+            rows.append(row)
+    x = np.stack(rows)
+    assert_quantized_equal(quantize_gpu(nv, f32_tensor(x)), oracle.quantize(x))
+
+
 def test_quantize_empty(nv):
     out = quantize_gpu(nv, torch.zeros((0, 64), device="cuda"))
     torch.cuda.synchronize()
