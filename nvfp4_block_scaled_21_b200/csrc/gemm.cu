@@ -109,12 +109,12 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         prefetch_tensormap(&tmB);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&sf_full[s], 128);
+            mbar_init(&sf_full[s], 4);     // one arrive per scale warp
             mbar_init(&empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&tfull[s], 1);
-            mbar_init(&tempty[s], 256);
+            mbar_init(&tempty[s], 8);      // one arrive per epilogue warp
         }
         *abort_flag = 0u;
         fence_mbar_init();
@@ -288,15 +288,31 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const uint32_t sf = tmem_base + lane_off + C::kSfBase + stage * C::kSfCols;
                 const uint8_t *a_src = sSfa + stage * C::kSfaStage + lane * 16;
                 const uint8_t *b_src = sSfb + stage * C::kSfbStage + lane * 16;
-                for (int j = 0; j < nk; ++j) {
-                    tmem_st_32x32b_x4(sf + 4 * j, ld_shared_v4(a_src + j * 512));
+                // one 16-column store for A's scales and one 16*kNQT-column
+                // store for B's per stage (columns of K-steps a partial last
+                // stage does not have are never read)
+                uint32_t av[16], bv[16 * C::kNQT];
 #pragma unroll
-                    for (int q = 0; q < C::kNQT; ++q)
-                        tmem_st_32x32b_x4(sf + 16 + 4 * (j * C::kNQT + q), ld_shared_v4(b_src + q * 2048 + j * 512));
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 a = ld_shared_v4(a_src + j * 512);
+                    av[4 * j] = a.x; av[4 * j + 1] = a.y; av[4 * j + 2] = a.z; av[4 * j + 3] = a.w;
+#pragma unroll
+                    for (int q = 0; q < C::kNQT; ++q) {
+                        const uint4 b = ld_shared_v4(b_src + q * 2048 + j * 512);
+                        const int o = 4 * (j * C::kNQT + q);
+                        bv[o] = b.x; bv[o + 1] = b.y; bv[o + 2] = b.z; bv[o + 3] = b.w;
+                    }
                 }
+                (void)nk;
+                tmem_st_32x32b_x16(sf, av);
+                if constexpr (C::kNQT == 1)
+                    tmem_st_32x32b_x16(sf + 16, reinterpret_cast<uint32_t(&)[16]>(bv));
+                else
+                    tmem_st_32x32b_x32(sf + 16, reinterpret_cast<uint32_t(&)[32]>(bv));
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&sf_full[stage]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_full[stage]);
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
@@ -359,7 +375,8 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     if (c + 1 < NCH) tmem_ld_wait();
                 }
                 tc_fence_before();
-                mbar_arrive(&tempty[acc]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
             } else {
                 if (half == 0) {
                     constexpr int CH = BN < 32 ? BN : 32;
@@ -435,7 +452,8 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     }
                 }
                 tc_fence_before();
-                mbar_arrive(&tempty[acc]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
             }
             if (C::kAccStages == 2) {
                 acc ^= 1u;
@@ -550,6 +568,8 @@ cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void 
         NVFP4_SWAPPED(64)
 #undef NVFP4_SWAPPED
     }
+    if (pair_gemm_usable(M, N, num_sms))
+        return launch_gemm_pair(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, stream);
     const int64_t ptiles = ceil_div(M, 128);
     const bool wide = ptiles * ceil_div(N, 256) >= 2 * num_sms;
     if (wide)

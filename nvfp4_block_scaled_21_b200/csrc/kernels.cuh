@@ -30,6 +30,12 @@ cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void 
                         int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
                         cudaStream_t stream, bool weights_ready = false);
 
+// Two-CTA (cta_group::2) GEMM for large M: usable when enough 256x256 tiles
+// exist to fill the GPU with CTA pairs.
+bool pair_gemm_usable(int64_t M, int64_t N, int num_sms);
+cudaError_t launch_gemm_pair(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
+                             int64_t ldy, uint32_t *status, uint64_t timeout_ns, cudaStream_t stream);
+
 // h = SiLU(gate) * up elementwise in fp32 (n values).
 cudaError_t launch_silu_mul(const float *gate, const float *up, float *h, int64_t n, int num_sms,
                             cudaStream_t stream);

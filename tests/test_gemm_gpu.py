@@ -113,6 +113,28 @@ def test_gemm_wide_tiles(nv):
     assert_gemm_close(yc[ms, ns], ref, na, nb, K, True, "wide tiles")
 
 
+@pytest.mark.parametrize("pair", ["0", "1"])
+@pytest.mark.parametrize("M,N,K", [(2304, 4608, 256), (2000, 4700, 320)])
+def test_gemm_cta_pair_tiles(nv, M, N, K, pair, monkeypatch):
+    """Shapes large enough for the two-CTA 256x256 tiles (switched on with
+    NVFP4_GEMM_CTA_PAIR=1), including ragged M (the second CTA of the last row
+    pair partly or wholly outside), ragged N and a partial last K slab; sampled
+    outputs plus the last row and column, for both the pair and one-CTA paths."""
+    monkeypatch.setenv("NVFP4_GEMM_CTA_PAIR", pair)
+    rng = np.random.default_rng(M + N)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[rng.random(x.shape) < 1e-3] *= 50
+    wt = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    xq_o, wq_o = oracle.quantize(x), oracle.quantize(wt)
+    y = run_gemm(nv, quantize_gpu(nv, f32_tensor(x)), quantize_gpu(nv, f32_tensor(wt)), torch.bfloat16)
+    yc = to_numpy_f64(y)
+    ms = np.concatenate([rng.integers(0, M, 4000), np.full(N, M - 1), np.arange(M)])
+    ns = np.concatenate([rng.integers(0, N, 4000), np.arange(N), np.full(M, N - 1)])
+    ref, na, nb = oracle.gemm_entries(xq_o, wq_o, ms, ns)
+    assert_gemm_close(yc[ms, ns], ref, na, nb, K, True, f"pair {M}x{N}x{K}")
+    assert np.isfinite(yc).all()
+
+
 def test_gemm_special_operands(nv):
     # all-zero activations -> exact zeros; constant operands -> closed form
     z = quantize_gpu(nv, torch.zeros((8, 128), device="cuda"))
