@@ -507,6 +507,34 @@ CUresult encode_tensor_map_u8(CUtensorMap *map, const void *base, uint64_t inner
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+CUresult encode_scale_map(CUtensorMap *map, const void *scales, uint64_t k_steps, uint64_t row_tiles,
+                          uint32_t box_tiles) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return CUDA_ERROR_NOT_FOUND;
+    // x: 128 words of one 512-byte atom; y: K-step (atom) within a 128-row
+    // tile; z: 128-row tile.  A box holds 4 K-steps of box_tiles row tiles.
+    cuuint64_t dims[3] = {128, k_steps, row_tiles};
+    cuuint64_t strides[2] = {512, k_steps * 512};
+    cuuint32_t box[3] = {128, 4, box_tiles};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void *>(scales), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+CUresult encode_output_map_bf16(CUtensorMap *map, void *y, uint64_t rows, uint64_t cols, uint64_t ld,
+                                uint32_t box_cols, uint32_t box_rows) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return CUDA_ERROR_NOT_FOUND;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 template <int BN, bool SWAP, typename OutT>
 static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, void *y, int64_t ldy,
                             uint32_t *status, uint64_t timeout_ns, int num_sms, int preload,

@@ -10,20 +10,33 @@
 // with one M=256 MMA: each CTA loads and feeds only its own 128 A rows and its
 // own 128-row half of B, so shared-memory traffic per FLOP drops by a third.
 //
-// Pair protocol (cluster of 2, leader = rank 0):
-//   producer (each CTA)  TMA of its A and B halves, completion counted on the
-//                        leader's `full` barrier (cta_group::2 load form; the
-//                        leader posts the expected bytes of both CTAs); its
-//                        scale atoms by bulk copy onto its own `sfdata` barrier.
-//   scale warps (each)   own TMEM scale slot via tcgen05.st, then arrive on the
-//                        leader's `sf_full` barrier (remote arrive for rank 1).
-//   MMA (leader only)    tcgen05.mma.cta_group::2 M=256 N=256 K=64 into both
-//                        CTAs' TMEM; commits multicast to both CTAs' `empty`
-//                        and `tfull` barriers.
-//   epilogue (each)      drains its own 128 accumulator rows, then arrives on
-//                        the leader's `tempty` barrier.
+// Pair protocol (cluster of 2, leader = rank 0), K in slabs of 256 (4 MMA
+// K-steps of 64), slabs in groups of two:
+//   producer (each CTA)  TMA (cta_group::2 form) of its A rows and its half of
+//                        B, completing on the leader's `full` barrier (the
+//                        leader posts both CTAs' bytes); TMA of its A-scale
+//                        atoms and of all 256 B rows' atoms onto its own
+//                        `sfull` barrier.
+//   TMEM warps (8/CTA)   scale factors: shared -> registers -> tcgen05.st into
+//                        this CTA's TMEM scale slot, one slot per group of two
+//                        slabs; the two slots alternate and each belongs to
+//                        one half of the warps (one warp per lane quarter),
+//                        which writes the group with one x64 and one x32
+//                        store and then arrives remotely on the leader's
+//                        `sf_ready`.  Few, wide stores per handshake keep the
+//                        tensor pipe fed; one slab per handshake measured
+//                        about 50% slower per slab.
+//                        Epilogue: read this CTA's 128x256 accumulator into
+//                        registers, release it on the leader's `tempty`, then
+//                        scale, convert and store while the next tile runs.
+//   MMA (leader only)    per group: wait `sf_ready`; per slab: wait `full`,
+//                        4 pair MMAs M=256 N=256 K=64, commit to both CTAs'
+//                        `empty`; after the group commit to both CTAs'
+//                        `sf_free`; after a tile commit to both CTAs' `tfull`.
+// TMEM: accumulator columns [0,256), scale slots [256,352) and [352,448).
 // No load uses cluster multicast.  Every wait is bounded.
 #include <cstdlib>
+#include <cstring>
 #include "common.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -31,8 +44,6 @@
 namespace nvfp4 {
 
 struct PairArgs {
-    const uint8_t *sfa;      // tiled scales of A (M rows)
-    const uint8_t *sfb;      // tiled scales of B (N rows)
     const float *ga;
     const float *gb;
     void *y;
@@ -40,8 +51,7 @@ struct PairArgs {
     int32_t M, N;
     int32_t num_k_steps;     // K / 64
     int32_t num_pm, num_qn;  // 256-row / 256-column pair tiles
-    int32_t a_row_tiles;     // ceil(M / 128)
-    int32_t b_row_tiles;     // ceil(N / 128)
+    int32_t tma_store;       // bf16 output written by TMA stores (needs N % 8 == 0)
     uint32_t *status;
     uint64_t timeout_ns;
 };
@@ -50,24 +60,61 @@ struct PairCfg {
     static constexpr int kAStage = 128 * 128;     // own 128 A rows x 128 bytes
     static constexpr int kBStage = 128 * 128;     // own 128-row half of B
     static constexpr int kSfaStage = 4 * 512;     // own rows' atoms, 4 K-steps
-    static constexpr int kSfbStage = 2 * 4 * 512; // all 256 N rows' atoms, 4 K-steps
-    static constexpr int kStageBytes = kAStage + kBStage + kSfaStage + kSfbStage;
+    static constexpr int kSfbStage = 2 * 4 * 512; // both B row tiles' atoms, 4 K-steps
+    static constexpr int kABBytes = kAStage + kBStage;
+    static constexpr int kSfBytes = kSfaStage + kSfbStage;
+    static constexpr int kStageBytes = kABBytes + kSfBytes;
     static constexpr int kStages = 5;
-    static constexpr int kSfCols = 16 + 32;       // TMEM scale columns per stage
-    static constexpr int kAccCols = 256;
-    static constexpr int kSfBase = kAccCols;
+    static constexpr int kSlabCols = 48;          // scale columns of one slab: 16 A + 32 B
+    static constexpr int kSlotCols = 2 * kSlabCols;
+    static constexpr int kSfCol = 256;            // first scale slot
     static constexpr int kTmemCols = 512;
-    static constexpr int kBarBytes = 8 * (4 * kStages + 4) + 16;
-    static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;
-    static constexpr int kThreads = 448;
-    static_assert(kSfBase + kStages * kSfCols <= kTmemCols, "tensor memory budget");
+    static constexpr int kTmemWarps = 8;
+    static constexpr int kThreads = 32 * (2 + kTmemWarps);
+    static constexpr int kStagingBytes = kTmemWarps * 32 * 128;   // per warp: 32 rows x 64 bf16
+    static constexpr int kBarBytes = 8 * (3 * kStages + 4 + 2) + 16;
+    static constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + kBarBytes + 1024;
+    static_assert(kSfCol + 2 * kSlotCols <= kTmemCols, "tensor memory budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 template <typename OutT>
-__global__ void __launch_bounds__(448, 1)
+__device__ __forceinline__ void pair_store_chunk(const uint32_t (&r)[32], float alpha, OutT *yrow,
+                                                 int q0, int N) {
+    if constexpr (sizeof(OutT) == 2) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * k]), alpha),
+                                                      __fmul_rn(__uint_as_float(r[2 * k + 1]), alpha));
+            pk[k] = *reinterpret_cast<uint32_t *>(&b2);
+        }
+        if (q0 + 32 <= N) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<uint4 *>(yrow + q0 + 8 * i) =
+                    make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if (q0 + 2 * i < N)
+                    reinterpret_cast<unsigned short *>(yrow)[q0 + 2 * i] = static_cast<unsigned short>(pk[i] & 0xffffu);
+                if (q0 + 2 * i + 1 < N)
+                    reinterpret_cast<unsigned short *>(yrow)[q0 + 2 * i + 1] = static_cast<unsigned short>(pk[i] >> 16);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (q0 + i < N) yrow[q0 + i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+    }
+}
+
+template <typename OutT>
+__global__ void __launch_bounds__(PairCfg::kThreads, 1)
 gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const __grid_constant__ PairArgs args) {
+                      const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                      const __grid_constant__ CUtensorMap tmY, const __grid_constant__ PairArgs args) {
     using C = PairCfg;
     constexpr int STAGES = C::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -76,13 +123,15 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     uint8_t *sB = sA + STAGES * C::kAStage;
     uint8_t *sSfa = sB + STAGES * C::kBStage;
     uint8_t *sSfb = sSfa + STAGES * C::kSfaStage;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sSfb + STAGES * C::kSfbStage);   // leader's
-    uint64_t *sfdata = full + STAGES;                                                // each CTA's
-    uint64_t *sf_full = sfdata + STAGES;                                             // leader's
-    uint64_t *empty = sf_full + STAGES;                                              // each CTA's
-    uint64_t *tfull = empty + STAGES;                                                // each CTA's
-    uint64_t *tempty = tfull + 2;                                                    // leader's
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tempty + 2);
+    uint8_t *staging = sSfb + STAGES * C::kSfbStage;                                 // 1024-aligned
+    uint64_t *full = reinterpret_cast<uint64_t *>(staging + C::kStagingBytes);       // leader's
+    uint64_t *sfull = full + STAGES;                                                 // each CTA's
+    uint64_t *empty = sfull + STAGES;                                                // each CTA's
+    uint64_t *sf_ready = empty + STAGES;                                             // leader's [2]
+    uint64_t *sf_free = sf_ready + 2;                                                // each CTA's [2]
+    uint64_t *tfull = sf_free + 2;                                                   // each CTA's
+    uint64_t *tempty = tfull + 1;                                                    // leader's
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tempty + 1);
     volatile uint32_t *abort_flag = tmem_holder + 1;
 
     const int warp = threadIdx.x >> 5;
@@ -93,16 +142,20 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmSA);
+        prefetch_tensormap(&tmSB);
+        if (args.tma_store) prefetch_tensormap(&tmY);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&sfdata[s], 1);
-            mbar_init(&sf_full[s], 8);     // one arrive per scale warp, both CTAs
+            mbar_init(&sfull[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&tfull[s], 1);
-            mbar_init(&tempty[s], 16);     // one arrive per epilogue warp, both CTAs
+            mbar_init(&sf_ready[s], C::kTmemWarps);       // the slot's 4 warps in both CTAs
+            mbar_init(&sf_free[s], 1);
         }
+        mbar_init(tfull, 1);
+        mbar_init(tempty, 2 * C::kTmemWarps);
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -116,45 +169,33 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     const int ncl = static_cast<int>(gridDim.x >> 1);
     const int num_tiles = args.num_pm * args.num_qn;
     const int num_kstages = (args.num_k_steps + 3) / 4;
+    const int num_groups = (num_kstages + 1) / 2;
 
     if (warp == 0) {
         if (lane == 0) {
             // -------------------------------------------------------- producer
             asm volatile("griddepcontrol.wait;" ::: "memory");
             const uint64_t pol = policy_evict_normal();
+            const uint32_t leader_full0 = mapa_shared(smem_addr(&full[0]), 0);
             uint32_t stage = 0, phase = 0;
             for (int tile = cid; tile < num_tiles; tile += ncl) {
                 const int pm = tile % args.num_pm;
                 const int qn = tile / args.num_pm;
                 const int a_rt = 2 * pm + static_cast<int>(rank);   // this CTA's A row tile
+                const int b_rt = 2 * qn + static_cast<int>(rank);   // this CTA's half of B
                 bool ok = true;
                 for (int ks = 0; ks < num_kstages; ++ks) {
-                    if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, args.timeout_ns, abort_flag, args.status)) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, args.timeout_ns, abort_flag, args.status)) {
                         ok = false;
                         break;
                     }
-                    const int nk = min(4, args.num_k_steps - 4 * ks);
-                    const uint32_t leader_full = mapa_shared(smem_addr(&full[stage]), 0);
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (C::kAStage + C::kBStage));
-                    tma_load_2d_pair(sA + stage * C::kAStage, &tmA, leader_full, ks * 128, a_rt * 128, pol);
-                    tma_load_2d_pair(sB + stage * C::kBStage, &tmB, leader_full, ks * 128,
-                                     (2 * qn + static_cast<int>(rank)) * 128, pol);
-                    uint32_t sf_bytes = 0;
-                    const bool have_a = a_rt < args.a_row_tiles;
-                    sf_bytes += have_a ? nk * 512 : 0;
-                    for (int q = 0; q < 2; ++q) sf_bytes += (2 * qn + q < args.b_row_tiles) ? nk * 512 : 0;
-                    mbar_arrive_expect_tx(&sfdata[stage], sf_bytes);
-                    if (have_a)
-                        bulk_load(sSfa + stage * C::kSfaStage,
-                                  args.sfa + (static_cast<int64_t>(a_rt) * args.num_k_steps + 4 * ks) * 512,
-                                  nk * 512, &sfdata[stage], pol);
-                    for (int q = 0; q < 2; ++q) {
-                        const int rt = 2 * qn + q;
-                        if (rt < args.b_row_tiles)
-                            bulk_load(sSfb + stage * C::kSfbStage + q * 2048,
-                                      args.sfb + (static_cast<int64_t>(rt) * args.num_k_steps + 4 * ks) * 512,
-                                      nk * 512, &sfdata[stage], pol);
-                    }
+                    const uint32_t bar = leader_full0 + 8u * stage;
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kABBytes);
+                    tma_load_2d_pair(sA + stage * C::kAStage, &tmA, bar, ks * 128, a_rt * 128, pol);
+                    tma_load_2d_pair(sB + stage * C::kBStage, &tmB, bar, ks * 128, b_rt * 128, pol);
+                    mbar_arrive_expect_tx(&sfull[stage], C::kSfBytes);
+                    tma_load_3d(sSfa + stage * C::kSfaStage, &tmSA, &sfull[stage], 0, 4 * ks, a_rt, pol);
+                    tma_load_3d(sSfb + stage * C::kSfbStage, &tmSB, &sfull[stage], 0, 4 * ks, 2 * qn, pol);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
@@ -165,131 +206,184 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             // -------------------------------------------------------- MMA issuer
             constexpr uint32_t idesc = make_idesc_nvf4_pair(256);
             const uint32_t a_base = smem_addr(sA), b_base = smem_addr(sB);
-            uint32_t stage = 0, phase = 0, acc_phase = 0;
-            for (int tile = cid; tile < num_tiles; tile += ncl) {
-                if (!mbar_wait_cluster(&tempty[0], acc_phase ^ 1u, args.timeout_ns, abort_flag, args.status)) break;
+            uint32_t stage = 0, phase = 0;
+            uint32_t gcount = 0;     // groups issued so far (slot = gcount & 1)
+            int t = 0;
+            bool ok = true;
+            for (int tile = cid; tile < num_tiles && ok; tile += ncl, ++t) {
+                // the previous tile's accumulator has been read out of TMEM
+                if (t > 0 && !mbar_wait(tempty, static_cast<uint32_t>(t - 1) & 1u, args.timeout_ns,
+                                                abort_flag, args.status))
+                    break;
                 tc_fence_after();
-                bool ok = true;
-                for (int ks = 0; ks < num_kstages; ++ks) {
-                    if (!mbar_wait_cluster(&full[stage], phase, args.timeout_ns, abort_flag, args.status) ||
-                        !mbar_wait_cluster(&sf_full[stage], phase, args.timeout_ns, abort_flag, args.status)) {
+                for (int g = 0; g < num_groups && ok; ++g, ++gcount) {
+                    const uint32_t slot = gcount & 1u;
+                    if (!mbar_wait(&sf_ready[slot], (gcount >> 1) & 1u, args.timeout_ns, abort_flag,
+                                           args.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int nk = min(4, args.num_k_steps - 4 * ks);
-                    const uint32_t sf = tmem_base + C::kSfBase + stage * C::kSfCols;
-                    for (int j = 0; j < nk; ++j) {
-                        const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage + 32 * j);
-                        const uint64_t bdesc = make_operand_desc(b_base + stage * C::kBStage + 32 * j);
-                        mma_nvf4_pair(tmem_base, adesc, bdesc, idesc, sf + 4 * j, sf + 16 + 8 * j,
-                                      (ks | j) != 0 ? 1u : 0u);
+                    for (int h = 0; h < 2; ++h) {
+                        const int ks = 2 * g + h;
+                        if (ks >= num_kstages) break;
+                        if (!mbar_wait(&full[stage], phase, args.timeout_ns, abort_flag, args.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const int nk = min(4, args.num_k_steps - 4 * ks);
+                        const uint32_t sf = tmem_base + C::kSfCol + slot * C::kSlotCols + h * C::kSlabCols;
+                        for (int j = 0; j < nk; ++j) {
+                            const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage + 32 * j);
+                            const uint64_t bdesc = make_operand_desc(b_base + stage * C::kBStage + 32 * j);
+                            mma_nvf4_pair(tmem_base, adesc, bdesc, idesc, sf + 4 * j, sf + 16 + 8 * j,
+                                          (ks | j) != 0 ? 1u : 0u);
+                        }
+                        tc_commit_pair(&empty[stage], 0x3);
+                        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                     }
-                    tc_commit_pair(&empty[stage], 0x3);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                    if (ok) tc_commit_pair(&sf_free[slot], 0x3);
                 }
-                if (!ok) break;
-                tc_commit_pair(&tfull[0], 0x3);
-                acc_phase ^= 1u;
+                if (ok) tc_commit_pair(tfull, 0x3);
             }
-        }
-    } else if (warp < 6) {
-        // ------------------------------------------------------------ scale warps
-        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        uint32_t stage = 0, phase = 0;
-        for (int tile = cid; tile < num_tiles; tile += ncl) {
-            bool ok = true;
-            for (int ks = 0; ks < num_kstages; ++ks) {
-                const bool got = mbar_wait(&sfdata[stage], phase, args.timeout_ns, abort_flag, args.status);
-                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-                const int nk = min(4, args.num_k_steps - 4 * ks);
-                const uint32_t sf = tmem_base + lane_off + C::kSfBase + stage * C::kSfCols;
-                const uint8_t *a_src = sSfa + stage * C::kSfaStage + lane * 16;
-                const uint8_t *b_src = sSfb + stage * C::kSfbStage + lane * 16;
-                // one 16-column and one 32-column TMEM store per stage (columns
-                // of K-steps a partial last stage does not have are never read)
-                uint32_t av[16], bv[32];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint4 a = ld_shared_v4(a_src + j * 512);
-                    const uint4 b0 = ld_shared_v4(b_src + j * 512);
-                    const uint4 b1 = ld_shared_v4(b_src + 2048 + j * 512);
-                    av[4 * j] = a.x; av[4 * j + 1] = a.y; av[4 * j + 2] = a.z; av[4 * j + 3] = a.w;
-                    bv[8 * j] = b0.x; bv[8 * j + 1] = b0.y; bv[8 * j + 2] = b0.z; bv[8 * j + 3] = b0.w;
-                    bv[8 * j + 4] = b1.x; bv[8 * j + 5] = b1.y; bv[8 * j + 6] = b1.z; bv[8 * j + 7] = b1.w;
-                }
-                (void)nk;
-                tmem_st_32x32b_x16(sf, av);
-                tmem_st_32x32b_x32(sf + 16, bv);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&sf_full[stage]), 0));
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-            }
-            if (!ok) break;
         }
     } else {
-        // ------------------------------------------------------------ epilogue
-        asm volatile("griddepcontrol.wait;" ::: "memory");
+        // ------------------------------------------------------------ TMEM warps
         const int quarter = warp & 3;
-        const int half = (warp - 6) >> 2;
+        const int half = (warp - 2) >> 2;         // which slab of a group this warp's scales cover
         const int row = quarter * 32 + lane;
-        const float alpha = __fmul_rn(*args.ga, *args.gb);
-        const uint32_t leader_tempty = mapa_shared(smem_addr(&tempty[0]), 0);
-        uint32_t acc_phase = 0;
-        for (int tile = cid; tile < num_tiles; tile += ncl) {
-            const int pm = tile % args.num_pm;
-            const int qn = tile / args.num_pm;
-            const bool ok = mbar_wait_cluster(&tfull[0], acc_phase, args.timeout_ns, abort_flag, args.status);
-            if (!__all_sync(0xffffffffu, ok)) break;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+        const uint32_t leader_ready0 = mapa_shared(smem_addr(&sf_ready[0]), 0);
+        const uint32_t leader_tempty = mapa_shared(smem_addr(tempty), 0);
+        float alpha = 0.0f;
+        bool alpha_ready = false;
+        uint32_t gcount = 0;
+        int t = 0;
+        bool ok = true;
+        // Epilogue of tile number te (this CTA's count), pair-tile index tile_e.
+        auto epilogue = [&](int te, int tile_e) -> bool {
+            const bool got = mbar_wait(tfull, static_cast<uint32_t>(te) & 1u, args.timeout_ns, abort_flag,
+                                               args.status);
+            if (!__all_sync(0xffffffffu, got)) return false;
             tc_fence_after();
-            const int p = pm * 256 + static_cast<int>(rank) * 128 + row;
-            const uint32_t tb = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + half * 128;
-            OutT *yrow = static_cast<OutT *>(args.y) + static_cast<int64_t>(p) * args.ldy;
-            uint32_t r[2][32];
-            tmem_ld_32x32b_x32(tb, r[0]);
-            tmem_ld_wait();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if (c + 1 < 4) tmem_ld_32x32b_x32(tb + (c + 1) * 32, r[(c + 1) & 1]);
-                const int q0 = qn * 256 + half * 128 + c * 32;
-                if (p < args.M) {
-                    if constexpr (sizeof(OutT) == 2) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[c & 1][2 * k]), alpha),
-                                                                      __fmul_rn(__uint_as_float(r[c & 1][2 * k + 1]), alpha));
-                            pk[k] = *reinterpret_cast<uint32_t *>(&b2);
-                        }
-                        if (q0 + 32 <= args.N) {
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                *reinterpret_cast<uint4 *>(yrow + q0 + 8 * i) =
-                                    make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                if (q0 + 2 * i < args.N)
-                                    reinterpret_cast<unsigned short *>(yrow)[q0 + 2 * i] = static_cast<unsigned short>(pk[i] & 0xffffu);
-                                if (q0 + 2 * i + 1 < args.N)
-                                    reinterpret_cast<unsigned short *>(yrow)[q0 + 2 * i + 1] = static_cast<unsigned short>(pk[i] >> 16);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (q0 + i < args.N) yrow[q0 + i] = __fmul_rn(__uint_as_float(r[c & 1][i]), alpha);
-                    }
-                }
-                if (c + 1 < 4) tmem_ld_wait();
+            if (!alpha_ready) {
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                alpha = __fmul_rn(*args.ga, *args.gb);
+                alpha_ready = true;
             }
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(lane_base + half * 128 + c * 32, r[c]);
+            tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(leader_tempty);
-            acc_phase ^= 1u;
+            if (lane == 0) mbar_arrive_remote(leader_tempty);
+            const int pm = tile_e % args.num_pm;
+            const int qn = tile_e / args.num_pm;
+            if (sizeof(OutT) == 2 && args.tma_store) {
+                // bf16: stage 32 rows x 64 columns at a time (128-byte swizzle,
+                // 16-byte chunk c of row r at chunk c ^ (r % 8)) and let one
+                // TMA store write it; rows and columns past M and N are clipped
+                // (exactly, because rows are whole 16-byte units when N % 8 == 0).
+                uint8_t *stg = staging + (warp - 2) * (32 * 128);
+                const int row0 = pm * 256 + static_cast<int>(rank) * 128 + quarter * 32;
+                const int col0 = qn * 256 + half * 128;
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    if (lane == 0) bulk_wait_group_read0();   // staging buffer free again
+                    __syncwarp();
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint32_t *src = r[2 * c2 + (ch >> 2)] + (ch & 3) * 8;
+                        uint32_t w[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(src[2 * k]), alpha),
+                                                                      __fmul_rn(__uint_as_float(src[2 * k + 1]), alpha));
+                            w[k] = *reinterpret_cast<uint32_t *>(&b2);
+                        }
+                        st_shared_v4(stg + lane * 128 + ((ch ^ (lane & 7)) * 16), w[0], w[1], w[2], w[3]);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    // a box wholly past the last row or column is not issued
+                    if (lane == 0 && row0 < args.M && col0 + 64 * c2 < args.N) {
+                        tma_store_2d(&tmY, stg, col0 + 64 * c2, row0);
+                        bulk_commit_group();
+                    }
+                }
+            } else {
+                const int p = pm * 256 + static_cast<int>(rank) * 128 + row;
+                if (p < args.M) {
+                    OutT *yrow = static_cast<OutT *>(args.y) + static_cast<int64_t>(p) * args.ldy;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        pair_store_chunk<OutT>(r[c], alpha, yrow, qn * 256 + half * 128 + c * 32, args.N);
+                }
+            }
+            return true;
+        };
+        uint32_t sstage = 0, sphase = 0;   // scale-ring position of the next slab
+        int prev_tile = -1;
+        for (int tile = cid; tile < num_tiles && ok; tile += ncl, ++t) {
+            for (int g = 0; g < num_groups; ++g, ++gcount) {
+                const uint32_t slot = gcount & 1u;
+                const int nslab = min(2, num_kstages - 2 * g);
+                // slot h belongs to the warps of half h: one x64 and one x32
+                // store write both slabs' scales of the group for this lane quarter
+                if (slot == static_cast<uint32_t>(half)) {
+                    const bool freed = mbar_wait(&sf_free[slot], ((gcount >> 1) & 1u) ^ 1u, args.timeout_ns,
+                                                         abort_flag, args.status);
+                    if (!__all_sync(0xffffffffu, freed)) { ok = false; break; }
+                    tc_fence_after();
+                    uint32_t v[2 * C::kSlabCols];
+                    uint32_t st_i = sstage, ph_i = sphase;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (h < nslab) {
+                            const bool got = mbar_wait(&sfull[st_i], ph_i, args.timeout_ns, abort_flag, args.status);
+                            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                            const uint8_t *a_src = sSfa + st_i * C::kSfaStage + lane * 16;
+                            const uint8_t *b_src = sSfb + st_i * C::kSfbStage + lane * 16;
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const uint4 a = ld_shared_v4(a_src + j * 512);
+                                const uint4 b0 = ld_shared_v4(b_src + j * 512);
+                                const uint4 b1 = ld_shared_v4(b_src + 2048 + j * 512);
+                                uint32_t *va = v + h * C::kSlabCols + 4 * j;
+                                uint32_t *vb = v + h * C::kSlabCols + 16 + 8 * j;
+                                va[0] = a.x; va[1] = a.y; va[2] = a.z; va[3] = a.w;
+                                vb[0] = b0.x; vb[1] = b0.y; vb[2] = b0.z; vb[3] = b0.w;
+                                vb[4] = b1.x; vb[5] = b1.y; vb[6] = b1.z; vb[7] = b1.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < C::kSlabCols; ++i) v[h * C::kSlabCols + i] = 0u;   // never read
+                        }
+                        if (++st_i == STAGES) { st_i = 0; ph_i ^= 1u; }
+                    }
+                    if (!ok) break;
+                    const uint32_t sf = lane_base + C::kSfCol + slot * C::kSlotCols;
+                    tmem_st_32x32b_x64(sf, *reinterpret_cast<const uint32_t(*)[64]>(v));
+                    tmem_st_32x32b_x32(sf + 64, *reinterpret_cast<const uint32_t(*)[32]>(v + 64));
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(leader_ready0 + 8u * slot);
+                }
+                for (int h = 0; h < nslab; ++h)
+                    if (++sstage == STAGES) { sstage = 0; sphase ^= 1u; }
+                // once the first group of this tile is handed over, drain the previous tile
+                if (g == 0 && prev_tile >= 0) {
+                    if (!epilogue(t - 1, prev_tile)) { ok = false; break; }
+                    prev_tile = -1;
+                }
+            }
+            if (ok) prev_tile = tile;
         }
+        if (ok && prev_tile >= 0) epilogue(t - 1, prev_tile);
+        if (lane == 0) bulk_wait_group0();   // this warp's output stores are complete
     }
 
     tc_fence_before();
@@ -309,24 +403,31 @@ template <typename OutT>
 static cudaError_t run_pair(const Operand &act, const Operand &wgt, int64_t K, void *y, int64_t ldy,
                             uint32_t *status, uint64_t timeout_ns, int max_clusters, cudaStream_t stream) {
     using C = PairCfg;
-    CUtensorMap tmA, tmB;
+    const uint64_t k_steps = static_cast<uint64_t>(K / 64);
+    CUtensorMap tmA, tmB, tmSA, tmSB;
     if (encode_tensor_map_u8(&tmA, act.codes, K / 2, act.rows, 128, 128) != CUDA_SUCCESS ||
-        encode_tensor_map_u8(&tmB, wgt.codes, K / 2, wgt.rows, 128, 128) != CUDA_SUCCESS)
+        encode_tensor_map_u8(&tmB, wgt.codes, K / 2, wgt.rows, 128, 128) != CUDA_SUCCESS ||
+        encode_scale_map(&tmSA, act.scales, k_steps, ceil_div(act.rows, 128), 1) != CUDA_SUCCESS ||
+        encode_scale_map(&tmSB, wgt.scales, k_steps, ceil_div(wgt.rows, 128), 2) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    CUtensorMap tmY;
+    memset(&tmY, 0, sizeof(tmY));    // unused unless tma_store
+    const bool tma_store = sizeof(OutT) == 2 && wgt.rows % 8 == 0;
+    if (tma_store &&
+        encode_output_map_bf16(&tmY, y, static_cast<uint64_t>(act.rows), static_cast<uint64_t>(wgt.rows),
+                               static_cast<uint64_t>(ldy), 64, 32) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     PairArgs a;
-    a.sfa = act.scales;
-    a.sfb = wgt.scales;
     a.ga = act.g;
     a.gb = wgt.g;
     a.y = y;
     a.ldy = ldy;
     a.M = static_cast<int32_t>(act.rows);
     a.N = static_cast<int32_t>(wgt.rows);
-    a.num_k_steps = static_cast<int32_t>(K / 64);
+    a.num_k_steps = static_cast<int32_t>(k_steps);
     a.num_pm = static_cast<int32_t>(ceil_div(act.rows, 256));
     a.num_qn = static_cast<int32_t>(ceil_div(wgt.rows, 256));
-    a.a_row_tiles = static_cast<int32_t>(ceil_div(act.rows, 128));
-    a.b_row_tiles = static_cast<int32_t>(ceil_div(wgt.rows, 128));
+    a.tma_store = tma_store ? 1 : 0;
     a.status = status;
     a.timeout_ns = timeout_ns;
     const int tiles = a.num_pm * a.num_qn;
@@ -348,7 +449,7 @@ static cudaError_t run_pair(const Operand &act, const Operand &wgt, int64_t K, v
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<OutT>, tmA, tmB, a);
+    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<OutT>, tmA, tmB, tmSA, tmSB, tmY, a);
 }
 
 // How many 2-CTA clusters of the pair kernel can be resident at once (0 if
@@ -382,12 +483,12 @@ static int pair_max_clusters() {
 }
 
 bool pair_gemm_usable(int64_t M, int64_t N, int num_sms) {
-    // Opt-in (NVFP4_GEMM_CTA_PAIR=1): on the shapes measured so far the
-    // one-CTA kernel is faster, so the pair kernel is not the default.
+    // NVFP4_GEMM_CTA_PAIR=0 keeps every shape on the one-CTA kernel.
     const char *opt = getenv("NVFP4_GEMM_CTA_PAIR");
-    if (opt == nullptr || opt[0] != '1') return false;
+    if (opt != nullptr && opt[0] == '0') return false;
     const int maxc = pair_max_clusters();
-    return maxc > 0 && M >= 256 && ceil_div(M, 256) * ceil_div(N, 256) >= 2 * maxc && num_sms > 0;
+    // every resident pair gets at least one 256x256 tile
+    return maxc > 0 && num_sms > 0 && M >= 256 && ceil_div(M, 256) * ceil_div(N, 256) >= maxc;
 }
 
 cudaError_t launch_gemm_pair(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,

@@ -46,4 +46,14 @@ cudaError_t launch_wait_selftest(uint32_t *status, uint64_t timeout_ns, cudaStre
 CUresult encode_tensor_map_u8(CUtensorMap *map, const void *base, uint64_t inner_bytes,
                               uint64_t rows, uint32_t box_inner, uint32_t box_rows);
 
+// Tensor map over a tiled scale array: [row_tiles][k_steps][512-byte atom],
+// box = 4 K-steps x box_tiles row tiles (zero fill past either edge).
+CUresult encode_scale_map(CUtensorMap *map, const void *scales, uint64_t k_steps, uint64_t row_tiles,
+                          uint32_t box_tiles);
+
+// Tensor map over a bf16 output y[rows][cols] with row pitch ld elements,
+// 128-byte swizzled boxes of box_rows x box_cols (box_cols * 2 <= 128).
+CUresult encode_output_map_bf16(CUtensorMap *map, void *y, uint64_t rows, uint64_t cols, uint64_t ld,
+                                uint32_t box_cols, uint32_t box_rows);
+
 }  // namespace nvfp4

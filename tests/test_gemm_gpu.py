@@ -31,9 +31,10 @@ def quantize_gpu(nv, x):
 
 
 def run_gemm(nv, a, b, out_dtype):
-    # rows of y must start on 16-byte boundaries: pad the pitch, then slice
+    # rows of y must start on 16-byte boundaries: pad the pitch (always by at
+    # least one 16-byte unit, so that writes past N would be seen), then slice
     per16 = 16 // torch.empty((), dtype=out_dtype).element_size()
-    ldy = -(-b.rows // per16) * per16
+    ldy = -(-b.rows // per16) * per16 + per16
     buf = torch.full((a.rows, ldy), float("nan"), dtype=out_dtype, device="cuda")
     y = buf[:, :b.rows]
     ws = nv.workspace(nv.OP_GEMM, a.rows, b.rows, a.cols)
@@ -114,12 +115,13 @@ def test_gemm_wide_tiles(nv):
 
 
 @pytest.mark.parametrize("pair", ["0", "1"])
-@pytest.mark.parametrize("M,N,K", [(2304, 4608, 256), (2000, 4700, 320)])
+@pytest.mark.parametrize("M,N,K", [(2304, 4608, 256), (2000, 4700, 320), (1900, 4616, 256)])
 def test_gemm_cta_pair_tiles(nv, M, N, K, pair, monkeypatch):
-    """Shapes large enough for the two-CTA 256x256 tiles (switched on with
-    NVFP4_GEMM_CTA_PAIR=1), including ragged M (the second CTA of the last row
-    pair partly or wholly outside), ragged N and a partial last K slab; sampled
-    outputs plus the last row and column, for both the pair and one-CTA paths."""
+    """Shapes large enough for the two-CTA 256x256 tiles (NVFP4_GEMM_CTA_PAIR=0
+    keeps them on the one-CTA kernel), including ragged M (the second CTA of
+    the last row pair partly or wholly outside), ragged N with and without
+    N % 8 == 0 (TMA-store and per-row-store epilogues) and a partial last K
+    slab; sampled outputs plus the last row and column, for both kernels."""
     monkeypatch.setenv("NVFP4_GEMM_CTA_PAIR", pair)
     rng = np.random.default_rng(M + N)
     x = rng.standard_normal((M, K)).astype(np.float32)
