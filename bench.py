@@ -158,7 +158,7 @@ class Prefill:
         self.flops = 2.0 * self.M * self.N * self.K
         self.units = self.flops / 1e12          # TFLOP per step
         self.launches = 3                       # amax, encode, GEMM
-        self.dominant = {"kernel": "gemm_nvf4_kernel (128x256 tiles)", "bound": "tensor",
+        self.dominant = {"kernel": "gemm_nvf4_pair_kernel (CTA pair, 256x256 tiles)", "bound": "tensor",
                          "algorithmic": self.flops, "unit": "TFLOP/s"}
         self.config = {"workload": f"prefill W4A4 linear: quantize X bf16 {self.M}x{self.K} per call, "
                                    f"GEMM with pre-quantized W {self.N}x{self.K}, bf16 out",
