@@ -102,15 +102,17 @@ size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K) {
     case NVFP4_OP_QUANTIZE:
         return kQuantizeWs;
     case NVFP4_OP_DEQUANTIZE:
-    case NVFP4_OP_GEMM:
         return kWsStatusBytes;
+    case NVFP4_OP_GEMM:
+        // status | stream-K scratch
+        return kWsStatusBytes + splitk_ws_bytes(M, N);
     case NVFP4_OP_LINEAR_FUSED:
-        // partials | x_q (codes, scales, g)
-        return kQuantizeWs + quantized_bytes(M, K);
+        // status, partials | x_q (codes, scales, g) | stream-K scratch
+        return kQuantizeWs + quantized_bytes(M, K) + splitk_ws_bytes(M, N);
     case NVFP4_OP_LINEAR_FUSED_SILU:
-        // partials | x_q | gate, up, h (fp32 [M][N] each)
+        // status, partials | x_q | gate, up, h (fp32 [M][N] each) | stream-K scratch
         return kQuantizeWs + quantized_bytes(M, K) +
-               3 * align256(static_cast<size_t>(M * N) * sizeof(float));
+               3 * align256(static_cast<size_t>(M * N) * sizeof(float)) + splitk_ws_bytes(M, N);
     }
     return 0;
 }
@@ -169,7 +171,7 @@ static nvfp4_status check_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, voi
 // programmatic dependency, so every earlier writer of b has finished).
 static nvfp4_status gemm_impl(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y,
                               nvfp4_dtype yt, int64_t ldy, uint32_t *status, int num_sms,
-                              cudaStream_t stream, bool weights_ready = false) {
+                              cudaStream_t stream, bool weights_ready, void *splitk) {
     if (a->rows == 0 || b->rows == 0) return NVFP4_OK;
     if (a->cols == 0)   // empty reduction: y = 0
         return from_cuda(cudaMemset2DAsync(y, ldy * (yt == NVFP4_BF16 ? 2 : 4), 0,
@@ -177,18 +179,19 @@ static nvfp4_status gemm_impl(const nvfp4_tensor *a, const nvfp4_tensor *b, void
     Operand act{a->codes, a->scales, a->tensor_scale, a->rows};
     Operand wgt{b->codes, b->scales, b->tensor_scale, b->rows};
     return from_cuda(launch_gemm(act, wgt, a->cols, y, yt == NVFP4_BF16, ldy, status, timeout_ns(),
-                                 num_sms, stream, weights_ready));
+                                 num_sms, stream, weights_ready, splitk));
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y, nvfp4_dtype yt,
                         int64_t ldy, void *ws, size_t ws_bytes, nvfp4_stream_t stream) {
     nvfp4_status st = check_gemm(a, b, y, yt, ldy);
     if (st != NVFP4_OK) return st;
-    if ((st = check_ws(ws, ws_bytes, kWsStatusBytes)) != NVFP4_OK) return st;
+    const size_t sk = splitk_ws_bytes(a->rows, b->rows);
+    if ((st = check_ws(ws, ws_bytes, kWsStatusBytes + sk)) != NVFP4_OK) return st;
     DevInfo dev;
     if ((st = current_device(&dev)) != NVFP4_OK) return st;
     return gemm_impl(a, b, y, yt, ldy, static_cast<uint32_t *>(ws), dev.sms,
-                     reinterpret_cast<cudaStream_t>(stream));
+                     reinterpret_cast<cudaStream_t>(stream), false, sk ? ws_at(ws, kWsStatusBytes) : nullptr);
 }
 
 nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_t K, int64_t ldx,
@@ -245,17 +248,20 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
                                     dev.sms, stream);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     uint32_t *status = static_cast<uint32_t *>(ws);
+    const bool has_sk = splitk_ws_bytes(M, N) != 0;
+    const size_t mn = align256(static_cast<size_t>(M * N) * sizeof(float));
     if (epilogue == NVFP4_EPI_STORE)
-        return gemm_impl(&xq, w, y, yt, ldy, status, dev.sms, stream, true);
+        return gemm_impl(&xq, w, y, yt, ldy, status, dev.sms, stream, true,
+                         has_sk ? ws_at(ws, kQuantizeWs + quantized_bytes(M, K)) : nullptr);
 
     // SiLU(gate) * up, then re-quantize h for the down projection.
-    const size_t mn = align256(static_cast<size_t>(M * N) * sizeof(float));
     float *gate = reinterpret_cast<float *>(ws_at(ws, off));
     float *up = reinterpret_cast<float *>(ws_at(ws, off + mn));
     float *h = y ? static_cast<float *>(y) : reinterpret_cast<float *>(ws_at(ws, off + 2 * mn));
     const int64_t ldh = y ? ldy : N;
-    if ((st = gemm_impl(&xq, w, gate, NVFP4_F32, N, status, dev.sms, stream, true)) != NVFP4_OK) return st;
-    if ((st = gemm_impl(&xq, w_up, up, NVFP4_F32, N, status, dev.sms, stream, true)) != NVFP4_OK) return st;
+    void *sk = has_sk ? ws_at(ws, kQuantizeWs + quantized_bytes(M, K) + 3 * mn) : nullptr;
+    if ((st = gemm_impl(&xq, w, gate, NVFP4_F32, N, status, dev.sms, stream, true, sk)) != NVFP4_OK) return st;
+    if ((st = gemm_impl(&xq, w_up, up, NVFP4_F32, N, status, dev.sms, stream, true, sk)) != NVFP4_OK) return st;
     if (ldh == N) {
         if (launch_silu_mul(gate, up, h, M * N, dev.sms, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
     } else {

@@ -35,6 +35,7 @@
 // activation quantizer.
 // Every wait is bounded; a timeout sets the status word and winds the CTA
 // down without leaving tensor memory allocated.
+#include <cstdlib>
 #include "common.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -54,8 +55,52 @@ struct GemmArgs {
     int32_t q_row_tiles;     // ceil(Q / 128): 128-row scale tiles of B
     int32_t preload;         // stages of the weight operand loaded before the PDL wait
     int32_t weights_are_a;   // 1: the weights are the MMA A operand (swapped)
+    int32_t streamk;         // 1: CTAs take equal contiguous runs of (tile, K slab) units
+    int32_t q_pad;           // row pitch (floats) of acc_ws: num_q_tiles * BN
+    float *acc_ws;           // stream-K: fp32 partial sums [num_p_tiles*128][q_pad], zero between calls
+    int32_t *tile_cnt;       // stream-K: K slabs added per tile so far, zero between calls
     uint32_t *status;
     uint64_t timeout_ns;
+};
+
+// One CTA's work item: K slabs [ks0, ks1) of one output tile.
+struct Seg {
+    int tile, ks0, ks1;
+};
+
+// The sequence of work items of this CTA; every role walks the same sequence.
+// Tile mode: whole tiles blockIdx.x, blockIdx.x + gridDim.x, ...  Stream-K
+// mode: the CTA's equal share of the tiles x K-slabs units, in tile-major
+// order, cut at tile boundaries (at most a partial first and last tile).
+struct SegIter {
+    int64_t u, end;
+    int nks, tile, tstep, ntiles;
+    bool sk;
+    __device__ SegIter(const GemmArgs &a, int num_tiles, int num_kstages)
+        : u(0), end(0), nks(num_kstages), tile(static_cast<int>(blockIdx.x)), tstep(static_cast<int>(gridDim.x)),
+          ntiles(num_tiles), sk(a.streamk != 0) {
+        if (sk) {
+            const int64_t T = static_cast<int64_t>(num_tiles) * num_kstages;
+            u = T * blockIdx.x / gridDim.x;
+            end = T * (blockIdx.x + 1) / gridDim.x;
+        }
+    }
+    __device__ bool next(Seg &s) {
+        if (sk) {
+            if (u >= end) return false;
+            s.tile = static_cast<int>(u / nks);
+            s.ks0 = static_cast<int>(u % nks);
+            s.ks1 = static_cast<int>(min(static_cast<int64_t>(nks), s.ks0 + (end - u)));
+            u += s.ks1 - s.ks0;
+            return true;
+        }
+        if (tile >= ntiles) return false;
+        s.tile = tile;
+        s.ks0 = 0;
+        s.ks1 = nks;
+        tile += tstep;
+        return true;
+    }
 };
 
 template <int BN>
@@ -73,7 +118,7 @@ struct GemmCfg {
     static constexpr int kColsUsed = kSfBase + kStages * kSfCols;
     static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
-    static constexpr int kBarBytes = 8 * (3 * kStages + 4) + 16;
+    static constexpr int kBarBytes = 8 * (3 * kStages + 6) + 16;
     static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;   // + alignment slack
     static constexpr int kThreads = 448;                       // 14 warps
     static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -98,8 +143,11 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     uint64_t *empty = sf_full + STAGES;
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tempty + 2);
+    uint64_t *epi_done = tempty + 2;                    // stream-K: epilogue warps' partial sums added
+    uint64_t *epi_flag = epi_done + 1;                  // stream-K: last_flag published
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(epi_flag + 1);
     volatile uint32_t *abort_flag = tmem_holder + 1;
+    volatile uint32_t *last_flag = tmem_holder + 2;     // stream-K: this CTA completes the tile
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -116,6 +164,8 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             mbar_init(&tfull[s], 1);
             mbar_init(&tempty[s], 8);      // one arrive per epilogue warp
         }
+        mbar_init(epi_done, 8);
+        mbar_init(epi_flag, 1);
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -134,105 +184,74 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const uint64_t pol_a = SWAP ? policy_evict_first() : policy_evict_normal();
             const uint64_t pol_b = SWAP ? policy_evict_last() : policy_evict_normal();
             // The weights may be streamed before the dependent-launch wait for
-            // the first `pre` stages of this CTA's first tile.
-            const int pre = (static_cast<int>(blockIdx.x) < num_tiles) ? min(args.preload, min(STAGES, num_kstages)) : 0;
-            uint32_t stage = 0, phase = 0;
+            // the first `pre` stages of this CTA's first work item.
+            Seg first{0, 0, 0};
+            const bool has_first = SegIter(args, num_tiles, num_kstages).next(first);
+            const int pre = has_first ? min(args.preload, min(STAGES, first.ks1 - first.ks0)) : 0;
+            const int pt0 = first.tile % args.num_p_tiles;
+            const int qt0 = first.tile / args.num_p_tiles;
+            auto load_a = [&](uint32_t st, int pt, int ks, int nk) {
+                tma_load_2d(sA + st * C::kAStage, &tmA, &full[st], ks * 128, pt * 128, pol_a);
+                bulk_load(sSfa + st * C::kSfaStage,
+                          args.sfa + (static_cast<int64_t>(pt) * args.num_k_steps + 4 * ks) * 512,
+                          nk * 512, &full[st], pol_a);
+            };
+            auto load_b = [&](uint32_t st, int qt, int ks, int nk) {
+                tma_load_2d(sB + st * C::kBStage, &tmB, &full[st], ks * 128, qt * BN, pol_b);
+                for (int q = 0; q < C::kNQT; ++q) {
+                    const int rt = qt * C::kNQT + q;
+                    if (rt < args.q_row_tiles)
+                        bulk_load(sSfb + st * C::kSfbStage + q * 2048,
+                                  args.sfb + (static_cast<int64_t>(rt) * args.num_k_steps + 4 * ks) * 512,
+                                  nk * 512, &full[st], pol_b);
+                }
+            };
             bool waited = (pre == 0);
             if (waited) asm volatile("griddepcontrol.wait;" ::: "memory");
+            // after the wait: the dependent operand of the preloaded stages
+            // (stages 0..pre-1 = K slabs first.ks0 .. first.ks0+pre-1)
+            auto finish_preload = [&]() {
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                waited = true;
+                for (int p = 0; p < pre; ++p) {
+                    const int ks = first.ks0 + p;
+                    const int nk = min(4, args.num_k_steps - 4 * ks);
+                    if (args.weights_are_a) load_b(static_cast<uint32_t>(p), qt0, ks, nk);
+                    else load_a(static_cast<uint32_t>(p), pt0, ks, nk);
+                }
+            };
+            uint32_t stage = 0, phase = 0;
             int it = 0;   // stage index within this CTA's work
-            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-                const int pt = tile % args.num_p_tiles;
-                const int qt = tile / args.num_p_tiles;
-                bool ok = true;
+            SegIter segs(args, num_tiles, num_kstages);
+            Seg sg;
+            bool ok = true;
+            while (ok && segs.next(sg)) {
+                const int pt = sg.tile % args.num_p_tiles;
+                const int qt = sg.tile / args.num_p_tiles;
                 int nq_loaded = 0;
                 for (int q = 0; q < C::kNQT; ++q) nq_loaded += (qt * C::kNQT + q < args.q_row_tiles);
-                for (int ks = 0; ks < num_kstages; ++ks, ++it) {
+                for (int ks = sg.ks0; ks < sg.ks1; ++ks, ++it) {
                     const int nk = min(4, args.num_k_steps - 4 * ks);
                     const uint32_t bytes = C::kAStage + C::kBStage + nk * 512 * (1 + nq_loaded);
-                    auto load_a = [&]() {
-                        tma_load_2d(sA + stage * C::kAStage, &tmA, &full[stage], ks * 128, pt * 128, pol_a);
-                        bulk_load(sSfa + stage * C::kSfaStage,
-                                  args.sfa + (static_cast<int64_t>(pt) * args.num_k_steps + 4 * ks) * 512,
-                                  nk * 512, &full[stage], pol_a);
-                    };
-                    auto load_b = [&]() {
-                        tma_load_2d(sB + stage * C::kBStage, &tmB, &full[stage], ks * 128, qt * BN, pol_b);
-                        for (int q = 0; q < C::kNQT; ++q) {
-                            const int rt = qt * C::kNQT + q;
-                            if (rt < args.q_row_tiles)
-                                bulk_load(sSfb + stage * C::kSfbStage + q * 2048,
-                                          args.sfb + (static_cast<int64_t>(rt) * args.num_k_steps + 4 * ks) * 512,
-                                          nk * 512, &full[stage], pol_b);
-                        }
-                    };
                     if (it < pre) {
                         // fresh stage (first pass over the ring): no empty wait needed
                         mbar_arrive_expect_tx(&full[stage], bytes);
-                        if (args.weights_are_a) load_a(); else load_b();
+                        if (args.weights_are_a) load_a(stage, pt, ks, nk);
+                        else load_b(stage, qt, ks, nk);
                     } else {
-                        if (!waited) {
-                            // finish the preloaded stages with the dependent operand
-                            asm volatile("griddepcontrol.wait;" ::: "memory");
-                            waited = true;
-                            for (int p = 0; p < pre; ++p) {
-                                // the preloaded stages are stages 0..pre-1 of the first tile
-                                const int ks0 = p;
-                                const int nk0 = min(4, args.num_k_steps - 4 * ks0);
-                                const int pt0 = static_cast<int>(blockIdx.x) % args.num_p_tiles;
-                                const int qt0 = static_cast<int>(blockIdx.x) / args.num_p_tiles;
-                                if (args.weights_are_a) {
-                                    tma_load_2d(sB + p * C::kBStage, &tmB, &full[p], ks0 * 128, qt0 * BN, pol_b);
-                                    for (int q = 0; q < C::kNQT; ++q) {
-                                        const int rt = qt0 * C::kNQT + q;
-                                        if (rt < args.q_row_tiles)
-                                            bulk_load(sSfb + p * C::kSfbStage + q * 2048,
-                                                      args.sfb + (static_cast<int64_t>(rt) * args.num_k_steps + 4 * ks0) * 512,
-                                                      nk0 * 512, &full[p], pol_b);
-                                    }
-                                } else {
-                                    tma_load_2d(sA + p * C::kAStage, &tmA, &full[p], ks0 * 128, pt0 * 128, pol_a);
-                                    bulk_load(sSfa + p * C::kSfaStage,
-                                              args.sfa + (static_cast<int64_t>(pt0) * args.num_k_steps + 4 * ks0) * 512,
-                                              nk0 * 512, &full[p], pol_a);
-                                }
-                            }
-                        }
+                        if (!waited) finish_preload();
                         if (!mbar_wait(&empty[stage], phase ^ 1u, args.timeout_ns, abort_flag, args.status)) {
                             ok = false;
                             break;
                         }
                         mbar_arrive_expect_tx(&full[stage], bytes);
-                        load_a();
-                        load_b();
+                        load_a(stage, pt, ks, nk);
+                        load_b(stage, qt, ks, nk);
                     }
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                if (!ok) break;
             }
-            if (!waited) {
-                // everything fit in the preload: issue the dependent halves now
-                asm volatile("griddepcontrol.wait;" ::: "memory");
-                for (int p = 0; p < pre; ++p) {
-                    const int nk0 = min(4, args.num_k_steps - 4 * p);
-                    const int pt0 = static_cast<int>(blockIdx.x) % args.num_p_tiles;
-                    const int qt0 = static_cast<int>(blockIdx.x) / args.num_p_tiles;
-                    if (args.weights_are_a) {
-                        tma_load_2d(sB + p * C::kBStage, &tmB, &full[p], p * 128, qt0 * BN, pol_b);
-                        for (int q = 0; q < C::kNQT; ++q) {
-                            const int rt = qt0 * C::kNQT + q;
-                            if (rt < args.q_row_tiles)
-                                bulk_load(sSfb + p * C::kSfbStage + q * 2048,
-                                          args.sfb + (static_cast<int64_t>(rt) * args.num_k_steps + 4 * p) * 512,
-                                          nk0 * 512, &full[p], pol_b);
-                        }
-                    } else {
-                        tma_load_2d(sA + p * C::kAStage, &tmA, &full[p], p * 128, pt0 * 128, pol_a);
-                        bulk_load(sSfa + p * C::kSfaStage,
-                                  args.sfa + (static_cast<int64_t>(pt0) * args.num_k_steps + 4 * p) * 512,
-                                  nk0 * 512, &full[p], pol_a);
-                    }
-                }
-            }
+            if (!waited) finish_preload();   // everything fit in the preload
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -240,12 +259,14 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             constexpr uint32_t idesc = make_idesc_nvf4(BN);
             const uint32_t a_base = smem_addr(sA), b_base = smem_addr(sB);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            SegIter segs(args, num_tiles, num_kstages);
+            Seg sg;
+            while (segs.next(sg)) {
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.timeout_ns, abort_flag, args.status)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
                 bool ok = true;
-                for (int ks = 0; ks < num_kstages; ++ks) {
+                for (int ks = sg.ks0; ks < sg.ks1; ++ks) {
                     if (!mbar_wait(&full[stage], phase, args.timeout_ns, abort_flag, args.status) ||
                         !mbar_wait(&sf_full[stage], phase, args.timeout_ns, abort_flag, args.status)) {
                         ok = false;
@@ -258,7 +279,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage + 32 * j);
                         const uint64_t bdesc = make_operand_desc(b_base + stage * C::kBStage + 32 * j);
                         mma_nvf4(d_tmem, adesc, bdesc, idesc, sf + 4 * j, sf + 16 + 4 * C::kNQT * j,
-                                 (ks | j) != 0 ? 1u : 0u);
+                                 (ks != sg.ks0 || j != 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -279,9 +300,22 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // atom: columns c = 0..3 hold rows 32c + l, bytes = the 4 K-blocks.
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         uint32_t stage = 0, phase = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        uint32_t pend[2];
+        int npend = 0;
+        auto flush = [&]() {
+            if (npend == 0) return;
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                for (int i = 0; i < npend; ++i) mbar_arrive(&sf_full[pend[i]]);
+            npend = 0;
+        };
+        SegIter segs(args, num_tiles, num_kstages);
+        Seg sg;
+        while (segs.next(sg)) {
             bool ok = true;
-            for (int ks = 0; ks < num_kstages; ++ks) {
+            for (int ks = sg.ks0; ks < sg.ks1; ++ks) {
                 const bool got = mbar_wait(&full[stage], phase, args.timeout_ns, abort_flag, args.status);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 const int nk = min(4, args.num_k_steps - 4 * ks);
@@ -309,14 +343,16 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     tmem_st_32x32b_x16(sf + 16, reinterpret_cast<uint32_t(&)[16]>(bv));
                 else
                     tmem_st_32x32b_x32(sf + 16, reinterpret_cast<uint32_t(&)[32]>(bv));
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sf_full[stage]);
+                // Hand stages over two at a time: one store-completion wait and
+                // handshake per pair keeps the MMA fed (one per stage left the
+                // tensor pipe waiting on the handshake's latency).
+                pend[npend++] = stage;
+                if (npend == 2) flush();
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
         }
+        flush();
     } else {
         // ------------------------------------------------------------ epilogue
         asm volatile("griddepcontrol.wait;" ::: "memory");   // tensor scales may be fresh
@@ -326,16 +362,135 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const float alpha = __fmul_rn(*args.ga, *args.gb);
         constexpr bool kFastDrain = !SWAP && sizeof(OutT) == 2 && BN >= 64;
         uint32_t acc = 0, acc_phase = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            const int pt = tile % args.num_p_tiles;
-            const int qt = tile / args.num_p_tiles;
+        uint32_t npart = 0;      // partial (stream-K) work items so far: epi_done/epi_flag phase
+        SegIter segs(args, num_tiles, num_kstages);
+        Seg sg;
+        while (segs.next(sg)) {
+            const int pt = sg.tile % args.num_p_tiles;
+            const int qt = sg.tile / args.num_p_tiles;
             // The decision must be warp-uniform: tcgen05.ld below is .sync.aligned.
             const bool ok = mbar_wait(&tfull[acc], acc_phase, args.timeout_ns, abort_flag, args.status);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const int p = pt * 128 + row;
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
-            if constexpr (kFastDrain) {
+            // (stream-K is never chosen for 256-wide tiles; keep that path out of them)
+            const bool partial = BN <= 128 && (sg.ks0 != 0 || sg.ks1 != num_kstages);
+            if (partial) {
+                // ---- stream-K: part of the tile's K range.  Add the partial
+                // sums into acc_ws; the CTA that brings the tile's slab count
+                // to num_kstages scales, converts and stores it, and re-zeroes
+                // its accumulators and counter for the next call.
+                constexpr int WC = BN >= 64 ? BN / 2 : BN;          // columns per warp
+                constexpr int CH = WC < 32 ? WC : 32;
+                const int c0 = BN >= 64 ? half * WC : 0;
+                if (BN >= 64 || half == 0) {
+                    float *accrow = args.acc_ws + static_cast<int64_t>(p) * args.q_pad + qt * BN + c0;
+#pragma unroll
+                    for (int c = 0; c < WC / CH; ++c) {
+                        uint32_t r[CH];
+                        if constexpr (CH == 32)
+                            tmem_ld_32x32b_x32(tbase + c0 + c * CH, reinterpret_cast<uint32_t(&)[32]>(r));
+                        else
+                            tmem_ld_32x32b_x16(tbase + c0 + c * CH, reinterpret_cast<uint32_t(&)[16]>(r));
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < CH; i += 4)
+                            red_add_v4_f32(accrow + c * CH + i, __uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                                           __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+                __threadfence();                                 // this thread's adds before the count
+                __syncwarp();
+                if (lane == 0) mbar_arrive(epi_done);
+                // Warp 6 (all lanes, so that no warp spins on two barriers at
+                // once) waits until the 8 epilogue warps have added, counts
+                // this CTA's slabs and publishes whether it completed the tile.
+                bool is_last;
+                if (warp == 6) {
+                    const bool done_ok = mbar_wait(epi_done, npart & 1u, args.timeout_ns, abort_flag, args.status);
+                    uint32_t last = 0u;
+                    if (lane == 0 && done_ok) {
+                        const int add = sg.ks1 - sg.ks0;
+                        const int before = atomicAdd(&args.tile_cnt[sg.tile], add);
+                        last = (before + add == num_kstages) ? 1u : 0u;
+                    }
+                    last = __shfl_sync(0xffffffffu, last, 0);
+                    if (lane == 0) {
+                        *last_flag = last;
+                        mbar_arrive(epi_flag);
+                    }
+                    is_last = last != 0u;
+                } else {
+                    const bool flag_ok = mbar_wait(epi_flag, npart & 1u, args.timeout_ns, abort_flag, args.status);
+                    is_last = flag_ok && *last_flag != 0u;
+                }
+                ++npart;
+                if (is_last) {
+                    // Coalesced: a warp covers contiguous output, so that each
+                    // store instruction writes whole sectors.
+                    __threadfence();
+                    const int ew = warp - 6;                       // 0..7
+                    OutT *y = static_cast<OutT *>(args.y);
+                    float *tile_acc = args.acc_ws + static_cast<int64_t>(pt) * 128 * args.q_pad + qt * BN;
+                    if constexpr (!SWAP) {
+                        // y[p][q]: warp ew takes rows ew, ew + 8, ...; lane l columns 4l..4l+3 (+128 k)
+                        for (int rr = ew; rr < 128; rr += 8) {
+                            const int pr = pt * 128 + rr;
+                            float *src = tile_acc + static_cast<int64_t>(rr) * args.q_pad;
+                            for (int c = lane * 4; c < BN; c += 128) {
+                                const float4 f = __ldcg(reinterpret_cast<const float4 *>(src + c));
+                                __stcg(reinterpret_cast<float4 *>(src + c), make_float4(0.f, 0.f, 0.f, 0.f));
+                                const float v0 = __fmul_rn(f.x, alpha), v1 = __fmul_rn(f.y, alpha);
+                                const float v2 = __fmul_rn(f.z, alpha), v3 = __fmul_rn(f.w, alpha);
+                                const int q = qt * BN + c;
+                                if (pr < args.P) {
+                                    OutT *dst = y + static_cast<int64_t>(pr) * args.ldy + q;
+                                    if (q + 4 <= args.Q) {
+                                        if constexpr (sizeof(OutT) == 2) {
+                                            __nv_bfloat162 lo = __floats2bfloat162_rn(v0, v1);
+                                            __nv_bfloat162 hi = __floats2bfloat162_rn(v2, v3);
+                                            *reinterpret_cast<uint2 *>(dst) =
+                                                make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+                                        } else {
+                                            *reinterpret_cast<float4 *>(dst) = make_float4(v0, v1, v2, v3);
+                                        }
+                                    } else {
+                                        const float vv[4] = {v0, v1, v2, v3};
+#pragma unroll
+                                        for (int k = 0; k < 4; ++k)
+                                            if (q + k < args.Q) {
+                                                if constexpr (sizeof(OutT) == 2) dst[k] = __float2bfloat16_rn(vv[k]);
+                                                else dst[k] = vv[k];
+                                            }
+                                    }
+                                }
+                            }
+                        }
+                    } else {
+                        // y[q][p]: warp ew takes columns q = ew, ew + 8, ...; lanes run along p
+                        for (int qq = ew; qq < BN; qq += 8) {
+                            const int q = qt * BN + qq;
+                            for (int rr = lane; rr < 128; rr += 32) {
+                                const int pr = pt * 128 + rr;
+                                float *src = tile_acc + static_cast<int64_t>(rr) * args.q_pad + qq;
+                                const float v = __fmul_rn(__ldcg(src), alpha);
+                                __stcg(src, 0.f);
+                                if (pr < args.P && q < args.Q) {
+                                    if constexpr (sizeof(OutT) == 2)
+                                        y[static_cast<int64_t>(q) * args.ldy + pr] = __float2bfloat16_rn(v);
+                                    else
+                                        y[static_cast<int64_t>(q) * args.ldy + pr] = v;
+                                }
+                            }
+                        }
+                    }
+                    if (threadIdx.x == 192) args.tile_cnt[sg.tile] = 0;
+                }
+            } else if constexpr (kFastDrain) {
                 // each warp drains and stores its half of the columns, the next
                 // 32-column chunk in flight while the current one is stored
                 constexpr int HC = BN / 2;
@@ -535,10 +690,37 @@ CUresult encode_output_map_bf16(CUtensorMap *map, void *y, uint64_t rows, uint64
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+// Stream-K scratch layout for a GEMM of M activation rows and N weight rows:
+// fp32 partial sums [p_rows][q_cols] over the padded tile grid, then one int32
+// counter per tile.  The path is only taken for few tiles (<= kMaxStreamKTiles).
+static constexpr int64_t kMaxStreamKTiles = 1024;
+struct SplitKLayout {
+    int64_t p_rows, q_cols, tiles;
+    size_t acc_bytes, bytes;
+};
+static SplitKLayout splitk_layout(int64_t M, int64_t N) {
+    SplitKLayout l;
+    if (M <= 64) {      // swapped: weights on the MMA's M, activations on N (BN <= 64)
+        l.p_rows = round_up(N, 128);
+        l.q_cols = 64;
+        l.tiles = ceil_div(N, 128);
+    } else {            // 128x128 tiles
+        l.p_rows = round_up(M, 128);
+        l.q_cols = round_up(N, 128);
+        l.tiles = ceil_div(M, 128) * ceil_div(N, 128);
+    }
+    auto a256 = [](size_t v) { return (v + 255) & ~size_t(255); };
+    l.acc_bytes = a256(static_cast<size_t>(l.p_rows * l.q_cols) * sizeof(float));
+    l.bytes = (l.tiles <= kMaxStreamKTiles) ? l.acc_bytes + a256(static_cast<size_t>(l.tiles) * sizeof(int32_t)) : 0;
+    return l;
+}
+
+size_t splitk_ws_bytes(int64_t M, int64_t N) { return splitk_layout(M, N).bytes; }
+
 template <int BN, bool SWAP, typename OutT>
 static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, void *y, int64_t ldy,
                             uint32_t *status, uint64_t timeout_ns, int num_sms, int preload,
-                            cudaStream_t stream) {
+                            uint8_t *splitk_ws, const SplitKLayout &skl, cudaStream_t stream) {
     using C = GemmCfg<BN>;
     CUtensorMap tmA, tmB;
     if (encode_tensor_map_u8(&tmA, pa.codes, K / 2, pa.rows, 128, 128) != CUDA_SUCCESS ||
@@ -562,11 +744,24 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     a.status = status;
     a.timeout_ns = timeout_ns;
     const int tiles = a.num_p_tiles * a.num_q_tiles;
+    const int64_t units = static_cast<int64_t>(tiles) * ((a.num_k_steps + 3) / 4);
+    // Stream-K when the tiles alone would leave at least half of the SMs idle
+    // (NVFP4_GEMM_STREAMK=0 turns it off): its reduction adds a serial tail
+    // that only pays off there.
+    const char *sk_opt = getenv("NVFP4_GEMM_STREAMK");
+    const bool sk = BN <= 128 && splitk_ws != nullptr && skl.bytes != 0 && 2 * tiles <= num_sms &&
+                    !(sk_opt != nullptr && sk_opt[0] == '0') &&
+                    units >= 2 * tiles && a.num_q_tiles * BN <= skl.q_cols && a.num_p_tiles * 128 <= skl.p_rows;
+    a.streamk = sk ? 1 : 0;
+    a.q_pad = a.num_q_tiles * BN;
+    a.acc_ws = sk ? reinterpret_cast<float *>(splitk_ws) : nullptr;
+    a.tile_cnt = sk ? reinterpret_cast<int32_t *>(splitk_ws + skl.acc_bytes) : nullptr;
     auto kern = gemm_nvf4_kernel<BN, SWAP, OutT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(tiles < num_sms ? tiles : num_sms);
+    const int64_t work = sk ? units : tiles;
+    cfg.gridDim = dim3(static_cast<unsigned>(work < num_sms ? work : num_sms));
     cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
@@ -580,17 +775,19 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
 
 cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
                         int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
-                        cudaStream_t stream, bool weights_ready) {
+                        cudaStream_t stream, bool weights_ready, void *splitk_ws) {
     // weights_ready: the weights were not written by the kernel launched just
     // before this one, so they may be streamed before the dependent-launch wait.
     const int preload = weights_ready ? 8 : 0;
     const int64_t M = act.rows, N = wgt.rows;
+    const SplitKLayout skl = splitk_layout(M, N);
+    uint8_t *skw = static_cast<uint8_t *>(splitk_ws);
     if (M <= 64) {
         // weights on the MMA's M side, activations on N; y[m][n] = acc[n][m]
         const int bn = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
 #define NVFP4_SWAPPED(BNV)                                                                          \
-    return y_bf16 ? run_gemm<BNV, true, __nv_bfloat16>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, stream) \
-                  : run_gemm<BNV, true, float>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, stream);
+    return y_bf16 ? run_gemm<BNV, true, __nv_bfloat16>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, stream) \
+                  : run_gemm<BNV, true, float>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, stream);
         if (bn == 16) { NVFP4_SWAPPED(16) }
         if (bn == 32) { NVFP4_SWAPPED(32) }
         NVFP4_SWAPPED(64)
@@ -601,10 +798,10 @@ cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void 
     const int64_t ptiles = ceil_div(M, 128);
     const bool wide = ptiles * ceil_div(N, 256) >= 2 * num_sms;
     if (wide)
-        return y_bf16 ? run_gemm<256, false, __nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, stream)
-                      : run_gemm<256, false, float>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, stream);
-    return y_bf16 ? run_gemm<128, false, __nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, stream)
-                  : run_gemm<128, false, float>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, stream);
+        return y_bf16 ? run_gemm<256, false, __nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, stream)
+                      : run_gemm<256, false, float>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, stream);
+    return y_bf16 ? run_gemm<128, false, __nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, stream)
+                  : run_gemm<128, false, float>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -26,9 +26,14 @@ struct Operand {
 // y[M][N] = (A . B^T) * gA * gB, A = act [M][K], B = wgt [N][K].
 // weights_ready: the weights were not written by the kernel launched just
 // before (they may be streamed before the programmatic-dependent-launch wait).
+// splitk_ws: splitk_ws_bytes(M, N) bytes of zero-filled scratch (or null: no
+// stream-K); a successful call leaves it zero-filled.
 cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
                         int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
-                        cudaStream_t stream, bool weights_ready = false);
+                        cudaStream_t stream, bool weights_ready = false, void *splitk_ws = nullptr);
+
+// Bytes of stream-K scratch a GEMM of M activation rows and N weight rows may use (0: never).
+size_t splitk_ws_bytes(int64_t M, int64_t N);
 
 // Two-CTA (cta_group::2) GEMM for large M: usable when enough 256x256 tiles
 // exist to fill the GPU with CTA pairs.

@@ -30,14 +30,15 @@ def quantize_gpu(nv, x):
     return out
 
 
-def run_gemm(nv, a, b, out_dtype):
+def run_gemm(nv, a, b, out_dtype, ws=None):
     # rows of y must start on 16-byte boundaries: pad the pitch (always by at
     # least one 16-byte unit, so that writes past N would be seen), then slice
     per16 = 16 // torch.empty((), dtype=out_dtype).element_size()
     ldy = -(-b.rows // per16) * per16 + per16
     buf = torch.full((a.rows, ldy), float("nan"), dtype=out_dtype, device="cuda")
     y = buf[:, :b.rows]
-    ws = nv.workspace(nv.OP_GEMM, a.rows, b.rows, a.cols)
+    if ws is None:
+        ws = nv.workspace(nv.OP_GEMM, a.rows, b.rows, a.cols)
     nv.nvfp4_gemm(a, b, y, ws)
     assert nv.nvfp4_get_device_status(ws) == nv.OK
     assert torch.isnan(buf[:, b.rows:].float()).all()      # nothing written past N
@@ -135,6 +136,34 @@ def test_gemm_cta_pair_tiles(nv, M, N, K, pair, monkeypatch):
     ref, na, nb = oracle.gemm_entries(xq_o, wq_o, ms, ns)
     assert_gemm_close(yc[ms, ns], ref, na, nb, K, True, f"pair {M}x{N}x{K}")
     assert np.isfinite(yc).all()
+
+
+@pytest.mark.parametrize("M,N,K,dt", [(24, 1000, 1088, torch.bfloat16), (8, 17408, 5120, torch.float32),
+                                      (200, 700, 2048, torch.bfloat16), (130, 520, 4096, torch.float32)])
+def test_gemm_stream_k(nv, M, N, K, dt):
+    """Few output tiles: CTAs split K, partial sums meet in fp32 in the
+    workspace and the last contributor of each tile writes it.  Covers the
+    swapped (M <= 64) and 128x128 layouts, ragged M and N, bf16 and fp32 out;
+    two calls on one workspace both match the oracle, and each leaves the
+    workspace's stream-K scratch zero-filled again."""
+    rng = np.random.default_rng(M * 7 + N)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[rng.random(x.shape) < 1e-3] *= 50
+    wt = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    xq_o, wq_o = oracle.quantize(x), oracle.quantize(wt)
+    xq, wq = quantize_gpu(nv, f32_tensor(x)), quantize_gpu(nv, f32_tensor(wt))
+    ws = nv.workspace(nv.OP_GEMM, M, N, K)
+    assert ws.numel() > 256                                  # the shape has stream-K scratch
+    ms = np.concatenate([rng.integers(0, M, 3000), np.full(N, M - 1), np.arange(M)])
+    ns = np.concatenate([rng.integers(0, N, 3000), np.arange(N), np.full(M, N - 1)])
+    ref, na, nb = oracle.gemm_entries(xq_o, wq_o, ms, ns)
+    for call in range(2):
+        y = run_gemm(nv, xq, wq, dt, ws=ws)
+        yc = to_numpy_f64(y)
+        assert np.isfinite(yc).all()
+        assert_gemm_close(yc[ms, ns], ref, na, nb, K, dt == torch.bfloat16, f"stream-K {M}x{N}x{K} call {call}")
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(ws[256:]) == 0, "stream-K scratch not re-zeroed"
 
 
 def test_gemm_special_operands(nv):
