@@ -339,7 +339,9 @@ def torch_empty_pinned(torch, like):
 # measurement
 # ---------------------------------------------------------------------------
 
-def dist_setup(args):
+def dist_setup(backend=None):
+    """One process per GPU from torchrun's environment.  NCCL on GPUs; gloo
+    (CPU tensors) when asked for or when there is no GPU (host-side tests)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -347,9 +349,13 @@ def dist_setup(args):
         import datetime
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
@@ -360,13 +366,27 @@ def barrier(world):
 
 
 def max_over_ranks(world, value):
+    """The largest of every rank's value (each rank's device time)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def emit(line, rank):
+    """Rank 0 alone prints the result line."""
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def dist_teardown(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
 
 
 def _capture(torch, fn, n):
@@ -519,7 +539,7 @@ def reference_arm(args):
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(),
                              "kind": "oracle", "sample": f"{rows} X rows per step"},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(line))
+    emit(line, rank)
     return 0
 
 
@@ -549,7 +569,7 @@ def main():
     if args.impl == "reference":
         return reference_arm(args)
 
-    world, rank, local = dist_setup(args)
+    world, rank, local = dist_setup()
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}; using {world}", file=sys.stderr)
     import torch
@@ -597,11 +617,8 @@ def main():
             "peaks": peaks}
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "prefill":
         line["cpu_baseline"] = cpu_oracle_prefill(args.cpu_rows)
-    if rank == 0:
-        print(json.dumps(line))
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    emit(line, rank)
+    dist_teardown(world)
     return 0
 
 
