@@ -437,53 +437,70 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     OutT *y = static_cast<OutT *>(args.y);
                     float *tile_acc = args.acc_ws + static_cast<int64_t>(pt) * 128 * args.q_pad + qt * BN;
                     if constexpr (!SWAP) {
-                        // y[p][q]: warp ew takes rows ew, ew + 8, ...; lane l columns 4l..4l+3 (+128 k)
-                        for (int rr = ew; rr < 128; rr += 8) {
-                            const int pr = pt * 128 + rr;
-                            float *src = tile_acc + static_cast<int64_t>(rr) * args.q_pad;
-                            for (int c = lane * 4; c < BN; c += 128) {
-                                const float4 f = __ldcg(reinterpret_cast<const float4 *>(src + c));
-                                __stcg(reinterpret_cast<float4 *>(src + c), make_float4(0.f, 0.f, 0.f, 0.f));
-                                const float v0 = __fmul_rn(f.x, alpha), v1 = __fmul_rn(f.y, alpha);
-                                const float v2 = __fmul_rn(f.z, alpha), v3 = __fmul_rn(f.w, alpha);
-                                const int q = qt * BN + c;
-                                if (pr < args.P) {
-                                    OutT *dst = y + static_cast<int64_t>(pr) * args.ldy + q;
-                                    if (q + 4 <= args.Q) {
-                                        if constexpr (sizeof(OutT) == 2) {
-                                            __nv_bfloat162 lo = __floats2bfloat162_rn(v0, v1);
-                                            __nv_bfloat162 hi = __floats2bfloat162_rn(v2, v3);
-                                            *reinterpret_cast<uint2 *>(dst) =
-                                                make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
-                                        } else {
-                                            *reinterpret_cast<float4 *>(dst) = make_float4(v0, v1, v2, v3);
-                                        }
-                                    } else {
-                                        const float vv[4] = {v0, v1, v2, v3};
+                        // y[p][q] (BN = 128 here): warp ew takes rows ew, ew + 8, ...,
+                        // lane l columns 4l..4l+3.  All loads are issued before
+                        // any is used (the finalize is on the kernel's tail).
+                        constexpr int RPW = 128 / 8;
+                        float4 f[RPW];
 #pragma unroll
-                                        for (int k = 0; k < 4; ++k)
-                                            if (q + k < args.Q) {
-                                                if constexpr (sizeof(OutT) == 2) dst[k] = __float2bfloat16_rn(vv[k]);
-                                                else dst[k] = vv[k];
-                                            }
+                        for (int i = 0; i < RPW; ++i)
+                            f[i] = __ldcg(reinterpret_cast<const float4 *>(
+                                tile_acc + static_cast<int64_t>(ew + 8 * i) * args.q_pad + lane * 4));
+#pragma unroll
+                        for (int i = 0; i < RPW; ++i) {
+                            const int rr = ew + 8 * i;
+                            const int pr = pt * 128 + rr;
+                            __stcg(reinterpret_cast<float4 *>(tile_acc + static_cast<int64_t>(rr) * args.q_pad + lane * 4),
+                                   make_float4(0.f, 0.f, 0.f, 0.f));
+                            const float v0 = __fmul_rn(f[i].x, alpha), v1 = __fmul_rn(f[i].y, alpha);
+                            const float v2 = __fmul_rn(f[i].z, alpha), v3 = __fmul_rn(f[i].w, alpha);
+                            const int q = qt * BN + lane * 4;
+                            if (pr < args.P && lane * 4 < BN) {
+                                OutT *dst = y + static_cast<int64_t>(pr) * args.ldy + q;
+                                if (q + 4 <= args.Q) {
+                                    if constexpr (sizeof(OutT) == 2) {
+                                        __nv_bfloat162 lo = __floats2bfloat162_rn(v0, v1);
+                                        __nv_bfloat162 hi = __floats2bfloat162_rn(v2, v3);
+                                        *reinterpret_cast<uint2 *>(dst) =
+                                            make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+                                    } else {
+                                        *reinterpret_cast<float4 *>(dst) = make_float4(v0, v1, v2, v3);
                                     }
+                                } else {
+                                    const float vv[4] = {v0, v1, v2, v3};
+#pragma unroll
+                                    for (int k = 0; k < 4; ++k)
+                                        if (q + k < args.Q) {
+                                            if constexpr (sizeof(OutT) == 2) dst[k] = __float2bfloat16_rn(vv[k]);
+                                            else dst[k] = vv[k];
+                                        }
                                 }
                             }
                         }
                     } else {
-                        // y[q][p]: warp ew takes columns q = ew, ew + 8, ...; lanes run along p
-                        for (int qq = ew; qq < BN; qq += 8) {
-                            const int q = qt * BN + qq;
-                            for (int rr = lane; rr < 128; rr += 32) {
+                        // y[q][p]: warp ew takes columns q = ew, ew + 8, ...; lanes
+                        // run along p (rows lane, lane + 32, ...).  Loads first.
+                        constexpr int QPW = BN / 8;
+                        float v[QPW][4];
+#pragma unroll
+                        for (int j = 0; j < QPW; ++j)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                v[j][i] = __ldcg(tile_acc + static_cast<int64_t>(lane + 32 * i) * args.q_pad + ew + 8 * j);
+#pragma unroll
+                        for (int j = 0; j < QPW; ++j) {
+                            const int q = qt * BN + ew + 8 * j;
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int rr = lane + 32 * i;
                                 const int pr = pt * 128 + rr;
-                                float *src = tile_acc + static_cast<int64_t>(rr) * args.q_pad + qq;
-                                const float v = __fmul_rn(__ldcg(src), alpha);
-                                __stcg(src, 0.f);
+                                __stcg(tile_acc + static_cast<int64_t>(rr) * args.q_pad + ew + 8 * j, 0.f);
+                                const float o = __fmul_rn(v[j][i], alpha);
                                 if (pr < args.P && q < args.Q) {
                                     if constexpr (sizeof(OutT) == 2)
-                                        y[static_cast<int64_t>(q) * args.ldy + pr] = __float2bfloat16_rn(v);
+                                        y[static_cast<int64_t>(q) * args.ldy + pr] = __float2bfloat16_rn(o);
                                     else
-                                        y[static_cast<int64_t>(q) * args.ldy + pr] = v;
+                                        y[static_cast<int64_t>(q) * args.ldy + pr] = o;
                                 }
                             }
                         }
@@ -746,8 +763,11 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     const int tiles = a.num_p_tiles * a.num_q_tiles;
     const int64_t units = static_cast<int64_t>(tiles) * ((a.num_k_steps + 3) / 4);
     // Stream-K when the tiles alone would leave at least half of the SMs idle
-    // (NVFP4_GEMM_STREAMK=0 turns it off): its reduction adds a serial tail
-    // that only pays off there.
+    // (NVFP4_GEMM_STREAMK=0 turns it off).  Its reduction tail (partial sums
+    // through L2, then the finishing CTA's pass) costs a few microseconds, so
+    // with about one tile per SM the plain tile loop is faster (measured: M=8
+    // and M=128 at N=17408, 136 tiles); the 40-tile MLP down projection gains
+    // about 30%.
     const char *sk_opt = getenv("NVFP4_GEMM_STREAMK");
     const bool sk = BN <= 128 && splitk_ws != nullptr && skl.bytes != 0 && 2 * tiles <= num_sms &&
                     !(sk_opt != nullptr && sk_opt[0] == '0') &&
