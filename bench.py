@@ -291,7 +291,7 @@ class Mlp:
         hq_bytes = M * N // 2 + M * N // 16
         self.bytes = per_step + M * K * 2 + M * K * 2 + 2 * hq_bytes
         self.units = self.bytes / 1e9
-        self.launches = 8
+        self.launches = 5                       # amax, encode (x); gate+up GEMM; encode (h); down GEMM
         self.dominant = {"kernel": "gemm_nvf4_kernel (down projection, K=17408)", "bound": "hbm",
                          "algorithmic": N * K // 2 + N * K // 16 + hq_bytes + M * K * 2,
                          "unit": "GB/s"}

@@ -110,9 +110,8 @@ size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K) {
         // status, partials | x_q (codes, scales, g) | stream-K scratch
         return kQuantizeWs + quantized_bytes(M, K) + splitk_ws_bytes(M, N);
     case NVFP4_OP_LINEAR_FUSED_SILU:
-        // status, partials | x_q | gate, up, h (fp32 [M][N] each) | stream-K scratch
-        return kQuantizeWs + quantized_bytes(M, K) +
-               3 * align256(static_cast<size_t>(M * N) * sizeof(float)) + splitk_ws_bytes(M, N);
+        // status, partials | x_q | h (fp32 [M][N])
+        return kQuantizeWs + quantized_bytes(M, K) + align256(static_cast<size_t>(M * N) * sizeof(float));
     }
     return 0;
 }
@@ -248,31 +247,24 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
                                     dev.sms, stream);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     uint32_t *status = static_cast<uint32_t *>(ws);
-    const bool has_sk = splitk_ws_bytes(M, N) != 0;
-    const size_t mn = align256(static_cast<size_t>(M * N) * sizeof(float));
     if (epilogue == NVFP4_EPI_STORE)
         return gemm_impl(&xq, w, y, yt, ldy, status, dev.sms, stream, true,
-                         has_sk ? ws_at(ws, kQuantizeWs + quantized_bytes(M, K)) : nullptr);
+                         splitk_ws_bytes(M, N) != 0 ? ws_at(ws, kQuantizeWs + quantized_bytes(M, K)) : nullptr);
 
-    // SiLU(gate) * up, then re-quantize h for the down projection.
-    float *gate = reinterpret_cast<float *>(ws_at(ws, off));
-    float *up = reinterpret_cast<float *>(ws_at(ws, off + mn));
-    float *h = y ? static_cast<float *>(y) : reinterpret_cast<float *>(ws_at(ws, off + 2 * mn));
+    // Gate and up in one GEMM whose epilogue writes h = SiLU(gate) * up and the
+    // per-CTA max |h|; then the quantizer's encode pass turns h into NVFP4.
+    float *h = y ? static_cast<float *>(y) : reinterpret_cast<float *>(ws_at(ws, off));
     const int64_t ldh = y ? ldy : N;
-    void *sk = has_sk ? ws_at(ws, kQuantizeWs + quantized_bytes(M, K) + 3 * mn) : nullptr;
-    if ((st = gemm_impl(&xq, w, gate, NVFP4_F32, N, status, dev.sms, stream, true, sk)) != NVFP4_OK) return st;
-    if ((st = gemm_impl(&xq, w_up, up, NVFP4_F32, N, status, dev.sms, stream, true, sk)) != NVFP4_OK) return st;
-    if (ldh == N) {
-        if (launch_silu_mul(gate, up, h, M * N, dev.sms, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
-    } else {
-        for (int64_t r = 0; r < M; ++r)
-            if (launch_silu_mul(gate + r * N, up + r * N, h + r * ldh, N, dev.sms, stream) != cudaSuccess)
-                return NVFP4_ERR_CUDA;
-    }
-    return from_cuda(launch_quantize(h, false, M, N, ldh, y_q->codes, y_q->scales,
-                                     y_q->tensor_scale,
-                                     reinterpret_cast<float *>(ws_at(ws, kPartialsOff)), dev.sms,
-                                     stream));
+    Operand act{xq.codes, xq.scales, xq.tensor_scale, M};
+    Operand og{w->codes, w->scales, w->tensor_scale, N};
+    Operand ou{w_up->codes, w_up->scales, w_up->tensor_scale, N};
+    float *partials = reinterpret_cast<float *>(ws_at(ws, kPartialsOff));
+    int nparts = 0;
+    if (launch_gemm_dual_silu(act, og, ou, K, h, ldh, partials, kMaxAmaxPartials, &nparts, status,
+                              timeout_ns(), dev.sms, stream, true) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return from_cuda(launch_encode_f32(h, M, N, ldh, partials, nparts, y_q->codes, y_q->scales,
+                                       y_q->tensor_scale, dev.sms, stream));
 }
 
 nvfp4_status nvfp4_get_device_status(void *ws, nvfp4_stream_t stream) {

@@ -825,27 +825,6 @@ cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void 
 }
 
 // ---------------------------------------------------------------------------
-// Elementwise SiLU(gate) * up (fp32), SiLU(z) = z / (1 + exp(-z)).
-// ---------------------------------------------------------------------------
-__global__ void silu_mul_kernel(const float *__restrict__ gate, const float *__restrict__ up,
-                                float *__restrict__ h, int64_t n) {
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const float z = gate[i];
-        h[i] = __fmul_rn(__fdiv_rn(z, __fadd_rn(1.0f, expf(-z))), up[i]);
-    }
-}
-
-cudaError_t launch_silu_mul(const float *gate, const float *up, float *h, int64_t n, int num_sms,
-                            cudaStream_t stream) {
-    int64_t blocks = ceil_div(n, 256);
-    const int64_t cap = static_cast<int64_t>(num_sms) * 8;
-    blocks = blocks < 1 ? 1 : (blocks < cap ? blocks : cap);
-    silu_mul_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(gate, up, h, n);
-    return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
 // Bounded-wait self test: one thread waits on a barrier nothing completes.
 // ---------------------------------------------------------------------------
 __global__ void wait_selftest_kernel(uint32_t *status, uint64_t timeout_ns) {

@@ -41,9 +41,21 @@ bool pair_gemm_usable(int64_t M, int64_t N, int num_sms);
 cudaError_t launch_gemm_pair(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
                              int64_t ldy, uint32_t *status, uint64_t timeout_ns, cudaStream_t stream);
 
-// h = SiLU(gate) * up elementwise in fp32 (n values).
-cudaError_t launch_silu_mul(const float *gate, const float *up, float *h, int64_t n, int num_sms,
-                            cudaStream_t stream);
+// The quantizer's second pass alone, on fp32 x whose first pass (max |x| per
+// part, num_partials values) was produced elsewhere.
+cudaError_t launch_encode_f32(const float *x, int64_t rows, int64_t cols, int64_t ld, const float *partials,
+                              int num_partials, uint8_t *codes, uint8_t *scales, float *g_out, int num_sms,
+                              cudaStream_t stream);
+
+// h[M][N] = SiLU(x wg^T * gx*gwg) * (x wu^T * gx*gwu) in fp32 (128x128 tiles,
+// both products per tile), and max |h| per CTA into partials (the quantizer's
+// first-pass format); *num_partials receives how many were written
+// (<= max_partials).
+cudaError_t launch_gemm_dual_silu(const Operand &act, const Operand &wg, const Operand &wu, int64_t K,
+                                  float *h, int64_t ldh, float *partials, int max_partials, int *num_partials,
+                                  uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t stream,
+                                  bool weights_ready);
+
 
 cudaError_t launch_wait_selftest(uint32_t *status, uint64_t timeout_ns, cudaStream_t stream);
 

@@ -508,6 +508,24 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
                               g_out);
 }
 
+cudaError_t launch_encode_f32(const float *x, int64_t rows, int64_t cols, int64_t ld, const float *partials,
+                              int num_partials, uint8_t *codes, uint8_t *scales, float *g_out, int num_sms,
+                              cudaStream_t stream) {
+    static const int occ_encode = resident_ctas(encode_kernel<float>);
+    const int g2 = quantize_grid(rows, cols, 1, num_sms, occ_encode);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(g2);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, encode_kernel<float>, x, rows, cols, ld, partials, num_partials, codes,
+                              scales, g_out);
+}
+
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scales, const float *g,
                               int64_t rows, int64_t cols, void *y, bool bf16, int64_t ldy,
                               int num_sms, cudaStream_t stream) {

@@ -98,6 +98,14 @@ def test_mlp_small(nv):
     check_mlp(nv, w["X"], w["Wg"], w["Wu"], w["Wd"], M, K, N)
 
 
+def test_mlp_ragged_tiles(nv):
+    """Two 128-row tiles with a partial second one, a partial last 128-column
+    tile of h and a partial last K slab, through the fused gate/up kernel."""
+    M, K, N = 200, 320, 320
+    w = workloads.make("mlp", M=M, K=K, N=N, seed=41)
+    check_mlp(nv, w["X"], w["Wg"], w["Wu"], w["Wd"], M, K, N)
+
+
 def test_mlp_workload_full(nv):
     """The fused MLP workload at full size: M=128, K=5120, N=17408 (seed 4)."""
     w = workloads.make("mlp")
