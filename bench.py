@@ -30,6 +30,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 L2_BYTES = 126 * 1024 * 1024
+# DRAM bytes read + written per launch of each workload's dominant kernel(s),
+# from one ncu capture of the current kernels (profiles/*.md, "DRAM read /
+# write"); set an entry to None when its kernel changes.
+NCU_TRAFFIC = {"prefill": 161_869_056, "decode": 50_261_760, "quantize": 176_702_976, "mlp": 54_093_056}
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP4_PER_BF16 = 4.0          # dense FP4 : dense BF16 on B200 (9 : 2.25 PFLOP/s nominal)
@@ -478,7 +482,7 @@ def roofline(wl, kern_us, peaks):
         unit = "GB/s"
         peak_note = f"{peaks['source']} HBM copy bandwidth"
     return {"bound": d["bound"], "achieved": round(achieved, 1), "peak": round(peak, 1),
-            "unit": unit, "frac": round(achieved / peak, 4), "traffic": None,
+            "unit": unit, "frac": round(achieved / peak, 4), "traffic": NCU_TRAFFIC.get(wl.name),
             "kernel": d["kernel"], "kernel_us": round(kern_us, 2),
             "algorithmic_per_launch": d["algorithmic"], "peak_source": peak_note}
 
