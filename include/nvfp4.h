@@ -40,9 +40,8 @@
  *     device memory.  Zero-fill it once after allocating; the library keeps a
  *     sticky status word in its first 16 bytes and uses the rest as scratch.
  *     GEMMs with few output tiles split K across SMs and add fp32 partial
- *     sums in a part of the scratch that every successful call leaves
- *     zero-filled again; after a call whose status reports a device-side
- *     give-up, zero-fill the workspace again before reusing it.
+ *     sums in the scratch (zero-filled by the call itself, so workspaces may
+ *     be shared between operations and shapes that do not overlap in time).
  *     Calls that share one workspace must not overlap on the GPU.
  */
 #ifndef NVFP4_H

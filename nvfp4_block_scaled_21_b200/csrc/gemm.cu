@@ -57,8 +57,8 @@ struct GemmArgs {
     int32_t weights_are_a;   // 1: the weights are the MMA A operand (swapped)
     int32_t streamk;         // 1: CTAs take equal contiguous runs of (tile, K slab) units
     int32_t q_pad;           // row pitch (floats) of acc_ws: num_q_tiles * BN
-    float *acc_ws;           // stream-K: fp32 partial sums [num_p_tiles*128][q_pad], zero between calls
-    int32_t *tile_cnt;       // stream-K: K slabs added per tile so far, zero between calls
+    float *acc_ws;           // stream-K: fp32 partial sums [num_p_tiles*128][q_pad], zeroed per call
+    int32_t *tile_cnt;       // stream-K: K slabs added per tile so far, zeroed per call
     uint32_t *status;
     uint64_t timeout_ns;
 };
@@ -378,9 +378,9 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const bool partial = BN <= 128 && (sg.ks0 != 0 || sg.ks1 != num_kstages);
             if (partial) {
                 // ---- stream-K: part of the tile's K range.  Add the partial
-                // sums into acc_ws; the CTA that brings the tile's slab count
-                // to num_kstages scales, converts and stores it, and re-zeroes
-                // its accumulators and counter for the next call.
+                // sums into acc_ws (zero-filled by the launcher); the CTA that
+                // brings the tile's slab count to num_kstages scales, converts
+                // and stores it.
                 constexpr int WC = BN >= 64 ? BN / 2 : BN;          // columns per warp
                 constexpr int CH = WC < 32 ? WC : 32;
                 const int c0 = BN >= 64 ? half * WC : 0;
@@ -450,8 +450,6 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         for (int i = 0; i < RPW; ++i) {
                             const int rr = ew + 8 * i;
                             const int pr = pt * 128 + rr;
-                            __stcg(reinterpret_cast<float4 *>(tile_acc + static_cast<int64_t>(rr) * args.q_pad + lane * 4),
-                                   make_float4(0.f, 0.f, 0.f, 0.f));
                             const float v0 = __fmul_rn(f[i].x, alpha), v1 = __fmul_rn(f[i].y, alpha);
                             const float v2 = __fmul_rn(f[i].z, alpha), v3 = __fmul_rn(f[i].w, alpha);
                             const int q = qt * BN + lane * 4;
@@ -494,7 +492,6 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                             for (int i = 0; i < 4; ++i) {
                                 const int rr = lane + 32 * i;
                                 const int pr = pt * 128 + rr;
-                                __stcg(tile_acc + static_cast<int64_t>(rr) * args.q_pad + ew + 8 * j, 0.f);
                                 const float o = __fmul_rn(v[j][i], alpha);
                                 if (pr < args.P && q < args.Q) {
                                     if constexpr (sizeof(OutT) == 2)
@@ -505,7 +502,6 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                             }
                         }
                     }
-                    if (threadIdx.x == 192) args.tile_cnt[sg.tile] = 0;
                 }
             } else if constexpr (kFastDrain) {
                 // each warp drains and stores its half of the columns, the next
@@ -779,6 +775,9 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     auto kern = gemm_nvf4_kernel<BN, SWAP, OutT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
+    // The stream-K scratch is zero-filled for every call, so it may share a
+    // workspace with whatever other calls left there.
+    if (sk && (e = cudaMemsetAsync(splitk_ws, 0, skl.bytes, stream)) != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     const int64_t work = sk ? units : tiles;
     cfg.gridDim = dim3(static_cast<unsigned>(work < num_sms ? work : num_sms));

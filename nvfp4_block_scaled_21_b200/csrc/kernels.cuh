@@ -26,8 +26,8 @@ struct Operand {
 // y[M][N] = (A . B^T) * gA * gB, A = act [M][K], B = wgt [N][K].
 // weights_ready: the weights were not written by the kernel launched just
 // before (they may be streamed before the programmatic-dependent-launch wait).
-// splitk_ws: splitk_ws_bytes(M, N) bytes of zero-filled scratch (or null: no
-// stream-K); a successful call leaves it zero-filled.
+// splitk_ws: splitk_ws_bytes(M, N) bytes of scratch (or null: no stream-K);
+// any contents (the call zero-fills what it uses).
 cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
                         int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
                         cudaStream_t stream, bool weights_ready = false, void *splitk_ws = nullptr);

@@ -144,8 +144,8 @@ def test_gemm_stream_k(nv, M, N, K, dt):
     """Few output tiles: CTAs split K, partial sums meet in fp32 in the
     workspace and the last contributor of each tile writes it.  Covers the
     swapped (M <= 64) and 128x128 layouts, ragged M and N, bf16 and fp32 out;
-    two calls on one workspace both match the oracle, and each leaves the
-    workspace's stream-K scratch zero-filled again."""
+    the workspace's scratch starts full of garbage (as another operation may
+    have left it) and two calls on it both match the oracle."""
     rng = np.random.default_rng(M * 7 + N)
     x = rng.standard_normal((M, K)).astype(np.float32)
     x[rng.random(x.shape) < 1e-3] *= 50
@@ -154,6 +154,7 @@ def test_gemm_stream_k(nv, M, N, K, dt):
     xq, wq = quantize_gpu(nv, f32_tensor(x)), quantize_gpu(nv, f32_tensor(wt))
     ws = nv.workspace(nv.OP_GEMM, M, N, K)
     assert ws.numel() > 256                                  # the shape has stream-K scratch
+    ws[256:] = 0x7f                                          # garbage (large finite floats)
     ms = np.concatenate([rng.integers(0, M, 3000), np.full(N, M - 1), np.arange(M)])
     ns = np.concatenate([rng.integers(0, N, 3000), np.arange(N), np.full(M, N - 1)])
     ref, na, nb = oracle.gemm_entries(xq_o, wq_o, ms, ns)
@@ -162,8 +163,6 @@ def test_gemm_stream_k(nv, M, N, K, dt):
         yc = to_numpy_f64(y)
         assert np.isfinite(yc).all()
         assert_gemm_close(yc[ms, ns], ref, na, nb, K, dt == torch.bfloat16, f"stream-K {M}x{N}x{K} call {call}")
-        torch.cuda.synchronize()
-        assert torch.count_nonzero(ws[256:]) == 0, "stream-K scratch not re-zeroed"
 
 
 def test_gemm_special_operands(nv):
