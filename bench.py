@@ -430,6 +430,16 @@ def measure(wl, torch, K, W, world, local, sample_clocks=False):
     barrier(world)
     torch.cuda.synchronize()
     elapsed = max_over_ranks(world, start.elapsed_time(end) / 1e3)
+    # per-step distribution (this rank): K more replays, each between its own events
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        evs[i][0].record()
+        steps[(W + i) % wl.R].replay()
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    per = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)
+    dist = {"median": round(per[K // 2], 2), "p10": round(per[int(0.1 * (K - 1))], 2),
+            "p90": round(per[int(0.9 * (K - 1))], 2), "unit": "us", "rank": "local"}
     for i in range(W):
         kern[i % wl.R].replay()
     torch.cuda.synchronize()
@@ -441,7 +451,7 @@ def measure(wl, torch, K, W, world, local, sample_clocks=False):
     torch.cuda.synchronize()
     kern_us = max_over_ranks(world, ks.elapsed_time(ke) * 1e3 / K)
     del steps, kern
-    return elapsed, kern_us, (sampler.summary() if sampler else None)
+    return elapsed, kern_us, (sampler.summary() if sampler else None), dist
 
 
 class _Null:
@@ -491,6 +501,17 @@ def roofline(wl, kern_us, peaks):
 # CPU baseline: the oracle as it stands, on a bounded sample
 # ---------------------------------------------------------------------------
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_oracle_prefill(rows: int):
     """Oracle time for quantizing `rows` activation rows and their fp64 GEMM
     against the whole pre-quantized weight (prefill workload, seed 3)."""
@@ -505,7 +526,7 @@ def cpu_oracle_prefill(rows: int):
     dt = time.perf_counter() - t0
     flops = 2.0 * rows * w["N"] * w["K"]
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
-            "kind": "oracle", "seconds": round(dt, 2),
+            "cpu_model": _cpu_model(), "kind": "oracle", "seconds": round(dt, 2),
             "sample": f"prefill workload: oracle quantize of {rows} of 4096 X rows + fp64 GEMM of "
                       f"those rows against all 17408 pre-quantized W rows (K=5120), "
                       f"{os.cpu_count()} threads"}
@@ -540,7 +561,7 @@ def reference_arm(args):
             "config": {"workload": f"{w['name']} W4A4 linear, CPU oracle: each step quantizes "
                                    f"{rows} X rows and runs their fp64 GEMM against all "
                                    f"{w['N']} pre-quantized W rows (K={w['K']})"},
-            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(),
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(), "cpu_model": _cpu_model(),
                              "kind": "oracle", "sample": f"{rows} X rows per step"},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     emit(line, rank)
@@ -566,7 +587,7 @@ def main():
     ap.add_argument("--workload", choices=list(WORKLOADS), default="prefill")
     ap.add_argument("--only", action="store_true", help="measure the headline workload only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=64)
+    ap.add_argument("--cpu-rows", type=int, default=1024)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -588,15 +609,15 @@ def main():
     for n in names:
         wl = WORKLOADS[n](nv, torch)
         is_head = n == args.workload
-        elapsed, kern_us, clocks = measure(wl, torch, args.steps, args.warmup, world, local,
-                                           sample_clocks=is_head)
+        elapsed, kern_us, clocks, dist = measure(wl, torch, args.steps, args.warmup, world, local,
+                                                 sample_clocks=is_head)
         sps = elapsed / args.steps
         value = wl.value(sps) * world
         e2e_steps = min(args.steps, 20)
         e2e_elapsed = measure_e2e(wl, torch, e2e_steps, world)
         e2e_value = wl.value(e2e_elapsed / e2e_steps) * world
         res = {"metric": wl.metric, "value": round(value, 2), "unit": wl.unit,
-               "ms_per_step": round(sps * 1e3, 4), "config": wl.config,
+               "ms_per_step": round(sps * 1e3, 4), "step_us": dist, "config": wl.config,
                "roofline": roofline(wl, kern_us, peaks),
                "e2e": {"value": round(e2e_value, 3), "unit": wl.unit,
                        "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h},
@@ -611,7 +632,8 @@ def main():
 
     line = {"metric": head["metric"], "value": head["value"], "unit": head["unit"],
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": head["ms_per_step"], "step_us": head["step_us"],
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4",
             "data": "synthetic (seeded numpy PCG64: N(0,1) activations with 0.1% x50 outliers, "
                     "N(0,0.02) weights, bf16)",
