@@ -8,8 +8,8 @@ MLP step.  Prints ONE JSON line (rank 0).
 
 A step is one pass of the hot path over one batch of synthetic input already
 resident in HBM.  The headline workload (default: prefill, M=4096 N=17408
-K=5120) is timed over exactly K steps (CUDA-graph replays, one step each)
-bracketed by a barrier and a device
+K=5120) is timed over exactly K steps (CUDA-graph replays: a graph holds one
+step per rotating input slot) bracketed by a barrier and a device
 synchronize; the other workloads are measured the same way and reported under
 "workloads".  L2 (126 MB) is defeated by rotating enough input copies that
 each step's operands were evicted by the steps before it.  Multi-GPU runs are
@@ -405,17 +405,42 @@ def _capture(torch, fn, n):
     return graphs
 
 
+def _capture_rotation(torch, fn, n):
+    """One CUDA graph holding fn(0), fn(1), ..., fn(n-1): a full rotation of
+    the input slots, so consecutive steps run without a graph launch between
+    them (as consecutive layers would inside one captured forward pass)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for r in range(n):
+            fn(r)
+    torch.cuda.synchronize()
+    return g
+
+
+def _replay_k(singles, rotation, R, K):
+    """Exactly K steps starting at slot 0: full rotations, then single steps."""
+    for _ in range(K // R):
+        rotation.replay()
+    for i in range(K % R):
+        singles[i].replay()
+
+
 def measure(wl, torch, K, W, world, local, sample_clocks=False):
-    """Device time of exactly K steps (CUDA-graph replays, one step per
-    replay, rotating input slots), bracketed by barrier + synchronize; then the
-    dominant kernel alone over K launches on the same slots."""
+    """Device time of exactly K steps (CUDA-graph replays of whole rotations of
+    the input slots, then single steps for K mod R), bracketed by barrier +
+    synchronize; the per-step distribution from K single-step replays, each
+    between its own events; then the dominant kernel alone over K calls the
+    same way."""
     for i in range(W):                       # eager warm-up (also resolves lazy set-up)
         wl.step(i)
     torch.cuda.synchronize()
     steps = _capture(torch, wl.step, wl.R)
     kern = _capture(torch, wl.dominant_call, wl.R)
+    steps_rot = _capture_rotation(torch, wl.step, wl.R)
+    kern_rot = _capture_rotation(torch, wl.dominant_call, wl.R)
     for i in range(W):
         steps[i % wl.R].replay()
+    steps_rot.replay()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
@@ -423,8 +448,7 @@ def measure(wl, torch, K, W, world, local, sample_clocks=False):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with (sampler if sampler else _Null()):
         start.record()
-        for i in range(K):
-            steps[(W + i) % wl.R].replay()
+        _replay_k(steps, steps_rot, wl.R, K)
         end.record()
         torch.cuda.synchronize()
     barrier(world)
@@ -442,15 +466,15 @@ def measure(wl, torch, K, W, world, local, sample_clocks=False):
             "p90": round(per[int(0.9 * (K - 1))], 2), "unit": "us", "rank": "local"}
     for i in range(W):
         kern[i % wl.R].replay()
+    kern_rot.replay()
     torch.cuda.synchronize()
     ks, ke = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ks.record()
-    for i in range(K):
-        kern[(W + i) % wl.R].replay()
+    _replay_k(kern, kern_rot, wl.R, K)
     ke.record()
     torch.cuda.synchronize()
     kern_us = max_over_ranks(world, ks.elapsed_time(ke) * 1e3 / K)
-    del steps, kern
+    del steps, kern, steps_rot, kern_rot
     return elapsed, kern_us, (sampler.summary() if sampler else None), dist
 
 
