@@ -43,6 +43,11 @@
  *     sums in the scratch (zero-filled by the call itself, so workspaces may
  *     be shared between operations and shapes that do not overlap in time).
  *     Calls that share one workspace must not overlap on the GPU.
+ *   - Kernel choice is automatic.  Two environment switches, read at each
+ *     call, exist for A/B measurements: NVFP4_GEMM_CTA_PAIR=0 keeps large-M
+ *     GEMMs on the one-CTA kernel; NVFP4_GEMM_STREAMK=0 disables the split-K
+ *     (stream-K) path for GEMMs with few output tiles.  Results stay within
+ *     the same tolerance either way.
  */
 #ifndef NVFP4_H
 #define NVFP4_H

@@ -21,10 +21,10 @@ __host__ __device__ __forceinline__ int64_t kb4_of(int64_t cols) { return round_
 
 // Byte offset of the scale of block kb of row r in the tiled layout: 128-row x
 // 4-block atoms of 512 bytes, row r%32 at 16*(r%32), row quarter (r/32)%4 at
-// 4*((r/32)%4), block kb%4 at kb%4.  This is the order in which tcgen05.cp
-// (32x128b, replicated to four lane quarters) places scales where the
-// block-scaled MMA reads them: lane r%32 of every quarter, column (r/32)%4,
-// byte kb%4.
+// 4*((r/32)%4), block kb%4 at kb%4.  Lane l of every TMEM lane quarter
+// receives the atom's 16 bytes at 16*l (the GEMMs' scale warps copy them with
+// tcgen05.st), which is where the block-scaled MMA reads the scales: lane
+// r%32 of every quarter, column (r/32)%4, byte kb%4.
 __host__ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t kb, int64_t kb4) {
     int64_t tile = (r >> 7) * (kb4 >> 2) + (kb >> 2);
     return tile * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3);

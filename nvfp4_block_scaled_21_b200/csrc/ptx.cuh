@@ -136,7 +136,7 @@ __device__ __forceinline__ uint64_t policy_evict_normal() {
 }
 
 // Make generic-proxy writes to shared memory visible to the async proxy
-// (tensor-core operand reads, tcgen05.cp).
+// (tensor-core operand reads, TMA stores).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -225,20 +225,6 @@ __device__ __forceinline__ void tc_commit(uint64_t *bar) {
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             smem_addr(bar))
         : "memory");
-}
-
-// Copy 32 rows x 16 bytes from shared memory (descriptor) into TMEM lanes
-// 0..31, columns taddr..taddr+3, replicated into all four 32-lane quarters.
-__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
-}
-
-// Each thread of the warp writes 4 consecutive 32-bit columns of its lane.
-__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr),
-                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
 }
 
 // Each thread of the warp writes 16 (32) consecutive 32-bit columns of its lane.
@@ -351,12 +337,6 @@ __device__ __forceinline__ uint64_t make_operand_desc(uint32_t saddr) {
     return make_smem_desc(saddr, 16, 1024, 2);
 }
 
-// Scale-factor atom for tcgen05.cp 32x128b: 32 rows of 16 bytes, 8-row core
-// matrices 128 bytes apart, no swizzle.
-__device__ __forceinline__ uint64_t make_sf_desc(uint32_t saddr) {
-    return make_smem_desc(saddr, 0, 128, 0);
-}
-
 // Instruction descriptor of kind::mxf4nvf4 with E2M1 A and B, UE4M3 scales,
 // K-major A and B, dense K = 64, M = 128, and the given N (multiple of 8/16).
 __host__ __device__ constexpr uint32_t make_idesc_nvf4(uint32_t n) {
@@ -410,18 +390,6 @@ __device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorM
         : "memory");
 }
 
-// 3-D tiled load, otherwise as tma_load_2d_pair (used for scale-factor atoms:
-// x = 32-bit word within a 512-byte atom, y = K-step, z = 128-row tile).
-__device__ __forceinline__ void tma_load_3d_pair(void *smem_dst, const CUtensorMap *map,
-                                                 uint32_t leader_bar, int32_t c0, int32_t c1,
-                                                 int32_t c2, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_addr(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(leader_bar), "l"(policy)
-        : "memory");
-}
-
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(dst)),
@@ -457,14 +425,6 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t *bar, uint16_t mask) {
         " [%0], %1;" ::"r"(smem_addr(bar)),
         "h"(mask)
         : "memory");
-}
-
-// Pair form of the scale copy, issued by the leader: each CTA's 32 rows x 16
-// bytes at the descriptor's shared-memory offset go to that CTA's TMEM lanes
-// 0..31 (replicated to the four lane quarters), columns taddr..taddr+3.
-__device__ __forceinline__ void tc_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
 }
 
 // Instruction descriptor of the pair MMA: M = 256.
