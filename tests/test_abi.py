@@ -42,6 +42,30 @@ def test_sizes():
     assert nv.version() >= 100
 
 
+def test_workspace_sizes_follow_the_kernel_choices():
+    """GEMM-bearing ops reserve fp32 stream-K scratch (the padded output tile
+    grid plus one counter per 128x128 tile) only for shapes with at most 1024
+    output tiles; the fused MLP keeps fp32 h; quantize keeps the pass-1
+    partial maxima."""
+    a256 = lambda v: (v + 255) // 256 * 256
+    # decode-shaped (M <= 64, swapped): roundup(N,128) x 64 floats + ceil(N/128) counters
+    M, N, K = 8, 17408, 5120
+    assert nv.workspace_bytes(nv.OP_GEMM, M, N, K) == 256 + a256(17408 * 64 * 4) + a256(136 * 4)
+    # 128-row activations: roundup(M,128) x roundup(N,128) floats + tiles counters
+    M, N = 128, 5120
+    assert nv.workspace_bytes(nv.OP_GEMM, M, N, 17408) == 256 + a256(128 * 5120 * 4) + a256(40 * 4)
+    # prefill-sized: 32 x 136 = 4352 tiles > 1024, no scratch
+    assert nv.workspace_bytes(nv.OP_GEMM, 4096, 17408, 5120) == 256
+    # the fused MLP: status + partials, x_q (codes, scales, g) and fp32 h, no stream-K scratch
+    M, N, K = 128, 17408, 5120
+    xq = a256(M * K // 2) + a256(((M + 127) // 128 * 128) * (K // 16)) + 256
+    assert nv.workspace_bytes(nv.OP_LINEAR_FUSED_SILU, M, N, K) == 256 + 4096 * 4 + xq + a256(M * N * 4)
+    # the plain linear layer adds the GEMM's stream-K scratch after x_q
+    M, N = 128, 5120
+    xq = a256(M * K // 2) + a256(128 * (K // 16)) + 256
+    assert nv.workspace_bytes(nv.OP_LINEAR_FUSED, M, N, K) == 256 + 4096 * 4 + xq + a256(128 * 5120 * 4) + a256(40 * 4)
+
+
 def test_status_strings():
     assert nv.status_string(nv.OK) == "ok"
     assert "timed out" in nv.status_string(nv.ERR_TIMEOUT)
