@@ -156,7 +156,8 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor *q, void *y, nvfp4_dt
  * y[M][N] = (A . B^T) * gA * gB with A = a [M][K], B = b [N][K] (K = a->cols
  * = b->cols, K % 64 == 0), both NVFP4, consumed directly by tcgen05
  * block-scaled FP4 MMAs with fp32 accumulation in tensor memory.  y has row
- * pitch ldy (elements) and dtype yt (BF16 or F32).  W4A4 linear layer: a is
+ * pitch ldy (elements) and dtype yt (BF16 or F32); y may be NULL when M*N == 0
+ * (nothing is written), and K == 0 zero-fills y.  W4A4 linear layer: a is
  * the activations, b the weights.
  */
 NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y, nvfp4_dtype yt,

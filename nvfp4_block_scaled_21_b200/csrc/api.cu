@@ -152,7 +152,8 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor *q, void *y, nvfp4_dtype yt, in
 
 static nvfp4_status check_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y,
                                nvfp4_dtype yt, int64_t ldy) {
-    if (!a || !b || !y || (yt != NVFP4_F32 && yt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if (!a || !b || (yt != NVFP4_F32 && yt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if (!y && a->rows * b->rows != 0) return NVFP4_ERR_INVALID_ARG;   // an empty y may be NULL
     if (a->cols != b->cols) return NVFP4_ERR_INVALID_ARG;
     nvfp4_status st = check_tensor(a, a->rows, a->cols);
     if (st != NVFP4_OK) return st;
@@ -210,7 +211,8 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
     if (!aligned16(x) || (ldx * xeb) % 16) return NVFP4_ERR_MISALIGNED;
     const int64_t N = w->rows;
     if (epilogue == NVFP4_EPI_STORE) {
-        if (!y || (yt != NVFP4_F32 && yt != NVFP4_BF16) || ldy < N) return NVFP4_ERR_INVALID_ARG;
+        if ((!y && M * N != 0) || (yt != NVFP4_F32 && yt != NVFP4_BF16) || ldy < N)
+            return NVFP4_ERR_INVALID_ARG;
         if (!aligned16(y) || (ldy * (yt == NVFP4_BF16 ? 2 : 4)) % 16) return NVFP4_ERR_MISALIGNED;
     } else {
         if (!w_up || (st = check_tensor(w_up, N, K)) != NVFP4_OK)

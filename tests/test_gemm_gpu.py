@@ -176,6 +176,28 @@ def test_gemm_special_operands(nv):
     assert torch.all(y == -128 * 2688.0 * 5376.0)
 
 
+def test_gemm_degenerate_shapes(nv):
+    """M = 0 and N = 0 launch nothing and write nothing; K = 0 is an empty
+    reduction, so y is all zeros."""
+    b = quantize_gpu(nv, torch.randn((40, 64), device="cuda"))
+    a0 = nv.NVFP4Tensor.empty(0, 64)
+    y0 = torch.empty((0, 40), dtype=torch.bfloat16, device="cuda")
+    ws = nv.workspace(nv.OP_GEMM, 0, 40, 64)
+    nv.nvfp4_gemm(a0, b, y0, ws)
+    a = quantize_gpu(nv, torch.randn((5, 64), device="cuda"))
+    b0 = nv.NVFP4Tensor.empty(0, 64)
+    buf = torch.full((5, 8), float("nan"), dtype=torch.float32, device="cuda")
+    nv.nvfp4_gemm(a, b0, buf[:, :0], nv.workspace(nv.OP_GEMM, 5, 0, 64))
+    assert torch.isnan(buf).all()                                # nothing written
+    ak, bk = nv.NVFP4Tensor.empty(5, 0), nv.NVFP4Tensor.empty(8, 0)
+    yk = torch.full((5, 8), float("nan"), dtype=torch.float32, device="cuda")
+    ws = nv.workspace(nv.OP_GEMM, 5, 8, 0)
+    nv.nvfp4_gemm(ak, bk, yk, ws)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(yk) == 0
+    assert nv.nvfp4_get_device_status(ws) == nv.OK
+
+
 def test_decode_workload_full(nv):
     """M=8, N=17408, K=5120 (seed 2): every output against the fp64 oracle."""
     w = workloads.make("decode")
