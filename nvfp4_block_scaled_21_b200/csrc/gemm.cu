@@ -275,11 +275,19 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     tc_fence_after();
                     const int nk = min(4, args.num_k_steps - 4 * ks);
                     const uint32_t sf = tmem_base + C::kSfBase + stage * C::kSfCols;
-                    for (int j = 0; j < nk; ++j) {
-                        const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage + 32 * j);
-                        const uint64_t bdesc = make_operand_desc(b_base + stage * C::kBStage + 32 * j);
-                        mma_nvf4(d_tmem, adesc, bdesc, idesc, sf + 4 * j, sf + 16 + 4 * C::kNQT * j,
-                                 (ks != sg.ks0 || j != 0) ? 1u : 0u);
+                    // K-step j: +32 bytes = +2 in the descriptors' address field
+                    const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage);
+                    const uint64_t bdesc = make_operand_desc(b_base + stage * C::kBStage);
+                    const uint32_t acc0 = ks != sg.ks0 ? 1u : 0u;
+                    if (nk == 4) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            mma_nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j,
+                                     sf + 16 + 4 * C::kNQT * j, (acc0 | j) != 0 ? 1u : 0u);
+                    } else {
+                        for (int j = 0; j < nk; ++j)
+                            mma_nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j,
+                                     sf + 16 + 4 * C::kNQT * j, (acc0 | j) != 0 ? 1u : 0u);
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }

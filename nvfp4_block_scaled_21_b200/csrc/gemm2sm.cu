@@ -234,11 +234,19 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                         tc_fence_after();
                         const int nk = min(4, args.num_k_steps - 4 * ks);
                         const uint32_t sf = tmem_base + C::kSfCol + slot * C::kSlotCols + h * C::kSlabCols;
-                        for (int j = 0; j < nk; ++j) {
-                            const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage + 32 * j);
-                            const uint64_t bdesc = make_operand_desc(b_base + stage * C::kBStage + 32 * j);
-                            mma_nvf4_pair(tmem_base, adesc, bdesc, idesc, sf + 4 * j, sf + 16 + 8 * j,
-                                          (ks | j) != 0 ? 1u : 0u);
+                        // K-step j is 32 bytes further along the swizzled rows: +2 in
+                        // the descriptors' address field (units of 16 bytes)
+                        const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage);
+                        const uint64_t bdesc = make_operand_desc(b_base + stage * C::kBStage);
+                        if (nk == 4) {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                mma_nvf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j,
+                                              sf + 16 + 8 * j, (ks | j) != 0 ? 1u : 0u);
+                        } else {
+                            for (int j = 0; j < nk; ++j)
+                                mma_nvf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j,
+                                              sf + 16 + 8 * j, (ks | j) != 0 ? 1u : 0u);
                         }
                         tc_commit_pair(&empty[stage], 0x3);
                         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
