@@ -186,13 +186,21 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                     tc_fence_after();
                     const int nk = min(4, args.num_k_steps - 4 * ks);
                     const uint32_t sf = tmem_base + C::kSfBase + stage * C::kSfCols;
-                    for (int j = 0; j < nk; ++j) {
-                        const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage + 32 * j);
+                    // K-step j: +32 bytes = +2 in the descriptors' address field
+                    const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage);
+                    const uint64_t gdesc = make_operand_desc(bg_base + stage * C::kBStage);
+                    const uint64_t udesc = make_operand_desc(bu_base + stage * C::kBStage);
+                    auto kstep = [&](int j) {
                         const uint32_t acc = (ks | j) != 0 ? 1u : 0u;
-                        mma_nvf4(tmem_base, adesc, make_operand_desc(bg_base + stage * C::kBStage + 32 * j), idesc,
-                                 sf + 4 * j, sf + 16 + 4 * j, acc);
-                        mma_nvf4(tmem_base + 128, adesc, make_operand_desc(bu_base + stage * C::kBStage + 32 * j),
-                                 idesc, sf + 4 * j, sf + 32 + 4 * j, acc);
+                        mma_nvf4(tmem_base, adesc + 2 * j, gdesc + 2 * j, idesc, sf + 4 * j, sf + 16 + 4 * j, acc);
+                        mma_nvf4(tmem_base + 128, adesc + 2 * j, udesc + 2 * j, idesc, sf + 4 * j, sf + 32 + 4 * j,
+                                 acc);
+                    };
+                    if (nk == 4) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) kstep(j);
+                    } else {
+                        for (int j = 0; j < nk; ++j) kstep(j);
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
