@@ -7,7 +7,8 @@
 // scales are applied once in the epilogue (NVFP4 wiki page, section "技術原理":
 // a second-level FP32 scale over the whole tensor).
 //
-// Design (one persistent CTA per SM, 10 warps):
+// Design (one persistent CTA per SM, 14 warps; large M runs on the CTA-pair
+// kernel of gemm2sm.cu instead):
 //   warp 0      TMA producer: for every 256-element K slab, a 128-row tile of
 //               the MMA's A operand and a BN-row tile of its B operand (packed
 //               E2M1, 128-byte swizzle) plus their 512-byte scale atoms (bulk
@@ -19,9 +20,10 @@
 //               memory into its own 32-lane quarter of tensor memory with
 //               tcgen05.st (the four quarters hold the same scales, which is the
 //               replicated layout the block-scaled MMA reads), into a TMEM scale
-//               slot owned by the stage.  This keeps scale movement off the
-//               tensor pipe, where a tcgen05.cp per 512-byte atom would cost
-//               about as much tensor-pipe time as the MMAs themselves.
+//               slot owned by the stage, handing stages to the MMA two at a
+//               time.  This keeps scale movement off the tensor pipe, where a
+//               tcgen05.cp per 512-byte atom would cost about as much
+//               tensor-pipe time as the MMAs themselves.
 //   warps 6..13 epilogue, two warps per TMEM lane quarter, each owning half
 //               of the tile's columns (bf16 output, tiles >= 64 wide):
 //               tcgen05.ld of the accumulator with the next chunk in flight,
@@ -29,6 +31,10 @@
 //               released to the MMA warp as soon as both halves are read.
 // Small M (decode) runs "swapped": the weights ride the MMA's M = 128 and the
 // few activation rows ride N = BN, so the weight stream spreads over all SMs.
+// When the output tiles would leave at least half of the SMs idle, CTAs take
+// equal runs of (tile, K slab) units instead of whole tiles (stream-K): partial
+// tiles are added in fp32 in the workspace and the CTA that completes a
+// tile's K range writes it.
 // When the weights are known not to come from the kernel launched just before
 // (inside nvfp4_linear_fused), the producer starts streaming them before the
 // programmatic-dependent-launch wait, hiding the pipeline fill behind the
