@@ -26,7 +26,10 @@
  *
  * Conventions for every entry point:
  *   - All pointers are DEVICE pointers owned by the caller, 16-byte aligned.
- *     Row pitches (ld, in elements) must keep every row 16-byte aligned.
+ *     Row pitches (ld, in elements) must keep every row 16-byte aligned.  An
+ *     empty matrix (a zero dimension) is never read or written: its data
+ *     pointer may be NULL and its pointer and pitch are not checked (a pitch
+ *     must still be at least the row length).
  *   - Calls are asynchronous and stream-ordered on `stream`; none allocates
  *     memory and none synchronises, except nvfp4_get_device_status.
  *   - Argument errors are returned synchronously and launch nothing.
@@ -178,6 +181,9 @@ NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, 
  *     not NULL it receives h itself in fp32 (yt must be F32), for inspection.
  *   If x_q is not NULL it receives the quantized activations (x_q->rows == M,
  *   x_q->cols == K); otherwise they live in ws.
+ *   K == 0 is an empty reduction: the STORE form zero-fills y; the SiLU form
+ *   gives h = 0, so y_q gets zero codes and scales and g = 0 (and y, if
+ *   given, zeros).  M == 0 writes nothing; N == 0 writes only y_q's g (0).
  */
 NVFP4_API nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_t K, int64_t ldx,
                                 const nvfp4_tensor *w, const nvfp4_tensor *w_up,

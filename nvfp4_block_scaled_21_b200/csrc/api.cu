@@ -124,7 +124,8 @@ nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype xt, int64_t rows, int64_t
     nvfp4_status st = check_tensor(out, rows, cols);
     if (st != NVFP4_OK) return st;
     const int eb = xt == NVFP4_BF16 ? 2 : 4;
-    if (!aligned16(x) || (ld * eb) % 16) return NVFP4_ERR_MISALIGNED;
+    // an empty x is never read: its pointer and pitch are not checked
+    if (rows * cols != 0 && (!aligned16(x) || (ld * eb) % 16)) return NVFP4_ERR_MISALIGNED;
     if ((st = check_ws(ws, ws_bytes, kQuantizeWs)) != NVFP4_OK) return st;
     DevInfo dev;
     if ((st = current_device(&dev)) != NVFP4_OK) return st;
@@ -136,12 +137,14 @@ nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype xt, int64_t rows, int64_t
 
 nvfp4_status nvfp4_dequantize(const nvfp4_tensor *q, void *y, nvfp4_dtype yt, int64_t ldy,
                               nvfp4_stream_t stream) {
-    if (!q || !y || (yt != NVFP4_F32 && yt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if (!q || (yt != NVFP4_F32 && yt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
     nvfp4_status st = check_tensor(q, q->rows, q->cols);
     if (st != NVFP4_OK) return st;
+    const bool empty = q->rows * q->cols == 0;     // an empty y may be NULL, any pitch
+    if (!y && !empty) return NVFP4_ERR_INVALID_ARG;
     const int eb = yt == NVFP4_BF16 ? 2 : 4;
     if (ldy < q->cols) return NVFP4_ERR_INVALID_ARG;
-    if (!aligned16(y) || (ldy * eb) % 16) return NVFP4_ERR_MISALIGNED;
+    if (!empty && (!aligned16(y) || (ldy * eb) % 16)) return NVFP4_ERR_MISALIGNED;
     DevInfo dev;
     if ((st = current_device(&dev)) != NVFP4_OK) return st;
     if (q->rows == 0 || q->cols == 0) return NVFP4_OK;
@@ -162,7 +165,7 @@ static nvfp4_status check_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, voi
     if (a->rows > INT32_MAX / 2 || b->rows > INT32_MAX / 2) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (ldy < b->rows) return NVFP4_ERR_INVALID_ARG;
     const int eb = yt == NVFP4_BF16 ? 2 : 4;
-    if (!aligned16(y) || (ldy * eb) % 16) return NVFP4_ERR_MISALIGNED;
+    if (a->rows * b->rows != 0 && (!aligned16(y) || (ldy * eb) % 16)) return NVFP4_ERR_MISALIGNED;
     return NVFP4_OK;
 }
 
@@ -200,7 +203,7 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
                                 const nvfp4_tensor *y_q, const nvfp4_tensor *x_q, void *ws,
                                 size_t ws_bytes, nvfp4_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    if (!x || !w || (xt != NVFP4_F32 && xt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if ((!x && M * K != 0) || !w || (xt != NVFP4_F32 && xt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
     if (M < 0 || K < 0 || ldx < K) return NVFP4_ERR_INVALID_ARG;
     if (epilogue != NVFP4_EPI_STORE && epilogue != NVFP4_EPI_SILU_MUL_REQUANT)
         return NVFP4_ERR_INVALID_ARG;
@@ -208,18 +211,19 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
     if (st != NVFP4_OK) return st;
     if (K % 64) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const int xeb = xt == NVFP4_BF16 ? 2 : 4;
-    if (!aligned16(x) || (ldx * xeb) % 16) return NVFP4_ERR_MISALIGNED;
+    if (M * K != 0 && (!aligned16(x) || (ldx * xeb) % 16)) return NVFP4_ERR_MISALIGNED;
     const int64_t N = w->rows;
     if (epilogue == NVFP4_EPI_STORE) {
         if ((!y && M * N != 0) || (yt != NVFP4_F32 && yt != NVFP4_BF16) || ldy < N)
             return NVFP4_ERR_INVALID_ARG;
-        if (!aligned16(y) || (ldy * (yt == NVFP4_BF16 ? 2 : 4)) % 16) return NVFP4_ERR_MISALIGNED;
+        if (M * N != 0 && (!aligned16(y) || (ldy * (yt == NVFP4_BF16 ? 2 : 4)) % 16))
+            return NVFP4_ERR_MISALIGNED;
     } else {
         if (!w_up || (st = check_tensor(w_up, N, K)) != NVFP4_OK)
             return st != NVFP4_OK ? st : NVFP4_ERR_INVALID_ARG;
         if ((st = check_tensor(y_q, M, N)) != NVFP4_OK) return st;
         if (y && (yt != NVFP4_F32 || ldy < N)) return NVFP4_ERR_INVALID_ARG;
-        if (y && (!aligned16(y) || (ldy * 4) % 16)) return NVFP4_ERR_MISALIGNED;
+        if (y && M * N != 0 && (!aligned16(y) || (ldy * 4) % 16)) return NVFP4_ERR_MISALIGNED;
     }
     if (x_q && (st = check_tensor(x_q, M, K)) != NVFP4_OK) return st;
     const nvfp4_op op = epilogue == NVFP4_EPI_STORE ? NVFP4_OP_LINEAR_FUSED : NVFP4_OP_LINEAR_FUSED_SILU;
@@ -252,6 +256,19 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
     if (epilogue == NVFP4_EPI_STORE)
         return gemm_impl(&xq, w, y, yt, ldy, status, dev.sms, stream, true,
                          splitk_ws_bytes(M, N) != 0 ? ws_at(ws, kQuantizeWs + quantized_bytes(M, K)) : nullptr);
+
+    // An empty reduction (K == 0) makes gate = up = 0, so h = SiLU(0) * 0 = 0:
+    // y_q gets all-zero codes and scales and g = 0, y (if given) zeros.  With
+    // N == 0 only the tensor scale is written.
+    if (N == 0 || K == 0) {
+        if (cudaMemsetAsync(y_q->tensor_scale, 0, sizeof(float), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
+        if (N == 0) return NVFP4_OK;
+        if (cudaMemsetAsync(y_q->codes, 0, nvfp4_codes_bytes(M, N), stream) != cudaSuccess ||
+            cudaMemsetAsync(y_q->scales, 0, nvfp4_scales_bytes(M, N), stream) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        if (y) return from_cuda(cudaMemset2DAsync(y, ldy * sizeof(float), 0, N * sizeof(float), M, stream));
+        return NVFP4_OK;
+    }
 
     // Gate and up in one GEMM whose epilogue writes h = SiLU(gate) * up and the
     // per-CTA max |h|; then the quantizer's encode pass turns h into NVFP4.

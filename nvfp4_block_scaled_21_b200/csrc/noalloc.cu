@@ -92,9 +92,10 @@ extern "C" nvfp4_status nvfp4_linear_noalloc(const void *x, nvfp4_dtype xt, int6
     if (st != NVFP4_OK) return st;
     if (K % 64) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const int64_t N = w->rows;
-    if (!y || (yt != NVFP4_F32 && yt != NVFP4_BF16) || ldy < N) return NVFP4_ERR_INVALID_ARG;
+    if ((!y && M * N != 0) || (yt != NVFP4_F32 && yt != NVFP4_BF16) || ldy < N) return NVFP4_ERR_INVALID_ARG;
     const int xeb = xt == NVFP4_BF16 ? 2 : 4, yeb = yt == NVFP4_BF16 ? 2 : 4;
-    if (!aligned16(x) || (ldx * xeb) % 16 || !aligned16(y) || (ldy * yeb) % 16)
+    // empty operands are never touched: their pointers and pitches are not checked
+    if ((M * K != 0 && (!aligned16(x) || (ldx * xeb) % 16)) || (M * N != 0 && (!aligned16(y) || (ldy * yeb) % 16)))
         return NVFP4_ERR_MISALIGNED;
     if (M > INT32_MAX / 2 || N > INT32_MAX / 2) return NVFP4_ERR_UNSUPPORTED_SHAPE;
 

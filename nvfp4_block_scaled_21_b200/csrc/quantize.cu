@@ -472,6 +472,8 @@ static int resident_ctas(K kernel) {
 cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld,
                             uint8_t *codes, uint8_t *scales, float *g_out, float *partials,
                             int num_sms, cudaStream_t stream) {
+    // An empty tensor has no codes and no scale bytes; its amax is 0, so g = 0.
+    if (rows == 0 || cols == 0) return cudaMemsetAsync(g_out, 0, sizeof(float), stream);
     const int eb = bf16 ? 2 : 4;
     static const int occ_amax[2] = {resident_ctas(amax_partials_kernel<float>),
                                     resident_ctas(amax_partials_kernel<__nv_bfloat16>)};

@@ -119,6 +119,26 @@ def test_linear_fused_rejects_bad_arguments_without_launch():
     assert f(nv.EPI_SILU_MUL_REQUANT, _t(rows=16, cols=128), _t(rows=8, cols=32), None) == nv.ERR_INVALID_ARG
 
 
+def test_empty_operands_skip_pointer_and_pitch_checks():
+    """An empty matrix is never read or written: a NULL pointer and any pitch
+    at least its row length pass validation.  Each call below then stops at
+    the too-small workspace, before any launch."""
+    lib = nv.lib()
+    small = 8                                                    # below every workspace size
+    out = _t(codes=None, scales=None, rows=5, cols=0)            # quantize 5 x 0, x = NULL, pitch 1
+    assert lib.nvfp4_quantize(None, nv.F32, 5, 0, 1, ctypes.byref(out), 4096, small, None) == nv.ERR_WORKSPACE
+    a, b0 = _t(rows=8, cols=128), _t(codes=None, scales=None, rows=0, cols=128)   # GEMM with N = 0
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b0), None, nv.BF16, 1, 4096, small, None) == nv.ERR_WORKSPACE
+    w0 = _t(codes=None, scales=None, rows=32, cols=0)            # linear layer with K = 0, x = NULL
+    assert lib.nvfp4_linear_fused(None, nv.BF16, 8, 0, 1, ctypes.byref(w0), None, nv.EPI_STORE, 16, nv.BF16,
+                                  32, None, None, 4096, small, None) == nv.ERR_WORKSPACE
+    q0 = _t(codes=None, scales=None, rows=0, cols=64)            # dequantize of 0 x 64, y = NULL
+    assert lib.nvfp4_dequantize(ctypes.byref(q0), None, nv.F32, 64, None) in (nv.OK, nv.ERR_CUDA, nv.ERR_ARCH)
+    # a non-empty operand still has its pitch checked
+    assert lib.nvfp4_quantize(16, nv.F32, 5, 16, 17, ctypes.byref(_t(rows=5, cols=16)), 4096, small,
+                              None) == nv.ERR_MISALIGNED
+
+
 def test_package_fails_loudly_without_library(tmp_path):
     """The binding refuses to import when libnvfp4.so is absent: no CPU fallback."""
     import subprocess

@@ -106,6 +106,47 @@ def test_mlp_ragged_tiles(nv):
     check_mlp(nv, w["X"], w["Wg"], w["Wu"], w["Wd"], M, K, N)
 
 
+def test_linear_degenerate_shapes(nv):
+    """K = 0 is an empty reduction: the STORE form writes zeros and the
+    quantized x has g = 0; the SiLU form gives h = SiLU(0) * 0 = 0, so y_q has
+    all-zero codes and scales and g = 0.  With N = 0 the SiLU form writes
+    only y_q's g."""
+    M, N = 5, 64
+    x = torch.empty((M, 0), dtype=torch.bfloat16, device="cuda")
+    w, wu = nv.NVFP4Tensor.empty(N, 0), nv.NVFP4Tensor.empty(N, 0)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    xq = nv.NVFP4Tensor.empty(M, 0)
+    xq.tensor_scale.fill_(7.0)
+    ws = nv.workspace(nv.OP_LINEAR_FUSED, M, N, 0)
+    nv.nvfp4_linear_fused(x, w, ws, nv.EPI_STORE, y=y, x_q=xq)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(y) == 0 and xq.tensor_scale[0].item() == 0.0
+    assert nv.nvfp4_get_device_status(ws) == nv.OK
+
+    yq = nv.NVFP4Tensor.empty(M, N)
+    yq.codes.fill_(0x77)
+    yq.scales.fill_(0x38)
+    yq.tensor_scale.fill_(7.0)
+    h = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    ws = nv.workspace(nv.OP_LINEAR_FUSED_SILU, M, N, 0)
+    nv.nvfp4_linear_fused(x, w, ws, nv.EPI_SILU_MUL_REQUANT, y=h, w_up=wu, y_q=yq)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(h) == 0
+    assert torch.count_nonzero(yq.codes) == 0 and torch.count_nonzero(yq.scales) == 0
+    assert yq.tensor_scale[0].item() == 0.0
+    assert nv.nvfp4_get_device_status(ws) == nv.OK
+
+    x1 = torch.randn((M, 64), device="cuda").to(torch.bfloat16)
+    yq0 = nv.NVFP4Tensor.empty(M, 0)
+    yq0.tensor_scale.fill_(7.0)
+    ws = nv.workspace(nv.OP_LINEAR_FUSED_SILU, M, 0, 64)
+    nv.nvfp4_linear_fused(x1, nv.NVFP4Tensor.empty(0, 64), ws, nv.EPI_SILU_MUL_REQUANT,
+                          w_up=nv.NVFP4Tensor.empty(0, 64), y_q=yq0)
+    torch.cuda.synchronize()
+    assert yq0.tensor_scale[0].item() == 0.0
+    assert nv.nvfp4_get_device_status(ws) == nv.OK
+
+
 def test_mlp_workload_full(nv):
     """The fused MLP workload at full size: M=128, K=5120, N=17408 (seed 4)."""
     w = workloads.make("mlp")

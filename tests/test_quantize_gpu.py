@@ -144,8 +144,14 @@ def test_block_scale_ties_and_boundaries(nv):
     assert_quantized_equal(quantize_gpu(nv, f32_tensor(x)), oracle.quantize(x))
 
 
-def test_quantize_empty(nv):
-    out = quantize_gpu(nv, torch.zeros((0, 64), device="cuda"))
+@pytest.mark.parametrize("shape", [(0, 64), (5, 0), (0, 0)])
+def test_quantize_empty(nv, shape):
+    """An empty tensor has no codes and no scale bytes; its amax is 0, so g = 0
+    (written even though nothing else is)."""
+    out = nv.NVFP4Tensor.empty(*shape)
+    out.tensor_scale.fill_(7.0)
+    x = torch.zeros(shape, device="cuda")
+    nv.nvfp4_quantize(x, out, nv.workspace(nv.OP_QUANTIZE, shape[0], 0, shape[1]))
     torch.cuda.synchronize()
     assert out.tensor_scale[0].item() == 0.0
 
