@@ -138,6 +138,25 @@ def test_gemm_cta_pair_tiles(nv, M, N, K, pair, monkeypatch):
     assert np.isfinite(yc).all()
 
 
+def test_gemm_cta_pair_f32_output(nv, monkeypatch):
+    """The two-CTA kernel's fp32 epilogue (per-row stores; the TMA-store path
+    is bf16 only), with ragged M and N: sampled outputs plus the last row and
+    column, and nothing written past N."""
+    monkeypatch.setenv("NVFP4_GEMM_CTA_PAIR", "1")
+    M, N, K = 2000, 4616, 256
+    rng = np.random.default_rng(77)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    wt = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    xq_o, wq_o = oracle.quantize(x), oracle.quantize(wt)
+    y = run_gemm(nv, quantize_gpu(nv, f32_tensor(x)), quantize_gpu(nv, f32_tensor(wt)), torch.float32)
+    yc = to_numpy_f64(y)
+    ms = np.concatenate([rng.integers(0, M, 4000), np.full(N, M - 1), np.arange(M)])
+    ns = np.concatenate([rng.integers(0, N, 4000), np.arange(N), np.full(M, N - 1)])
+    ref, na, nb = oracle.gemm_entries(xq_o, wq_o, ms, ns)
+    assert_gemm_close(yc[ms, ns], ref, na, nb, K, False, f"pair f32 {M}x{N}x{K}")
+    assert np.isfinite(yc).all()
+
+
 @pytest.mark.parametrize("M,N,K,dt", [(24, 1000, 1088, torch.bfloat16), (8, 17408, 5120, torch.float32),
                                       (200, 700, 2048, torch.bfloat16), (130, 520, 4096, torch.float32)])
 def test_gemm_stream_k(nv, M, N, K, dt):
