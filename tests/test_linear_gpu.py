@@ -53,6 +53,27 @@ def test_linear_store(nv, M, N, K):
     assert_gemm_close(to_numpy_f64(y), ref, norms(xq_o)[:, None], norms(wq_o)[None, :], K, True, "linear")
 
 
+@pytest.mark.parametrize("M,N,K", [(12, 256, 320), (20, 200, 576)])
+def test_linear_store_f32_pitch(nv, M, N, K):
+    """fp32 activations with a row pitch wider than K, the quantized
+    activations kept in the workspace (x_q not requested), fp32 output."""
+    rng = np.random.default_rng(5 * M + N)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[rng.random(x.shape) < 1e-3] *= 50
+    wt = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    xq_o, wq_o = oracle.quantize(x), oracle.quantize(wt)
+    wq = quantize_gpu(nv, f32_tensor(wt))
+    buf = torch.zeros((M, K + 16), dtype=torch.float32, device="cuda")
+    buf[:, :K] = f32_tensor(x)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    ws = nv.workspace(nv.OP_LINEAR_FUSED, M, N, K)
+    nv.nvfp4_linear_fused(buf[:, :K], wq, ws, nv.EPI_STORE, y=y)
+    assert nv.nvfp4_get_device_status(ws) == nv.OK
+    ref = oracle.gemm_f64(xq_o, wq_o)
+    assert_gemm_close(to_numpy_f64(y), ref, norms(xq_o)[:, None], norms(wq_o)[None, :], K, False,
+                      "linear fp32 pitch")
+
+
 def _silu(z):
     return z / (1.0 + np.exp(-z))
 
