@@ -16,6 +16,7 @@ import pytest
 import torch
 
 import oracle
+import reading_vectors
 from nvfp4_block_scaled_21_b200 import workloads
 
 pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
@@ -235,6 +236,37 @@ def test_codes_are_nearest_grid_points(random_case, facts):
             mag = cand[0] if len(cand) == 1 else cand[cand % 2 == 0][0]
             sign = 8 if np.signbit(v) else 0
             assert codes[r, c] == (sign | mag), (r, c, v)
+
+
+def test_element_step_multiplies_by_the_rounded_reciprocal():
+    """The element step is v = fl32(x * fl32(1/d)) (one correctly rounded
+    reciprocal per block, then a multiply), not x / d: on vector A of
+    reading_vectors the two readings round the same x to different E2M1
+    codes."""
+    (a, ga), _ = reading_vectors.vectors()
+    f = np.float32
+    x, d = a[0, 17], ga                                  # block 1 scale is E4M3 1.0: d = g
+    assert f(x / d) == f(2.5)                            # exact quotient: a tie -> even index (2.0)
+    assert f(x * (f(1) / d)) > f(2.5)                    # the reciprocal reading: above the tie -> 3.0
+    q = oracle.quantize(a)
+    assert q.g == ga and q.scales[0, 1] == 0x38
+    assert q.codes[0, 8] == 0x57                         # 6g -> 6.0 (7), 2.5g -> 3.0 (5)
+    assert q.codes[0, 9] == 0x0D                         # -2.5g -> -3.0
+
+
+def test_block_scale_is_a_correctly_rounded_quotient():
+    """The block scale is E4M3_rne(fl32(bamax / fl32(6g))), a correctly rounded
+    division: on vector B the quotient is exactly the E4M3 midpoint 1.0625,
+    which ties to the even code 1.0 (0x38); a reciprocal-multiply form would
+    give 1.0625001 and the code 1.125 (0x39)."""
+    _, (b, gb) = reading_vectors.vectors()
+    f = np.float32
+    six_g = f(6) * gb
+    assert f(b[0, 16] / six_g) == f(1.0625)
+    assert f(b[0, 16] * (f(1) / six_g)) > f(1.0625)
+    q = oracle.quantize(b)
+    assert q.g == gb
+    assert q.scales[0, 1] == 0x38
 
 
 def test_code_magnitudes_bounded_by_six(random_case):

@@ -9,6 +9,7 @@ import pytest
 import torch
 
 import oracle
+import reading_vectors
 from gpu_helpers import (assert_quantized_equal, bf16_tensor, f32_tensor, tiled_scales)
 
 pytestmark = pytest.mark.gpu
@@ -142,6 +143,18 @@ def test_block_scale_ties_and_boundaries(nv):
             rows.append(row)
     x = np.stack(rows)
     assert_quantized_equal(quantize_gpu(nv, f32_tensor(x)), oracle.quantize(x))
+
+
+def test_quotient_reading_vectors(nv):
+    """The two rows of reading_vectors, where a different formation of the
+    block-scale or element quotient would change a scale byte or a code: the
+    GPU agrees with the oracle bit for bit (vector B also takes the encode
+    pass's exact-division fallback for the block scale)."""
+    for x, g in reading_vectors.vectors():
+        q = quantize_gpu(nv, f32_tensor(x))
+        qo = oracle.quantize(x)
+        assert qo.g == g
+        assert_quantized_equal(q, qo)
 
 
 @pytest.mark.parametrize("shape", [(0, 64), (5, 0), (0, 0)])
