@@ -243,7 +243,7 @@ def test_element_step_multiplies_by_the_rounded_reciprocal():
     reciprocal per block, then a multiply), not x / d: on vector A of
     reading_vectors the two readings round the same x to different E2M1
     codes."""
-    (a, ga), _ = reading_vectors.vectors()
+    (a, ga), *_ = reading_vectors.vectors()
     f = np.float32
     x, d = a[0, 17], ga                                  # block 1 scale is E4M3 1.0: d = g
     assert f(x / d) == f(2.5)                            # exact quotient: a tie -> even index (2.0)
@@ -259,7 +259,7 @@ def test_block_scale_is_a_correctly_rounded_quotient():
     division: on vector B the quotient is exactly the E4M3 midpoint 1.0625,
     which ties to the even code 1.0 (0x38); a reciprocal-multiply form would
     give 1.0625001 and the code 1.125 (0x39)."""
-    _, (b, gb) = reading_vectors.vectors()
+    _, (b, gb), *_ = reading_vectors.vectors()
     f = np.float32
     six_g = f(6) * gb
     assert f(b[0, 16] / six_g) == f(1.0625)
@@ -267,6 +267,38 @@ def test_block_scale_is_a_correctly_rounded_quotient():
     q = oracle.quantize(b)
     assert q.g == gb
     assert q.scales[0, 1] == 0x38
+
+
+def test_block_scale_divides_by_the_rounded_six_g():
+    """The divisor of the block-scale quotient is fl32(6g), rounded before the
+    division: on vector C, 6g is half an ulp below fl32(6g), and only the
+    rounded divisor puts the quotient exactly on the E4M3 midpoint 1.0625."""
+    _, _, (c, gc), _ = reading_vectors.vectors()
+    f = np.float32
+    six_g = f(6) * gc
+    assert Fraction(float(six_g)) - 6 * Fraction(float(gc)) > 0            # fl32(6g) was rounded up
+    assert f(c[0, 16] / six_g) == f(1.0625)
+    assert f(float(Fraction(float(c[0, 16])) / (6 * Fraction(float(gc))))) > f(1.0625)
+    q = oracle.quantize(c)
+    assert q.g == gc
+    assert q.scales[0, 1] == 0x38
+
+
+def test_element_reciprocal_is_of_the_rounded_d():
+    """d = fl32(dec(s) * g) is rounded before its reciprocal is taken: on
+    vector D, x * fl32(1/d) is exactly the E2M1 midpoint 2.5 (code 2.0), while
+    the reciprocal of the unrounded dec(s) * g would give 2.5000002 (3.0)."""
+    *_, (dv, gd) = reading_vectors.vectors()
+    f = np.float32
+    x = dv[0, 17]
+    d = f(f(1.125) * gd)
+    assert Fraction(float(d)) != Fraction(9, 8) * Fraction(float(gd))       # d was rounded
+    assert f(x * (f(1) / d)) == f(2.5)
+    assert f(x * f(float(1 / (Fraction(9, 8) * Fraction(float(gd)))))) > f(2.5)
+    q = oracle.quantize(dv)
+    assert q.g == gd and q.scales[0, 1] == 0x39                             # E4M3 1.125
+    assert q.codes[0, 8] == 0x47                                            # 6.0 (7), 2.0 (4)
+    assert q.codes[0, 9] == 0x0C                                            # -2.0
 
 
 def test_code_magnitudes_bounded_by_six(random_case):
