@@ -301,6 +301,22 @@ def test_element_reciprocal_is_of_the_rounded_d():
     assert q.codes[0, 9] == 0x0C                                            # -2.0
 
 
+def test_dequantize_rounds_the_scaled_code_before_g():
+    """Dequantize order: y = fl32(fl32(e * dec(s)) * g), the first product
+    exact.  With e = 3, dec(s) = 4.5 (0x49) and g = 0.5201722979545593 that is
+    fl32(13.5 g) = 7.022326; the other order, fl32(e * fl32(dec(s) * g)),
+    gives 7.0223255."""
+    f = np.float32
+    g = f(0.5201722979545593)
+    codes = np.zeros((1, 8), np.uint8)
+    codes[0, 0] = 0x05                                   # element 0: +3.0
+    q = oracle.Quantized(codes, np.array([[0x49]], np.uint8), g, 1, 16)
+    y = oracle.dequantize(q)
+    assert y[0, 0] == f(f(13.5) * g)
+    assert y[0, 0] != f(f(3) * f(f(4.5) * g))
+    assert (y[0, 1:] == 0).all()
+
+
 def test_code_magnitudes_bounded_by_six(random_case):
     q = oracle.quantize(random_case * 1e3)
     nibbles = np.concatenate([q.codes & 15, q.codes >> 4]).ravel()

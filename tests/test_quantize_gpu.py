@@ -194,3 +194,21 @@ def test_dequantize_parity(nv, shape):
     yb = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
     nv.nvfp4_dequantize(t, yb)
     assert torch.equal(yb.cpu(), torch.from_numpy(ref).to(torch.bfloat16))
+
+
+def test_dequantize_rounding_order(nv):
+    """y = fl32(fl32(e * dec(s)) * g): e = 3 with dec(s) = 4.5 and
+    g = 0.5201722979545593 is a value where the other order of the two
+    roundings gives a different fp32 result; every code with that scale and g."""
+    f = np.float32
+    codes = np.array([[(2 * j) | ((2 * j + 1) << 4) for j in range(8)]], np.uint8)   # codes 0..15
+    q = oracle.Quantized(codes, np.array([[0x49]], np.uint8), f(0.5201722979545593), 1, 16)
+    ref = oracle.dequantize(q)
+    assert ref[0, 5] == f(f(13.5) * q.g)
+    t = nv.NVFP4Tensor.empty(1, 16)
+    t.codes.copy_(torch.from_numpy(q.codes))
+    t.scales.copy_(torch.from_numpy(tiled_scales(q.scales)))
+    t.tensor_scale[0] = float(q.g)
+    y = torch.empty((1, 16), dtype=torch.float32, device="cuda")
+    nv.nvfp4_dequantize(t, y)
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
