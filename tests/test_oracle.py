@@ -382,16 +382,20 @@ def test_zero_tensor_and_zero_blocks():
 def test_tiny_magnitudes_follow_zero_block_rule():
     """amax so small that block scales round to zero or 1/d overflows: those
     blocks are zero-scale blocks with all codes 0; other blocks stay exact."""
-    x = np.zeros((2, 32), np.float32)
+    x = np.zeros((3, 32), np.float32)
     x[0, 0] = np.float32(2688 * 2.0 ** -120)          # g = 2^-120
     x[0, 16] = np.float32(2.0 ** -134)                # t = 2^-134/(6*2^-120) << 2^-10 -> s = 0
     x[1, 0] = np.float32(-3.0 * 2.0 ** -130)
-    q = oracle.quantize(x)
+    x[2, 5] = np.float32(-1e-38)                      # t ~ 0.0022 -> s = 2^-9 (0x01), d = 2^-129:
+    q = oracle.quantize(x)                            # a non-zero d with no finite fp32 reciprocal
     assert q.g == np.float32(2.0 ** -120)
     assert q.scales[0, 1] == 0 and q.codes[0, 8:16].tolist() == [0] * 8
+    with np.errstate(over="ignore"):
+        assert np.isinf(np.float32(1) / (np.float32(2.0 ** -9) * q.g))
+    assert q.scales[2, 0] == 0x01 and q.codes[2, 0:8].tolist() == [0] * 8
     y = oracle.dequantize(q)
     assert y[0, 0] == x[0, 0]
-    assert y[0, 16] == 0.0
+    assert y[0, 16] == 0.0 and y[2, 5] == 0.0
 
 
 def test_negative_values_rounding_to_zero_keep_sign():
