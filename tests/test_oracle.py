@@ -481,6 +481,7 @@ def test_gemm_transpose_convention(tiny_q):
     e, na, nb = oracle.gemm_entries(xq, wq, [0, 5, 15], [63, 0, 17])
     np.testing.assert_allclose(e, y[[0, 5, 15], [63, 0, 17]], rtol=1e-13, atol=0)
     np.testing.assert_allclose(na, np.linalg.norm(dx[[0, 5, 15]], axis=1), rtol=1e-12)
+    np.testing.assert_allclose(nb, np.linalg.norm(dw[[63, 0, 17]], axis=1), rtol=1e-12)
 
 
 def test_gemm_closed_form_constant_operands():
