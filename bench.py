@@ -602,6 +602,34 @@ def reference_arm(args):
     return 0
 
 
+def workload_result(wl, value, sps, dist, kern_us, e2e_value, steps, peaks):
+    """One workload's measured entry: metric value, step time and spread, the
+    dominant kernel's roofline, the end-to-end figure and the launch count."""
+    return {"metric": wl.metric, "value": round(value, 2), "unit": wl.unit,
+            "ms_per_step": round(sps * 1e3, 4), "step_us": dist, "config": wl.config,
+            "roofline": roofline(wl, kern_us, peaks),
+            "e2e": {"value": round(e2e_value, 3), "unit": wl.unit,
+                    "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h},
+            "gpu_launches": wl.launches * steps}
+
+
+def result_line(head, results, world, steps, warmup, peaks):
+    """The one JSON line: the headline workload's measurement (`head`, one
+    entry of the per-workload results) with the run's parameters; the other
+    workloads under "workloads"."""
+    return {"metric": head["metric"], "value": head["value"], "unit": head["unit"],
+            "n_gpus": world, "steps": steps, "warmup": warmup,
+            "ms_per_step": head["ms_per_step"], "step_us": head["step_us"],
+            "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4",
+            "data": "synthetic (seeded numpy PCG64: N(0,1) activations with 0.1% x50 outliers, "
+                    "N(0,0.02) weights, bf16)",
+            "config": dict(head["config"], parallelism=f"independent batch per GPU x{world}"),
+            "roofline": head["roofline"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+            "clocks": head["clocks"], "workloads": results,
+            "peaks": peaks}
+
+
 def _build_library():
     """Compile libnvfp4.so in-tree if it is missing or stale (nvcc)."""
     import importlib.util
@@ -650,12 +678,7 @@ def main():
         e2e_steps = min(args.steps, 20)
         e2e_elapsed = measure_e2e(wl, torch, e2e_steps, world)
         e2e_value = wl.value(e2e_elapsed / e2e_steps) * world
-        res = {"metric": wl.metric, "value": round(value, 2), "unit": wl.unit,
-               "ms_per_step": round(sps * 1e3, 4), "step_us": dist, "config": wl.config,
-               "roofline": roofline(wl, kern_us, peaks),
-               "e2e": {"value": round(e2e_value, 3), "unit": wl.unit,
-                       "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h},
-               "gpu_launches": wl.launches * args.steps}
+        res = workload_result(wl, value, sps, dist, kern_us, e2e_value, args.steps, peaks)
         if is_head:
             head = res
             head["clocks"] = clocks
@@ -664,17 +687,7 @@ def main():
         del wl
         torch.cuda.empty_cache()
 
-    line = {"metric": head["metric"], "value": head["value"], "unit": head["unit"],
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": head["ms_per_step"], "step_us": head["step_us"],
-            "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "nvfp4",
-            "data": "synthetic (seeded numpy PCG64: N(0,1) activations with 0.1% x50 outliers, "
-                    "N(0,0.02) weights, bf16)",
-            "config": dict(head["config"], parallelism=f"independent batch per GPU x{world}"),
-            "roofline": head["roofline"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
-            "clocks": head["clocks"], "workloads": results,
-            "peaks": peaks}
+    line = result_line(head, results, world, args.steps, args.warmup, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "prefill":
         line["cpu_baseline"] = cpu_oracle_prefill(args.cpu_rows)
     emit(line, rank)

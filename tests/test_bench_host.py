@@ -48,3 +48,39 @@ def test_roofline_tensor_and_hbm():
     assert r["unit"] == "GB/s" and r["peak"] == pytest.approx(6536.7)
     assert r["achieved"] == pytest.approx(50_436_608 / 12.7e-6 / 1e9, abs=0.1)
     assert "traffic" in r
+
+
+class _FakeWl:
+    name = "prefill"
+    metric = "NVFP4 GEMM TFLOPS (prefill)"
+    unit = "TFLOP/s"
+    config = {"workload": "prefill W4A4 linear", "M": 4096, "N": 17408, "K": 5120, "l2": "rotating copies"}
+    dominant = {"kernel": "k", "bound": "tensor", "algorithmic": 730_144_440_320, "unit": "TFLOP/s"}
+    h2d, d2h, launches = 41_943_040, 142_606_336, 3
+
+
+def test_result_line_has_every_contract_key():
+    """The JSON line the driver parses: every key of the measurement contract
+    with the right types, the roofline and e2e sub-objects, and a round trip
+    through json."""
+    import json
+    peaks = {"hbm_gbs": 6536.7, "bf16_tflops": 1656.9, "bf16_tflops_sustained": 1387.5, "source": "measured"}
+    dist = {"median": 180.0, "p10": 179.5, "p90": 181.0, "unit": "us", "rank": "local"}
+    head = bench.workload_result(_FakeWl(), 4067.5, 179.5e-6, dist, 164.9, 198.7, 100, peaks)
+    head["clocks"] = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": [], "samples": 7}
+    line = bench.result_line(head, {"decode": dict(head)}, 1, 100, 10, peaks)
+    line["cpu_baseline"] = {"value": 0.02, "unit": "TFLOP/s", "cores": 16, "kind": "oracle", "sample": "1024 rows"}
+    line = json.loads(json.dumps(line))
+    for k, t in [("metric", str), ("value", float), ("unit", str), ("n_gpus", int), ("steps", int),
+                 ("warmup", int), ("ms_per_step", float), ("higher_is_better", bool), ("scaling", str),
+                 ("dtype", str), ("data", str), ("config", dict), ("roofline", dict), ("e2e", dict),
+                 ("gpu_launches", int), ("clocks", dict), ("cpu_baseline", dict)]:
+        assert isinstance(line[k], t), k
+    assert line["vs_baseline"] is None and line["scaling"] == "weak" and line["higher_is_better"] is True
+    assert line["gpu_launches"] == 300 and line["ms_per_step"] == pytest.approx(0.1795)
+    assert "workload" in line["config"] and "model" not in line["config"]
+    assert set(line["roofline"]) >= {"bound", "achieved", "peak", "unit", "frac", "traffic"}
+    assert set(line["e2e"]) >= {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
+    assert set(line["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
+    assert set(line["cpu_baseline"]) >= {"value", "unit", "cores", "kind", "sample"}
+    assert line["roofline"]["frac"] == pytest.approx(line["roofline"]["achieved"] / line["roofline"]["peak"], abs=1e-3)
