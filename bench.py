@@ -602,6 +602,25 @@ def reference_arm(args):
     return 0
 
 
+def device_info(torch, index):
+    """Name, compute capability, CUDA runtime and driver of the measured GPU
+    (for the record; any field that cannot be read is None)."""
+    info = {"name": None, "cc": None, "cuda_runtime": getattr(torch.version, "cuda", None), "driver": None}
+    try:
+        info["name"] = torch.cuda.get_device_name(index)
+        info["cc"] = "%d.%d" % torch.cuda.get_device_capability(index)
+    except Exception:
+        pass
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        d = pynvml.nvmlSystemGetDriverVersion()
+        info["driver"] = d.decode() if isinstance(d, bytes) else d
+    except Exception:
+        pass
+    return info
+
+
 def workload_result(wl, value, sps, dist, kern_us, e2e_value, steps, peaks):
     """One workload's measured entry: metric value, step time and spread, the
     dominant kernel's roofline, the end-to-end figure and the launch count."""
@@ -688,6 +707,7 @@ def main():
         torch.cuda.empty_cache()
 
     line = result_line(head, results, world, args.steps, args.warmup, peaks)
+    line["device"] = device_info(torch, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "prefill":
         line["cpu_baseline"] = cpu_oracle_prefill(args.cpu_rows)
     emit(line, rank)

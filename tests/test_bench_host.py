@@ -84,3 +84,11 @@ def test_result_line_has_every_contract_key():
     assert set(line["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
     assert set(line["cpu_baseline"]) >= {"value", "unit", "cores", "kind", "sample"}
     assert line["roofline"]["frac"] == pytest.approx(line["roofline"]["achieved"] / line["roofline"]["peak"], abs=1e-3)
+
+
+def test_device_info_never_raises():
+    """The device record in the line: every field present, None where it
+    cannot be read (as on a machine without a GPU)."""
+    import torch
+    info = bench.device_info(torch, 0)
+    assert set(info) == {"name", "cc", "cuda_runtime", "driver"}
