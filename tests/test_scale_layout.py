@@ -64,3 +64,13 @@ def test_padded_size_matches_library():
     for R, KB in [(1, 1), (8, 320), (130, 5), (8192, 320)]:
         R128, KB4 = _pad(R, KB)
         assert nv.scales_bytes(R, KB * 16) == R128 * KB4
+
+
+@pytest.mark.parametrize("R,KB", [(16, 16), (64, 16), (130, 5), (257, 8)])
+def test_smoke_untiling_inverts_the_test_layout(R, KB):
+    """smoke() reads the GPU's scale bytes back with its own loop; it must be
+    the inverse of the tests' tiling."""
+    import __graft_entry__
+    rng = np.random.default_rng(R + KB)
+    s = rng.integers(0, 256, size=(R, KB), dtype=np.uint8)
+    assert np.array_equal(__graft_entry__._untile_scales(tiled_scales(s), R, KB * 16), s)
