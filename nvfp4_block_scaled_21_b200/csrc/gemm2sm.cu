@@ -461,10 +461,9 @@ static cudaError_t run_pair(const Operand &act, const Operand &wgt, int64_t K, v
 }
 
 // How many 2-CTA clusters of the pair kernel can be resident at once (0 if
-// the kernel cannot be configured).
-static int pair_max_clusters() {
-    static int cached = -1;
-    if (cached >= 0) return cached;
+// the kernel cannot be configured).  Computed once (a function-local static's
+// initialiser runs exactly once, also under concurrent first calls).
+static int pair_max_clusters_query() {
     int n = 0;
     bool ok = true;
     auto kb = gemm_nvf4_pair_kernel<__nv_bfloat16>;
@@ -486,8 +485,12 @@ static int pair_max_clusters() {
         if (cudaOccupancyMaxActiveClusters(&n, kb, &cfg) != cudaSuccess) n = 0;
     }
     cudaGetLastError();
-    cached = n;
-    return cached;
+    return n;
+}
+
+static int pair_max_clusters() {
+    static const int n = pair_max_clusters_query();
+    return n;
 }
 
 bool pair_gemm_usable(int64_t M, int64_t N, int num_sms) {
