@@ -4,6 +4,7 @@
 // nvfp4_get_device_status.
 #include <atomic>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -38,8 +39,13 @@ nvfp4_status current_device(DevInfo *out) {
             cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         if (dev < 64) {
-            cache[dev] = d;
-            have[dev].store(true, std::memory_order_release);
+            // one writer per entry: a thread that lost the race leaves it alone
+            static std::mutex fill;
+            std::lock_guard<std::mutex> lock(fill);
+            if (!have[dev].load(std::memory_order_relaxed)) {
+                cache[dev] = d;
+                have[dev].store(true, std::memory_order_release);
+            }
         }
         *out = d;
     }
