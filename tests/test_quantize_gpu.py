@@ -146,10 +146,10 @@ def test_block_scale_ties_and_boundaries(nv):
 
 
 def test_quotient_reading_vectors(nv):
-    """The two rows of reading_vectors, where a different formation of the
+    """The four rows of reading_vectors, where a different formation of the
     block-scale or element quotient would change a scale byte or a code: the
-    GPU agrees with the oracle bit for bit (vector B also takes the encode
-    pass's exact-division fallback for the block scale)."""
+    GPU agrees with the oracle bit for bit (vectors B and C also take the
+    encode pass's exact-division fallback for the block scale)."""
     for x, g in reading_vectors.vectors():
         q = quantize_gpu(nv, f32_tensor(x))
         qo = oracle.quantize(x)
