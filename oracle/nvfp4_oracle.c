@@ -407,3 +407,112 @@ void oracle_bf16_to_f32(const uint16_t *x, int64_t n, float *out)
         memcpy(&out[i], &bits, sizeof bits);
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4 ([MX]: eefocus.com article on FP4 vs INT4, section                  */
+/* "FP4被视为下一代AI计算的核心标准": the OCP Microscaling format shares one */
+/* 8-bit scale, usually E8M0, among 32 consecutive elements, each an E2M1    */
+/* value; about 4.25 bits per value).  The page gives no rule for choosing   */
+/* the scale.  Readings taken:                                               */
+/*   M1  X = 2^e with e = ceil(log2(bamax / 6)): the smallest power of two   */
+/*       that brings every element of the block into the E2M1 range, so no   */
+/*       element saturates; e clamped to [-127, 127]; an all-zero block gets */
+/*       the smallest scale, byte 0.                                         */
+/*   M2  element code = E2M1 RNE(x / X) with R3's grid, tie and sign rules;  */
+/*       x / X is exact (a power-of-two scaling).                            */
+/*   M3  no second-level (tensor) scale.                                     */
+/*   M4  packing as R5; the oracle keeps scales row-major [rows][cols/32].   */
+/* ------------------------------------------------------------------------ */
+
+/* E8M0: eight exponent bits, bias 127, no sign and no mantissa; 0xFF is NaN. */
+double oracle_e8m0_value(unsigned byte)
+{
+    if ((byte & 0xFFu) == 0xFFu)
+        return NAN;
+    return ldexp(1.0, (int)(byte & 0xFFu) - 127);
+}
+
+/* M1.  bamax / 6 = f * 2^p with f in [0.5, 1) (frexp).  The quotient is a
+ * power of two exactly when f == 0.5 (bamax = 6 * 2^k is exact in binary, and
+ * any other fp32 bamax is at least 2^-24 away from it in relative terms, far
+ * more than the fp64 rounding of the quotient), and then ceil(log2) = p - 1;
+ * otherwise it is p. */
+unsigned oracle_mx_block_scale(float bamax)
+{
+    int p, e;
+    double f;
+    if (!(bamax > 0.0f))
+        return 0u;
+    f = frexp((double)bamax / 6.0, &p);
+    e = (f == 0.5) ? p - 1 : p;
+    if (e < -127)
+        e = -127;
+    if (e > 127)
+        e = 127;
+    return (unsigned)(e + 127);
+}
+
+/* Quantize the logical [rows][cols] window (cols % 32 == 0) of a row-major
+ * fp32 matrix with leading dimension ld to MXFP4: packed codes
+ * [rows][cols/2] and E8M0 scale bytes [rows][cols/32].  Returns 0, or -1 on
+ * bad arguments or a non-finite input. */
+int oracle_mx_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld,
+                       uint8_t *codes, uint8_t *scales)
+{
+    int64_t nblk = cols / 32;
+    if (rows < 0 || cols < 0 || cols % 32 != 0 || ld < cols)
+        return -1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            if (!isfinite(x[r * ld + c]))
+                return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nblk; ++b) {
+            const float *blk = x + r * ld + b * 32;
+            float bamax = 0.0f;
+            unsigned s;
+            double scale;
+            for (int i = 0; i < 32; ++i) {
+                float a = fabsf(blk[i]);
+                if (a > bamax)
+                    bamax = a;
+            }
+            s = oracle_mx_block_scale(bamax);
+            scales[r * nblk + b] = (uint8_t)s;
+            scale = oracle_e8m0_value(s);
+            for (int i = 0; i < 32; i += 2) {
+                /* exact quotients; a result below the fp32 normal range
+                 * rounds to a signed value far below 0.25, code 0 either way */
+                unsigned lo = oracle_e2m1_encode((float)((double)blk[i] / scale));
+                unsigned hi = oracle_e2m1_encode((float)((double)blk[i + 1] / scale));
+                codes[r * (cols / 2) + b * 16 + i / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+/* fp64 dequantization of an MXFP4 [rows][cols]: e * 2^(s - 127), exact.  (An
+ * fp32 result would overflow for the largest codes at the top scales, so the
+ * oracle keeps fp64.) */
+int oracle_mx_dequantize_f64(const uint8_t *codes, const uint8_t *scales,
+                             int64_t rows, int64_t cols, double *y)
+{
+    if (rows < 0 || cols < 0 || cols % 32 != 0)
+        return -1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            unsigned byte = codes[r * (cols / 2) + c / 2];
+            unsigned code = (c & 1) ? (byte >> 4) : (byte & 15u);
+            y[r * cols + c] = oracle_e2m1_value(code) *
+                              oracle_e8m0_value(scales[r * (cols / 32) + c / 32]);
+        }
+    return 0;
+}
+
+/* Storage of one MXFP4 [rows][cols] tensor in bytes: packed codes and one
+ * scale byte per 32 values ([MX]: about 4.25 bits per value). */
+int64_t oracle_mx_storage_bytes(int64_t rows, int64_t cols)
+{
+    return rows * cols / 2 + rows * cols / 32;
+}

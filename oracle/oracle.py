@@ -20,6 +20,12 @@ Parity status of each function (what pins it is in ``tests/test_oracle.py``):
                                       tiny case, closed form for constant
                                       operands.
 * ``silu_mul_f64``                   pinned: closed-form identities of SiLU.
+* ``mx_*`` (MXFP4: 32-value blocks,  pinned: E8M0 decode of all 256 bytes
+  E8M0 scales, no tensor scale)      against torch.float8_e8m0fnu; the scale
+                                      rule by brute force over every byte;
+                                      exact round trip; nearest-code check;
+                                      block granularity; 4.25-bit storage;
+                                      closed-form GEMM.
 * tiled scale layout, nibble order   parity unpinned by the pages: fixed by the
                                       tensor-core operand format and checked only
                                       through GPU GEMM parity.
@@ -102,6 +108,16 @@ def _declare(L):
     L.oracle_e4m3_encode_array.argtypes = [_P, _I64, _P]
     L.oracle_e4m3_value_array.argtypes = [_P, _I64, _P]
     L.oracle_bf16_to_f32.argtypes = [_P, _I64, _P]
+    L.oracle_e8m0_value.argtypes = [ctypes.c_uint]
+    L.oracle_e8m0_value.restype = ctypes.c_double
+    L.oracle_mx_block_scale.argtypes = [ctypes.c_float]
+    L.oracle_mx_block_scale.restype = ctypes.c_uint
+    L.oracle_mx_quantize.argtypes = [_P, _I64, _I64, _I64, _P, _P]
+    L.oracle_mx_quantize.restype = ctypes.c_int
+    L.oracle_mx_dequantize_f64.argtypes = [_P, _P, _I64, _I64, _P]
+    L.oracle_mx_dequantize_f64.restype = ctypes.c_int
+    L.oracle_mx_storage_bytes.argtypes = [_I64, _I64]
+    L.oracle_mx_storage_bytes.restype = _I64
 
 
 def _ptr(a: np.ndarray):
@@ -275,3 +291,69 @@ def mlp_chain_f64(x_q: Quantized, wg: Quantized, wu: Quantized):
     gate = gemm_f64(x_q, wg)
     up = gemm_f64(x_q, wu)
     return silu_mul_f64(gate, up)
+
+
+# --------------------------------------------------------------------------
+# MXFP4 (32-value blocks, E8M0 scales, no tensor scale; readings M1-M4 in
+# nvfp4_oracle.c)
+# --------------------------------------------------------------------------
+
+class QuantizedMX:
+    """One MXFP4 tensor as the oracle emits it.
+
+    codes:  uint8 [rows][cols/2], element 2j in the low nibble of byte j
+    scales: uint8 [rows][cols/32], row-major E8M0 block scales
+    """
+
+    def __init__(self, codes, scales, rows, cols):
+        self.codes, self.scales, self.rows, self.cols = codes, scales, rows, cols
+
+
+def e8m0_value(byte: int) -> float:
+    return lib().oracle_e8m0_value(int(byte))
+
+
+def mx_block_scale(bamax: float) -> int:
+    return lib().oracle_mx_block_scale(float(bamax))
+
+
+def mx_quantize(x: np.ndarray) -> QuantizedMX:
+    """Quantize a 2-D fp32 array (or bf16 given as its uint16 bit patterns) to MXFP4."""
+    if x.dtype == np.uint16:
+        x = bf16_bits_to_f32(x)
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if x.ndim != 2:
+        raise ValueError("mx_quantize expects a 2-D array")
+    rows, cols = x.shape
+    if cols % 32:
+        raise ValueError("cols must be a multiple of 32")
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, cols // 32), np.uint8)
+    rc = lib().oracle_mx_quantize(_ptr(x), rows, cols, cols, _ptr(codes), _ptr(scales))
+    if rc != 0:
+        raise ValueError("oracle_mx_quantize rejected the input (non-finite?)")
+    return QuantizedMX(codes, scales, rows, cols)
+
+
+def mx_dequantize_f64(q: QuantizedMX) -> np.ndarray:
+    y = np.empty((q.rows, q.cols), np.float64)
+    rc = lib().oracle_mx_dequantize_f64(_ptr(q.codes), _ptr(q.scales), q.rows, q.cols, _ptr(y))
+    assert rc == 0
+    return y
+
+
+def mx_gemm_f64(a: QuantizedMX, b: QuantizedMX, nthreads: int | None = None) -> np.ndarray:
+    """Y = deq(A) . deq(B)^T in fp64, A [M][K], B [N][K], both MXFP4."""
+    if a.cols != b.cols:
+        raise ValueError("K mismatch")
+    da = mx_dequantize_f64(a)
+    db = mx_dequantize_f64(b)
+    y = np.empty((a.rows, b.rows), np.float64)
+    nt = nthreads or os.cpu_count() or 1
+    rc = lib().oracle_gemm_f64(_ptr(da), _ptr(db), a.rows, b.rows, a.cols, _ptr(y), int(nt))
+    assert rc == 0
+    return y
+
+
+def mx_storage_bytes(rows: int, cols: int) -> int:
+    return int(lib().oracle_mx_storage_bytes(rows, cols))

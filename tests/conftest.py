@@ -30,6 +30,14 @@ def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
 
 
+@pytest.fixture(scope="session")
+def facts(golden_dir):
+    """Format facts the pages state (tests/golden/format_facts.json, each with its citation)."""
+    import json
+    with open(os.path.join(golden_dir, "format_facts.json")) as f:
+        return json.load(f)
+
+
 def has_gpu() -> bool:
     try:
         import torch

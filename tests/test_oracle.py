@@ -22,10 +22,6 @@ from nvfp4_block_scaled_21_b200 import workloads
 pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
 
 
-@pytest.fixture(scope="module")
-def facts(golden_dir):
-    with open(os.path.join(golden_dir, "format_facts.json")) as f:
-        return json.load(f)
 
 
 # ---------------------------------------------------------------------------
