@@ -119,6 +119,75 @@ def test_linear_fused_rejects_bad_arguments_without_launch():
     assert f(nv.EPI_SILU_MUL_REQUANT, _t(rows=16, cols=128), _t(rows=8, cols=32), None) == nv.ERR_INVALID_ARG
 
 
+def test_dequantize_rejects_bad_arguments_without_launch():
+    lib = nv.lib()
+    q = _t(rows=4, cols=64)
+    d = lambda t, y, yt, ldy: lib.nvfp4_dequantize(ctypes.byref(t) if t else None, y, yt, ldy, None)
+    assert d(None, 16, nv.F32, 64) == nv.ERR_INVALID_ARG
+    assert d(q, 16, 7, 64) == nv.ERR_INVALID_ARG                                    # dtype
+    assert d(q, None, nv.F32, 64) == nv.ERR_INVALID_ARG                             # y missing
+    assert d(q, 16, nv.F32, 32) == nv.ERR_INVALID_ARG                               # ldy < cols
+    assert d(q, 24, nv.F32, 64) == nv.ERR_MISALIGNED                                # y
+    assert d(q, 16, nv.BF16, 66) == nv.ERR_MISALIGNED                               # row pitch
+    assert d(_t(rows=4, cols=24), 16, nv.F32, 24) == nv.ERR_UNSUPPORTED_SHAPE       # cols % 16
+    assert d(_t(codes=None, rows=4, cols=64), 16, nv.F32, 64) == nv.ERR_INVALID_ARG
+    assert d(_t(scales=24), 16, nv.F32, 64) == nv.ERR_MISALIGNED
+
+
+def test_linear_fused_rejects_more_bad_arguments_without_launch():
+    """Each call breaks exactly one rule of nvfp4_linear_fused and stops at it."""
+    lib = nv.lib()
+    w, wu = _t(rows=32, cols=128), _t(rows=32, cols=128)
+
+    def f(x=16, xt=nv.BF16, M=8, K=128, ldx=128, w_=w, wu_=None, epi=nv.EPI_STORE, y=16, yt=nv.BF16, ldy=32,
+          yq=None, xq=None, ws=4096, wb=1 << 30):
+        return lib.nvfp4_linear_fused(x, xt, M, K, ldx, ctypes.byref(w_), ctypes.byref(wu_) if wu_ else None, epi,
+                                      y, yt, ldy, ctypes.byref(yq) if yq else None,
+                                      ctypes.byref(xq) if xq else None, ws, wb, None)
+
+    assert f(x=None) == nv.ERR_INVALID_ARG                                          # x missing
+    assert f(xt=9) == nv.ERR_INVALID_ARG
+    assert f(M=-1) == nv.ERR_INVALID_ARG
+    assert f(ldx=64) == nv.ERR_INVALID_ARG                                          # ldx < K
+    assert f(w_=_t(rows=32, cols=64)) == nv.ERR_INVALID_ARG                         # w's K differs
+    assert f(K=96, ldx=96, w_=_t(rows=32, cols=96)) == nv.ERR_UNSUPPORTED_SHAPE     # K % 64
+    assert f(x=24) == nv.ERR_MISALIGNED
+    assert f(ldx=132) == nv.ERR_MISALIGNED                                          # 264-byte pitch
+    assert f(ldy=16) == nv.ERR_INVALID_ARG                                          # ldy < N
+    assert f(yt=5) == nv.ERR_INVALID_ARG
+    assert f(y=24) == nv.ERR_MISALIGNED
+    assert f(ldy=36) == nv.ERR_MISALIGNED                                           # 72-byte pitch
+    silu = dict(epi=nv.EPI_SILU_MUL_REQUANT, wu_=wu, yq=_t(rows=8, cols=32), yt=nv.F32)
+    assert f(**{**silu, "yt": nv.BF16}) == nv.ERR_INVALID_ARG                       # h must be fp32
+    assert f(**{**silu, "y": 24}) == nv.ERR_MISALIGNED
+    assert f(**{**silu, "wu_": _t(rows=16, cols=128)}) == nv.ERR_INVALID_ARG        # w_up rows differ
+    assert f(xq=_t(rows=8, cols=64)) == nv.ERR_INVALID_ARG                          # x_q shape
+    assert f(ws=None) == nv.ERR_WORKSPACE
+    assert f(wb=64) == nv.ERR_WORKSPACE
+    assert f(ws=4100) == nv.ERR_MISALIGNED
+
+
+def test_gemm_rejects_rows_beyond_its_index_range_and_bad_dtype():
+    lib = nv.lib()
+    a, b = _t(rows=8, cols=128), _t(rows=32, cols=128)
+    big = _t(rows=2 ** 31, cols=128)
+    assert lib.nvfp4_gemm(ctypes.byref(big), ctypes.byref(b), 16, nv.BF16, 32, 4096, 1 << 30, None) == \
+        nv.ERR_UNSUPPORTED_SHAPE
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), 16, 3, 32, 4096, 1 << 30, None) == nv.ERR_INVALID_ARG
+
+
+def test_selftest_and_timeout_setter_host_paths():
+    lib = nv.lib()
+    assert lib.nvfp4_selftest_bounded_wait(None, 1000, None) == nv.ERR_WORKSPACE
+    assert lib.nvfp4_selftest_bounded_wait(8, 1000, None) == nv.ERR_MISALIGNED
+    old = lib.nvfp4_set_wait_timeout_us(1234)
+    try:
+        assert lib.nvfp4_set_wait_timeout_us(0) == 1234                              # 0 is stored as 1
+        assert lib.nvfp4_set_wait_timeout_us(old) == 1
+    finally:
+        lib.nvfp4_set_wait_timeout_us(old)
+
+
 def test_empty_operands_skip_pointer_and_pitch_checks():
     """An empty matrix is never read or written: a NULL pointer and any pitch
     at least its row length pass validation.  Each call below then stops at
