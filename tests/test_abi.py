@@ -188,6 +188,30 @@ def test_selftest_and_timeout_setter_host_paths():
         lib.nvfp4_set_wait_timeout_us(old)
 
 
+def test_noalloc_rejects_bad_arguments_and_oversized_shapes_without_launch():
+    """nvfp4_linear_noalloc checks its arguments and the size of its static
+    scratch before its first device call (the scratch address lookup)."""
+    lib = nv.lib()
+    w = _t(rows=32, cols=128)
+
+    def f(x=16, xt=nv.BF16, M=8, K=128, ldx=128, w_=w, y=16, yt=nv.BF16, ldy=32):
+        return lib.nvfp4_linear_noalloc(x, xt, M, K, ldx, ctypes.byref(w_), y, yt, ldy, None)
+
+    assert f(x=None) == nv.ERR_INVALID_ARG
+    assert f(xt=4) == nv.ERR_INVALID_ARG
+    assert f(ldx=100) == nv.ERR_INVALID_ARG                                         # ldx < K
+    assert f(w_=_t(rows=32, cols=64)) == nv.ERR_INVALID_ARG                         # w's K differs
+    assert f(K=96, ldx=96, w_=_t(rows=32, cols=96)) == nv.ERR_UNSUPPORTED_SHAPE     # K % 64
+    assert f(y=None) == nv.ERR_INVALID_ARG
+    assert f(ldy=8) == nv.ERR_INVALID_ARG                                           # ldy < N
+    assert f(yt=2) == nv.ERR_INVALID_ARG
+    assert f(x=40) == nv.ERR_MISALIGNED
+    assert f(y=40) == nv.ERR_MISALIGNED
+    # quantized activations beyond the 4 MiB static scratch: 8192 x 5120 needs 21 MB
+    w5k = _t(rows=32, cols=5120)
+    assert f(M=8192, K=5120, ldx=5120, w_=w5k) == nv.ERR_UNSUPPORTED_SHAPE
+
+
 def test_empty_operands_skip_pointer_and_pitch_checks():
     """An empty matrix is never read or written: a NULL pointer and any pitch
     at least its row length pass validation.  Each call below then stops at
