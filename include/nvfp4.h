@@ -74,7 +74,9 @@ typedef struct CUstream_st *nvfp4_stream_t;
 typedef enum {
     NVFP4_OK = 0,
     NVFP4_ERR_INVALID_ARG = 1,           /* NULL pointer, negative size, mismatched shapes */
-    NVFP4_ERR_UNSUPPORTED_SHAPE = 2,     /* cols % 16 (quantize) or K % 64 (GEMM) not 0 */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 2,     /* cols % 16 (quantize) or K % 64 (GEMM) not 0; a GEMM
+                                            with M or N above 2^30 - 1 or K above 2^31 (the
+                                            kernels' 32-bit row and tile-coordinate range) */
     NVFP4_ERR_MISALIGNED = 3,            /* a pointer or row pitch not 16-byte aligned */
     NVFP4_ERR_WORKSPACE = 4,             /* ws NULL or smaller than required */
     NVFP4_ERR_CUDA = 5,                  /* a CUDA runtime/driver call or launch failed */

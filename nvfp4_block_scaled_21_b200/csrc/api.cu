@@ -168,7 +168,8 @@ static nvfp4_status check_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, voi
     if (st != NVFP4_OK) return st;
     if ((st = check_tensor(b, b->rows, b->cols)) != NVFP4_OK) return st;
     if (a->cols % 64) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (a->rows > INT32_MAX / 2 || b->rows > INT32_MAX / 2) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (a->rows > kMaxGemmRows || b->rows > kMaxGemmRows || a->cols > kMaxGemmK)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (ldy < b->rows) return NVFP4_ERR_INVALID_ARG;
     const int eb = yt == NVFP4_BF16 ? 2 : 4;
     if (a->rows * b->rows != 0 && (!aligned16(y) || (ldy * eb) % 16)) return NVFP4_ERR_MISALIGNED;
@@ -219,6 +220,7 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
     const int xeb = xt == NVFP4_BF16 ? 2 : 4;
     if (M * K != 0 && (!aligned16(x) || (ldx * xeb) % 16)) return NVFP4_ERR_MISALIGNED;
     const int64_t N = w->rows;
+    if (M > kMaxGemmRows || N > kMaxGemmRows || K > kMaxGemmK) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (epilogue == NVFP4_EPI_STORE) {
         if ((!y && M * N != 0) || (yt != NVFP4_F32 && yt != NVFP4_BF16) || ldy < N)
             return NVFP4_ERR_INVALID_ARG;

@@ -30,6 +30,11 @@ __host__ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t kb, 
     return tile * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3);
 }
 
+// Largest GEMM sizes the kernels index in 32 bits: rows of either operand (and
+// sums of two row indices), and K (the TMA x coordinate reaches K/2 bytes).
+constexpr int64_t kMaxGemmRows = 0x3fffffff;            // INT32_MAX / 2
+constexpr int64_t kMaxGemmK = int64_t(1) << 31;
+
 // Workspace layout: [0,16) status words, [256, ...) scratch.
 constexpr size_t kWsStatusBytes = 256;
 constexpr int kMaxAmaxPartials = 4096;

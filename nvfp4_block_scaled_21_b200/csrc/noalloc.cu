@@ -97,7 +97,7 @@ extern "C" nvfp4_status nvfp4_linear_noalloc(const void *x, nvfp4_dtype xt, int6
     // empty operands are never touched: their pointers and pitches are not checked
     if ((M * K != 0 && (!aligned16(x) || (ldx * xeb) % 16)) || (M * N != 0 && (!aligned16(y) || (ldy * yeb) % 16)))
         return NVFP4_ERR_MISALIGNED;
-    if (M > INT32_MAX / 2 || N > INT32_MAX / 2) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M > kMaxGemmRows || N > kMaxGemmRows || K > kMaxGemmK) return NVFP4_ERR_UNSUPPORTED_SHAPE;
 
     // Quantized activations must fit in the static scratch.
     const size_t codes_bytes = align256(static_cast<size_t>(M) * static_cast<size_t>(K / 2));

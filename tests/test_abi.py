@@ -167,13 +167,33 @@ def test_linear_fused_rejects_more_bad_arguments_without_launch():
     assert f(ws=4100) == nv.ERR_MISALIGNED
 
 
-def test_gemm_rejects_rows_beyond_its_index_range_and_bad_dtype():
+def test_gemm_rejects_sizes_beyond_its_index_range_and_bad_dtype():
+    """Rows above 2^30 - 1 or K above 2^31 leave the kernels' 32-bit row and
+    tile-coordinate range: refused, not wrapped."""
     lib = nv.lib()
     a, b = _t(rows=8, cols=128), _t(rows=32, cols=128)
-    big = _t(rows=2 ** 31, cols=128)
-    assert lib.nvfp4_gemm(ctypes.byref(big), ctypes.byref(b), 16, nv.BF16, 32, 4096, 1 << 30, None) == \
-        nv.ERR_UNSUPPORTED_SHAPE
+    for x, w in [(_t(rows=2 ** 30, cols=128), b), (a, _t(rows=2 ** 30, cols=128)),
+                 (_t(rows=8, cols=2 ** 31 + 64), _t(rows=32, cols=2 ** 31 + 64))]:
+        assert lib.nvfp4_gemm(ctypes.byref(x), ctypes.byref(w), 16, nv.BF16, 2 ** 30 + 64, 4096, 1 << 30,
+                              None) == nv.ERR_UNSUPPORTED_SHAPE
+    ok = _t(rows=2 ** 30 - 1, cols=128)                     # the largest row count passes this check
+    assert lib.nvfp4_gemm(ctypes.byref(ok), ctypes.byref(b), 16, nv.BF16, 32, 4096, 8, None) == nv.ERR_WORKSPACE
     assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), 16, 3, 32, 4096, 1 << 30, None) == nv.ERR_INVALID_ARG
+
+
+def test_linear_layers_reject_sizes_beyond_the_gemm_index_range():
+    lib = nv.lib()
+    w, K = _t(rows=32, cols=128), 128
+    big_k = 2 ** 31 + 64
+    wk = _t(rows=32, cols=big_k)
+    fused = lambda x_rows, kk, ww: lib.nvfp4_linear_fused(16, nv.BF16, x_rows, kk, kk, ctypes.byref(ww), None,
+                                                          nv.EPI_STORE, 16, nv.BF16, ww.rows, None, None, 4096,
+                                                          1 << 62, None)
+    assert fused(2 ** 30, K, w) == nv.ERR_UNSUPPORTED_SHAPE                         # M
+    assert fused(8, K, _t(rows=2 ** 30, cols=128)) == nv.ERR_UNSUPPORTED_SHAPE     # N
+    assert fused(8, big_k, wk) == nv.ERR_UNSUPPORTED_SHAPE                          # K
+    assert lib.nvfp4_linear_noalloc(16, nv.BF16, 8, big_k, big_k, ctypes.byref(wk), 16, nv.BF16, 32,
+                                    None) == nv.ERR_UNSUPPORTED_SHAPE
 
 
 def test_selftest_and_timeout_setter_host_paths():
