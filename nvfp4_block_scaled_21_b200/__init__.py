@@ -151,6 +151,23 @@ class NVFP4Tensor:
                        self.tensor_scale.data_ptr(), self.rows, self.cols)
 
 
+def _on_device(*objs) -> None:
+    """Every buffer the library dereferences must live on the current CUDA
+    device: a host tensor's pointer, or another GPU's, would be read by the
+    kernels.  Raises before anything reaches the library."""
+    cur = None
+    for o in objs:
+        if o is None:
+            continue
+        for t in ((o.codes, o.scales, o.tensor_scale) if isinstance(o, NVFP4Tensor) else (o,)):
+            if not t.is_cuda:
+                raise TypeError(f"nvfp4: got a tensor on {t.device}; the library needs CUDA tensors")
+            if cur is None:
+                cur = _torch().cuda.current_device()
+            if t.device.index != cur:
+                raise ValueError(f"nvfp4: tensor on {t.device} but the current device is cuda:{cur}")
+
+
 def codes_bytes(rows: int, cols: int) -> int:
     return int(_lib.nvfp4_codes_bytes(rows, cols))
 
@@ -172,6 +189,7 @@ def workspace(op: int, M: int, N: int, K: int, device="cuda"):
 def nvfp4_quantize(x, out: NVFP4Tensor, ws, stream=None) -> NVFP4Tensor:
     """Quantize a 2-D bf16/fp32 CUDA tensor (row pitch x.stride(0)) into out."""
     assert x.dim() == 2 and x.stride(1) == 1
+    _on_device(x, out, ws)
     ct = out.c()
     st = _lib.nvfp4_quantize(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], x.stride(0),
                              ctypes.byref(ct), ws.data_ptr(), ws.numel(), _stream(stream))
@@ -181,6 +199,7 @@ def nvfp4_quantize(x, out: NVFP4Tensor, ws, stream=None) -> NVFP4Tensor:
 
 def nvfp4_dequantize(q: NVFP4Tensor, y, stream=None):
     assert y.dim() == 2 and y.stride(1) == 1
+    _on_device(q, y)
     ct = q.c()
     st = _lib.nvfp4_dequantize(ctypes.byref(ct), y.data_ptr(), _dtype_code(y), y.stride(0),
                                _stream(stream))
@@ -191,6 +210,7 @@ def nvfp4_dequantize(q: NVFP4Tensor, y, stream=None):
 def nvfp4_gemm(a: NVFP4Tensor, b: NVFP4Tensor, y, ws, stream=None):
     """y[M][N] = (a . b^T) * ga * gb."""
     assert y.dim() == 2 and y.stride(1) == 1
+    _on_device(a, b, y, ws)
     ca, cb = a.c(), b.c()
     st = _lib.nvfp4_gemm(ctypes.byref(ca), ctypes.byref(cb), y.data_ptr(), _dtype_code(y),
                          y.stride(0), ws.data_ptr(), ws.numel(), _stream(stream))
@@ -203,6 +223,7 @@ def nvfp4_linear_fused(x, w: NVFP4Tensor, ws, epilogue: int = EPI_STORE, y=None,
                        x_q: NVFP4Tensor | None = None, stream=None):
     """Quantize x on the device and run the W4A4 linear layer (see nvfp4.h)."""
     assert x.dim() == 2 and x.stride(1) == 1
+    _on_device(x, w, ws, y, w_up, y_q, x_q)
     cw = w.c()
     cwu = w_up.c() if w_up is not None else None
     cyq = y_q.c() if y_q is not None else None
@@ -225,6 +246,7 @@ def nvfp4_linear_noalloc(x, w: NVFP4Tensor, y, stream=None):
     allocate device memory.  See nvfp4_linear_noalloc in nvfp4.h for the size
     limit and the rule that calls must not overlap on the GPU."""
     assert x.dim() == 2 and x.stride(1) == 1 and y.dim() == 2 and y.stride(1) == 1
+    _on_device(x, w, y)
     cw = w.c()
     st = _lib.nvfp4_linear_noalloc(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1],
                                    x.stride(0), ctypes.byref(cw), y.data_ptr(), _dtype_code(y),
@@ -234,10 +256,12 @@ def nvfp4_linear_noalloc(x, w: NVFP4Tensor, y, stream=None):
 
 
 def nvfp4_get_device_status(ws, stream=None) -> int:
+    _on_device(ws)
     return int(_lib.nvfp4_get_device_status(ws.data_ptr(), _stream(stream)))
 
 
 def nvfp4_selftest_bounded_wait(ws, timeout_us: int, stream=None) -> None:
+    _on_device(ws)
     _check(_lib.nvfp4_selftest_bounded_wait(ws.data_ptr(), int(timeout_us), _stream(stream)),
            "nvfp4_selftest_bounded_wait")
 

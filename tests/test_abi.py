@@ -252,6 +252,30 @@ def test_empty_operands_skip_pointer_and_pitch_checks():
                               None) == nv.ERR_MISALIGNED
 
 
+def test_binding_refuses_host_tensors_before_the_library():
+    """A host tensor's pointer would be dereferenced by the kernels: every
+    wrapper raises before it calls into the library."""
+    import torch
+    x = torch.zeros((4, 64), dtype=torch.float32)
+    q = nv.NVFP4Tensor(torch.zeros((4, 32), dtype=torch.uint8), torch.zeros(512, dtype=torch.uint8),
+                       torch.zeros(4), 4, 64)
+    ws = torch.zeros(1 << 16, dtype=torch.uint8)
+    y = torch.zeros((4, 4), dtype=torch.float32)
+    calls = [
+        lambda: nv.nvfp4_quantize(x, q, ws),
+        lambda: nv.quantize(x),
+        lambda: nv.nvfp4_dequantize(q, torch.zeros((4, 64))),
+        lambda: nv.nvfp4_gemm(q, q, y, ws),
+        lambda: nv.nvfp4_linear_fused(x, q, ws, nv.EPI_STORE, y=y),
+        lambda: nv.nvfp4_linear_noalloc(x, q, y),
+        lambda: nv.nvfp4_get_device_status(ws),
+        lambda: nv.nvfp4_selftest_bounded_wait(ws, 1000),
+    ]
+    for call in calls:
+        with pytest.raises(TypeError, match="CUDA tensors"):
+            call()
+
+
 def test_package_fails_loudly_without_library(tmp_path):
     """The binding refuses to import when libnvfp4.so is absent: no CPU fallback."""
     import subprocess
