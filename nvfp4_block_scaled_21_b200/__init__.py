@@ -151,6 +151,16 @@ class NVFP4Tensor:
                        self.tensor_scale.data_ptr(), self.rows, self.cols)
 
 
+def _rows(*ts) -> None:
+    """2-D tensors whose rows are contiguous (any row pitch): the layout the C
+    ABI describes with a pointer and a row pitch.  A plain check, not an assert,
+    so that it also holds under python -O."""
+    for t in ts:
+        if t is not None and (t.dim() != 2 or t.stride(1) != 1):
+            raise ValueError(f"nvfp4: expected a 2-D tensor with contiguous rows, got shape "
+                             f"{tuple(t.shape)} strides {tuple(t.stride())}")
+
+
 def _on_device(*objs) -> None:
     """Every buffer the library dereferences must live on the current CUDA
     device: a host tensor's pointer, or another GPU's, would be read by the
@@ -188,7 +198,7 @@ def workspace(op: int, M: int, N: int, K: int, device="cuda"):
 
 def nvfp4_quantize(x, out: NVFP4Tensor, ws, stream=None) -> NVFP4Tensor:
     """Quantize a 2-D bf16/fp32 CUDA tensor (row pitch x.stride(0)) into out."""
-    assert x.dim() == 2 and x.stride(1) == 1
+    _rows(x)
     _on_device(x, out, ws)
     ct = out.c()
     st = _lib.nvfp4_quantize(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], x.stride(0),
@@ -198,7 +208,7 @@ def nvfp4_quantize(x, out: NVFP4Tensor, ws, stream=None) -> NVFP4Tensor:
 
 
 def nvfp4_dequantize(q: NVFP4Tensor, y, stream=None):
-    assert y.dim() == 2 and y.stride(1) == 1
+    _rows(y)
     _on_device(q, y)
     ct = q.c()
     st = _lib.nvfp4_dequantize(ctypes.byref(ct), y.data_ptr(), _dtype_code(y), y.stride(0),
@@ -209,7 +219,7 @@ def nvfp4_dequantize(q: NVFP4Tensor, y, stream=None):
 
 def nvfp4_gemm(a: NVFP4Tensor, b: NVFP4Tensor, y, ws, stream=None):
     """y[M][N] = (a . b^T) * ga * gb."""
-    assert y.dim() == 2 and y.stride(1) == 1
+    _rows(y)
     _on_device(a, b, y, ws)
     ca, cb = a.c(), b.c()
     st = _lib.nvfp4_gemm(ctypes.byref(ca), ctypes.byref(cb), y.data_ptr(), _dtype_code(y),
@@ -222,7 +232,7 @@ def nvfp4_linear_fused(x, w: NVFP4Tensor, ws, epilogue: int = EPI_STORE, y=None,
                        w_up: NVFP4Tensor | None = None, y_q: NVFP4Tensor | None = None,
                        x_q: NVFP4Tensor | None = None, stream=None):
     """Quantize x on the device and run the W4A4 linear layer (see nvfp4.h)."""
-    assert x.dim() == 2 and x.stride(1) == 1
+    _rows(x, y)
     _on_device(x, w, ws, y, w_up, y_q, x_q)
     cw = w.c()
     cwu = w_up.c() if w_up is not None else None
@@ -245,7 +255,7 @@ def nvfp4_linear_noalloc(x, w: NVFP4Tensor, y, stream=None):
     static scratch instead of a caller workspace; for callers that cannot
     allocate device memory.  See nvfp4_linear_noalloc in nvfp4.h for the size
     limit and the rule that calls must not overlap on the GPU."""
-    assert x.dim() == 2 and x.stride(1) == 1 and y.dim() == 2 and y.stride(1) == 1
+    _rows(x, y)
     _on_device(x, w, y)
     cw = w.c()
     st = _lib.nvfp4_linear_noalloc(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1],

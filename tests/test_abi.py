@@ -276,6 +276,23 @@ def test_binding_refuses_host_tensors_before_the_library():
             call()
 
 
+def test_binding_refuses_matrices_without_contiguous_rows():
+    """The C ABI describes a matrix by pointer and row pitch: a view whose
+    elements within a row are not adjacent is refused (a plain check, so it
+    also holds under python -O)."""
+    import torch
+    x = torch.zeros((8, 128))
+    q = nv.NVFP4Tensor(torch.zeros((8, 32), dtype=torch.uint8), torch.zeros(512, dtype=torch.uint8),
+                       torch.zeros(4), 8, 64)
+    ws = torch.zeros(1 << 16, dtype=torch.uint8)
+    for call in (lambda: nv.nvfp4_quantize(x[:, ::2], q, ws), lambda: nv.nvfp4_quantize(x.t(), q, ws),
+                 lambda: nv.nvfp4_linear_fused(x[:, ::2], q, ws, nv.EPI_STORE, y=x[:, :8]),
+                 lambda: nv.nvfp4_linear_fused(x[:, :64], q, ws, nv.EPI_STORE, y=x[:, ::16]),
+                 lambda: nv.nvfp4_gemm(q, q, x[:, ::16], ws)):
+        with pytest.raises(ValueError, match="contiguous rows"):
+            call()
+
+
 def test_package_fails_loudly_without_library(tmp_path):
     """The binding refuses to import when libnvfp4.so is absent: no CPU fallback."""
     import subprocess
