@@ -161,6 +161,37 @@ def _rows(*ts) -> None:
                              f"{tuple(t.shape)} strides {tuple(t.stride())}")
 
 
+def _buffers(*qs) -> None:
+    """The C ABI passes an NVFP4 tensor's buffers as bare pointers, so the
+    library cannot see their sizes: each must be contiguous and hold at least
+    what nvfp4_codes_bytes / nvfp4_scales_bytes give for its shape (and one
+    fp32 tensor scale), or the kernels would read or write past it."""
+    for q in qs:
+        if q is None:
+            continue
+        if q.tensor_scale.dtype != _torch().float32:
+            raise TypeError(f"nvfp4: tensor_scale must be float32, got {q.tensor_scale.dtype}")
+        for t, need, what in ((q.codes, codes_bytes(q.rows, q.cols), "codes"),
+                              (q.scales, scales_bytes(q.rows, q.cols), "scales"),
+                              (q.tensor_scale, 4, "tensor_scale")):
+            have = t.numel() * t.element_size()
+            if not t.is_contiguous() or have < need:
+                raise ValueError(f"nvfp4: {what} of a {q.rows}x{q.cols} NVFP4 tensor needs {need} contiguous "
+                                 f"bytes; got {have} bytes{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+def _shape(y, rows: int, cols: int) -> None:
+    """The library writes rows x cols elements at y's row pitch: y must have that shape."""
+    if y is not None and tuple(y.shape) != (rows, cols):
+        raise ValueError(f"nvfp4: output of shape {tuple(y.shape)}, expected ({rows}, {cols})")
+
+
+def _ws_bytes(ws) -> int:
+    if not ws.is_contiguous():
+        raise ValueError("nvfp4: the workspace must be contiguous")
+    return ws.numel() * ws.element_size()
+
+
 def _on_device(*objs) -> None:
     """Every buffer the library dereferences must live on the current CUDA
     device: a host tensor's pointer, or another GPU's, would be read by the
@@ -199,16 +230,19 @@ def workspace(op: int, M: int, N: int, K: int, device="cuda"):
 def nvfp4_quantize(x, out: NVFP4Tensor, ws, stream=None) -> NVFP4Tensor:
     """Quantize a 2-D bf16/fp32 CUDA tensor (row pitch x.stride(0)) into out."""
     _rows(x)
+    _buffers(out)
     _on_device(x, out, ws)
     ct = out.c()
     st = _lib.nvfp4_quantize(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], x.stride(0),
-                             ctypes.byref(ct), ws.data_ptr(), ws.numel(), _stream(stream))
+                             ctypes.byref(ct), ws.data_ptr(), _ws_bytes(ws), _stream(stream))
     _check(st, "nvfp4_quantize")
     return out
 
 
 def nvfp4_dequantize(q: NVFP4Tensor, y, stream=None):
     _rows(y)
+    _buffers(q)
+    _shape(y, q.rows, q.cols)
     _on_device(q, y)
     ct = q.c()
     st = _lib.nvfp4_dequantize(ctypes.byref(ct), y.data_ptr(), _dtype_code(y), y.stride(0),
@@ -220,10 +254,12 @@ def nvfp4_dequantize(q: NVFP4Tensor, y, stream=None):
 def nvfp4_gemm(a: NVFP4Tensor, b: NVFP4Tensor, y, ws, stream=None):
     """y[M][N] = (a . b^T) * ga * gb."""
     _rows(y)
+    _buffers(a, b)
+    _shape(y, a.rows, b.rows)
     _on_device(a, b, y, ws)
     ca, cb = a.c(), b.c()
     st = _lib.nvfp4_gemm(ctypes.byref(ca), ctypes.byref(cb), y.data_ptr(), _dtype_code(y),
-                         y.stride(0), ws.data_ptr(), ws.numel(), _stream(stream))
+                         y.stride(0), ws.data_ptr(), _ws_bytes(ws), _stream(stream))
     _check(st, "nvfp4_gemm")
     return y
 
@@ -233,6 +269,8 @@ def nvfp4_linear_fused(x, w: NVFP4Tensor, ws, epilogue: int = EPI_STORE, y=None,
                        x_q: NVFP4Tensor | None = None, stream=None):
     """Quantize x on the device and run the W4A4 linear layer (see nvfp4.h)."""
     _rows(x, y)
+    _buffers(w, w_up, y_q, x_q)
+    _shape(y, x.shape[0], w.rows)
     _on_device(x, w, ws, y, w_up, y_q, x_q)
     cw = w.c()
     cwu = w_up.c() if w_up is not None else None
@@ -244,7 +282,7 @@ def nvfp4_linear_fused(x, w: NVFP4Tensor, ws, epilogue: int = EPI_STORE, y=None,
         x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], x.stride(0), ctypes.byref(cw),
         ctypes.byref(cwu) if cwu is not None else None, epilogue, _ptr(y), yt, ldy,
         ctypes.byref(cyq) if cyq is not None else None,
-        ctypes.byref(cxq) if cxq is not None else None, ws.data_ptr(), ws.numel(),
+        ctypes.byref(cxq) if cxq is not None else None, ws.data_ptr(), _ws_bytes(ws),
         _stream(stream))
     _check(st, "nvfp4_linear_fused")
     return y
@@ -256,6 +294,8 @@ def nvfp4_linear_noalloc(x, w: NVFP4Tensor, y, stream=None):
     allocate device memory.  See nvfp4_linear_noalloc in nvfp4.h for the size
     limit and the rule that calls must not overlap on the GPU."""
     _rows(x, y)
+    _buffers(w)
+    _shape(y, x.shape[0], w.rows)
     _on_device(x, w, y)
     cw = w.c()
     st = _lib.nvfp4_linear_noalloc(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1],

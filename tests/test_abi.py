@@ -293,6 +293,41 @@ def test_binding_refuses_matrices_without_contiguous_rows():
             call()
 
 
+def test_binding_refuses_short_buffers_and_wrong_output_shapes():
+    """The C ABI cannot see buffer sizes or an output's row count: the binding
+    refuses an NVFP4 tensor whose buffers are too small or not contiguous, and
+    an output whose shape is not the one the call writes."""
+    import torch
+
+    def q(rows=8, cols=64, codes=None, scales=None, g=None):
+        return nv.NVFP4Tensor(codes if codes is not None else torch.zeros((rows, cols // 2), dtype=torch.uint8),
+                              scales if scales is not None else torch.zeros(nv.scales_bytes(rows, cols),
+                                                                            dtype=torch.uint8),
+                              g if g is not None else torch.zeros(4), rows, cols)
+
+    x, ws = torch.zeros((8, 64)), torch.zeros(1 << 16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="scales"):
+        nv.nvfp4_quantize(x, q(scales=torch.zeros(100, dtype=torch.uint8)), ws)
+    with pytest.raises(ValueError, match="codes"):
+        nv.nvfp4_quantize(x, q(codes=torch.zeros((8, 31), dtype=torch.uint8)), ws)
+    with pytest.raises(ValueError, match="not contiguous"):
+        nv.nvfp4_quantize(x, q(codes=torch.zeros((32, 8), dtype=torch.uint8).t()), ws)
+    with pytest.raises(TypeError, match="float32"):
+        nv.nvfp4_quantize(x, q(g=torch.zeros(4, dtype=torch.float64)), ws)
+    a, b = q(8, 64), q(16, 64)
+    with pytest.raises(ValueError, match="expected \\(8, 16\\)"):
+        nv.nvfp4_gemm(a, b, torch.zeros((7, 16)), ws)
+    with pytest.raises(ValueError, match="expected \\(8, 64\\)"):
+        nv.nvfp4_dequantize(a, torch.zeros((8, 32)))
+    with pytest.raises(ValueError, match="expected \\(8, 16\\)"):
+        nv.nvfp4_linear_fused(x, b, ws, nv.EPI_STORE, y=torch.zeros((8, 15)))
+    with pytest.raises(ValueError, match="expected \\(8, 16\\)"):
+        nv.nvfp4_linear_noalloc(x, b, torch.zeros((9, 16)))
+    with pytest.raises(ValueError, match="scales"):
+        nv.nvfp4_linear_fused(x, b, ws, nv.EPI_SILU_MUL_REQUANT, w_up=b,
+                              y_q=q(8, 16, scales=torch.zeros(8, dtype=torch.uint8)))
+
+
 def test_package_fails_loudly_without_library(tmp_path):
     """The binding refuses to import when libnvfp4.so is absent: no CPU fallback."""
     import subprocess
