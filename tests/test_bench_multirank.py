@@ -68,5 +68,5 @@ def test_reference_arm_under_torchrun_two_ranks():
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
-    assert line["cpu_baseline"]["cores"] == min(os.cpu_count(), 2)         # 2 rows: 2 GEMM threads at most
+    assert line["cpu_baseline"]["cores"] == min(os.cpu_count(), 8)         # 8 rows: 8 GEMM threads at most
     assert line["e2e"]["h2d_bytes_per_step"] == 0
