@@ -328,6 +328,51 @@ def test_binding_refuses_short_buffers_and_wrong_output_shapes():
                               y_q=q(8, 16, scales=torch.zeros(8, dtype=torch.uint8)))
 
 
+_C_CALLER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "nvfp4.h"
+
+int main(void) {
+    nvfp4_tensor t;
+    memset(&t, 0, sizeof t);
+    if (nvfp4_scales_bytes(8, 5120) != (size_t)128 * 320) return 1;
+    if (nvfp4_codes_bytes(8192, 5120) != (size_t)8192 * 2560) return 2;
+    if (nvfp4_version() <= 0) return 3;
+    if (strcmp(nvfp4_status_string(NVFP4_ERR_INVALID_ARG), "invalid argument") != 0) return 4;
+    /* argument errors return before any device call */
+    if (nvfp4_quantize(NULL, NVFP4_BF16, 4, 64, 64, &t, NULL, 0, NULL) != NVFP4_ERR_INVALID_ARG) return 5;
+    if (nvfp4_gemm(NULL, NULL, NULL, NVFP4_BF16, 0, NULL, 0, NULL) != NVFP4_ERR_INVALID_ARG) return 6;
+    puts("ok");
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_a_c_program_links_and_calls_the_library(tmp_path):
+    """The boundary is a C ABI: a C99 program built with warnings as errors
+    includes the header, links libnvfp4.so and makes host-only calls (sizes,
+    version, status strings, argument errors); the header also parses as C++."""
+    import shutil
+    import subprocess
+    if not shutil.which("gcc"):
+        pytest.skip("gcc not available")
+    src = tmp_path / "caller.c"
+    src.write_text(_C_CALLER)
+    exe = tmp_path / "caller"
+    pkg = os.path.join(ROOT, "nvfp4_block_scaled_21_b200")
+    inc = os.path.join(ROOT, "include")
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", inc, str(src),
+                        "-L", pkg, "-lnvfp4", f"-Wl,-rpath,{pkg}", "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", (run.returncode, run.stdout, run.stderr)
+    if shutil.which("g++"):
+        cxx = subprocess.run(["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-x", "c++",
+                              "-I", inc, str(src)], capture_output=True, text=True)
+        assert cxx.returncode == 0, cxx.stderr
+
+
 def test_package_fails_loudly_without_library(tmp_path):
     """The binding refuses to import when libnvfp4.so is absent: no CPU fallback."""
     import subprocess
