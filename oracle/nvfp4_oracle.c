@@ -21,6 +21,10 @@
  *           "核心差异：W4A4 vs W4A16": weights and activations are both 4-bit
  *           and the FP4 tensor cores consume them directly, with no
  *           dequantize-to-16-bit step.
+ *   [MX]    eefocus.com article, section "FP4被视为下一代AI计算的核心标准":
+ *           the OCP MXFP4 format, 32 E2M1 elements sharing one 8-bit (usually
+ *           E8M0) scale, about 4.25 bits per value (the MXFP4 section below,
+ *           readings M1-M4).
  *
  * The pages fix the structure but not the scale arithmetic.  The readings
  * taken here (each is also a rule the CUDA path follows):
