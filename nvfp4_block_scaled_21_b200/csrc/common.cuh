@@ -35,6 +35,32 @@ __host__ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t kb, 
 constexpr int64_t kMaxGemmRows = 0x3fffffff;            // INT32_MAX / 2
 constexpr int64_t kMaxGemmK = int64_t(1) << 31;
 
+// An fp32 result in the output type: bf16 by round-to-nearest-even.
+template <typename OutT> __device__ __forceinline__ OutT to_out(float v);
+template <> __device__ __forceinline__ float to_out<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// Running max |y| over the output values one thread stores, exact: bf16
+// words as two 15-bit magnitudes (non-negative floats order like their bit
+// patterns), fp32 values by fmaxf.  value() gives it as an fp32 number, in the
+// format of the quantizer's first pass (per-CTA partial maxima), so that a
+// GEMM whose output is re-quantized needs only the encode pass afterwards.
+struct YMax {
+    uint32_t b = 0u;
+    float f = 0.0f;
+    __device__ __forceinline__ void bf16x2(uint32_t w) { b = __vmaxu2(b, w & 0x7fff7fffu); }
+    __device__ __forceinline__ void bf16(__nv_bfloat16 v) {
+        b = __vmaxu2(b, static_cast<uint32_t>(__bfloat16_as_ushort(v)) & 0x7fffu);
+    }
+    __device__ __forceinline__ void f32(float v) { f = fmaxf(f, fabsf(v)); }
+    template <typename OutT> __device__ __forceinline__ void add(OutT v);
+    __device__ __forceinline__ float value() const {
+        return fmaxf(f, __uint_as_float(max(b & 0xffffu, b >> 16) << 16));
+    }
+};
+template <> __device__ __forceinline__ void YMax::add<float>(float v) { f32(v); }
+template <> __device__ __forceinline__ void YMax::add<__nv_bfloat16>(__nv_bfloat16 v) { bf16(v); }
+
 // Workspace layout: [0,16) status words, [256, ...) scratch.
 constexpr size_t kWsStatusBytes = 256;
 constexpr int kMaxAmaxPartials = 4096;

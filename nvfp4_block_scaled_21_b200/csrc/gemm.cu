@@ -51,7 +51,7 @@ namespace nvfp4 {
 struct GemmArgs {
     const uint8_t *sfa;      // tiled scales of the MMA A operand (P rows)
     const uint8_t *sfb;      // tiled scales of the MMA B operand (Q rows)
-    const float *ga;
+    const float *ga;         // tensor scales (null for MXFP4 operands, which have none)
     const float *gb;
     void *y;
     int64_t ldy;
@@ -65,6 +65,7 @@ struct GemmArgs {
     int32_t q_pad;           // row pitch (floats) of acc_ws: num_q_tiles * BN
     float *acc_ws;           // stream-K: fp32 partial sums [num_p_tiles*128][q_pad], zeroed per call
     int32_t *tile_cnt;       // stream-K: K slabs added per tile so far, zeroed per call
+    float *ymax_part;        // if set: this CTA's largest |y| as stored, at [blockIdx.x]
     uint32_t *status;
     uint64_t timeout_ns;
 };
@@ -124,7 +125,7 @@ struct GemmCfg {
     static constexpr int kColsUsed = kSfBase + kStages * kSfCols;
     static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
-    static constexpr int kBarBytes = 8 * (3 * kStages + 6) + 16;
+    static constexpr int kBarBytes = 8 * (3 * kStages + 7) + 16;
     static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;   // + alignment slack
     static constexpr int kThreads = 448;                       // 14 warps
     static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -132,11 +133,35 @@ struct GemmCfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
 };
 
-template <int BN, bool SWAP, typename OutT>
+// Scale atoms per 256-deep K stage and per 128-row tile: NVFP4 has one
+// 512-byte atom (4 blocks of 16) per K step of 64; MXFP4 one per two K steps
+// (4 blocks of 32), so a stage holds 4 or 2 atoms.
+template <bool MX> struct ScaleFmt {
+    static constexpr int kAtomsPerStage = MX ? 2 : 4;
+    __host__ __device__ static int atoms_per_row_tile(int k_steps) { return MX ? (k_steps + 1) / 2 : k_steps; }
+    __host__ __device__ static int stage_atoms(int nk) { return MX ? (nk + 1) / 2 : nk; }
+};
+
+// The block-scaled MMAs of K step j of a stage: NVFP4 reads the stage's
+// scale columns 4j (A) and 4*NQT*j past the A columns (B); MXFP4 reads the
+// columns of atom j/2 and picks their bytes {0,1} or {2,3} by the descriptor.
+template <bool MX, int BN, int NQT>
+__device__ __forceinline__ void mma_kstep(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t sf, int j,
+                                          uint32_t acc) {
+    if constexpr (MX) {
+        const uint32_t idesc = (j & 1) ? make_idesc_mxf4(BN, 128, 1) : make_idesc_mxf4(BN, 128, 0);
+        mma_mxf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * (j >> 1), sf + 16 + 4 * NQT * (j >> 1), acc);
+    } else {
+        mma_nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, make_idesc_nvf4(BN), sf + 4 * j, sf + 16 + 4 * NQT * j, acc);
+    }
+}
+
+template <int BN, bool SWAP, typename OutT, bool MX>
 __global__ void __launch_bounds__(448, 1)
 gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ GemmArgs args) {
     using C = GemmCfg<BN>;
+    using F = ScaleFmt<MX>;
     constexpr int STAGES = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -151,9 +176,11 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     uint64_t *tempty = tfull + 2;
     uint64_t *epi_done = tempty + 2;                    // stream-K: epilogue warps' partial sums added
     uint64_t *epi_flag = epi_done + 1;                  // stream-K: last_flag published
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(epi_flag + 1);
+    uint64_t *mma_done = epi_flag + 1;                  // every MMA of this CTA has completed
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile uint32_t *abort_flag = tmem_holder + 1;
     volatile uint32_t *last_flag = tmem_holder + 2;     // stream-K: this CTA completes the tile
+    __shared__ float s_ymax[8];                         // epilogue warps' largest |stored y|
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -172,6 +199,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         mbar_init(epi_done, 8);
         mbar_init(epi_flag, 1);
+        mbar_init(mma_done, 1);
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -196,11 +224,12 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const int pre = has_first ? min(args.preload, min(STAGES, first.ks1 - first.ks0)) : 0;
             const int pt0 = first.tile % args.num_p_tiles;
             const int qt0 = first.tile / args.num_p_tiles;
+            const int atoms_rt = F::atoms_per_row_tile(args.num_k_steps);
             auto load_a = [&](uint32_t st, int pt, int ks, int nk) {
                 tma_load_2d(sA + st * C::kAStage, &tmA, &full[st], ks * 128, pt * 128, pol_a);
                 bulk_load(sSfa + st * C::kSfaStage,
-                          args.sfa + (static_cast<int64_t>(pt) * args.num_k_steps + 4 * ks) * 512,
-                          nk * 512, &full[st], pol_a);
+                          args.sfa + (static_cast<int64_t>(pt) * atoms_rt + F::kAtomsPerStage * ks) * 512,
+                          F::stage_atoms(nk) * 512, &full[st], pol_a);
             };
             auto load_b = [&](uint32_t st, int qt, int ks, int nk) {
                 tma_load_2d(sB + st * C::kBStage, &tmB, &full[st], ks * 128, qt * BN, pol_b);
@@ -208,8 +237,8 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     const int rt = qt * C::kNQT + q;
                     if (rt < args.q_row_tiles)
                         bulk_load(sSfb + st * C::kSfbStage + q * 2048,
-                                  args.sfb + (static_cast<int64_t>(rt) * args.num_k_steps + 4 * ks) * 512,
-                                  nk * 512, &full[st], pol_b);
+                                  args.sfb + (static_cast<int64_t>(rt) * atoms_rt + F::kAtomsPerStage * ks) * 512,
+                                  F::stage_atoms(nk) * 512, &full[st], pol_b);
                 }
             };
             bool waited = (pre == 0);
@@ -238,7 +267,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 for (int q = 0; q < C::kNQT; ++q) nq_loaded += (qt * C::kNQT + q < args.q_row_tiles);
                 for (int ks = sg.ks0; ks < sg.ks1; ++ks, ++it) {
                     const int nk = min(4, args.num_k_steps - 4 * ks);
-                    const uint32_t bytes = C::kAStage + C::kBStage + nk * 512 * (1 + nq_loaded);
+                    const uint32_t bytes = C::kAStage + C::kBStage + F::stage_atoms(nk) * 512 * (1 + nq_loaded);
                     if (it < pre) {
                         // fresh stage (first pass over the ring): no empty wait needed
                         mbar_arrive_expect_tx(&full[stage], bytes);
@@ -258,11 +287,17 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 }
             }
             if (!waited) finish_preload();   // everything fit in the preload
+            // No copy may still be landing when the CTA exits: wait (bounded,
+            // also after an abort) for the last load issued into every stage.
+            // On the normal path the MMA thread has consumed them all already.
+            volatile uint32_t keep_waiting = 0u;
+            for (int j = it > STAGES ? it - STAGES : 0; j < it; ++j)
+                mbar_wait(&full[j % STAGES], static_cast<uint32_t>(j / STAGES) & 1u, args.timeout_ns,
+                          &keep_waiting, args.status);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // -------------------------------------------------------- MMA issuer
-            constexpr uint32_t idesc = make_idesc_nvf4(BN);
             const uint32_t a_base = smem_addr(sA), b_base = smem_addr(sB);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             SegIter segs(args, num_tiles, num_kstages);
@@ -288,12 +323,10 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     if (nk == 4) {
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
-                            mma_nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j,
-                                     sf + 16 + 4 * C::kNQT * j, (acc0 | j) != 0 ? 1u : 0u);
+                            mma_kstep<MX, BN, C::kNQT>(d_tmem, adesc, bdesc, sf, j, (acc0 | j) != 0 ? 1u : 0u);
                     } else {
                         for (int j = 0; j < nk; ++j)
-                            mma_nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j,
-                                     sf + 16 + 4 * C::kNQT * j, (acc0 | j) != 0 ? 1u : 0u);
+                            mma_kstep<MX, BN, C::kNQT>(d_tmem, adesc, bdesc, sf, j, (acc0 | j) != 0 ? 1u : 0u);
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -307,6 +340,11 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     acc_phase ^= 1u;
                 }
             }
+            // Tensor memory is freed below: first let every MMA this thread
+            // issued complete (bounded, also after an abort).
+            tc_commit(mma_done);
+            volatile uint32_t keep_waiting = 0u;
+            mbar_wait(mma_done, 0, args.timeout_ns, &keep_waiting, args.status);
         }
     } else if (warp < 6) {
         // ------------------------------------------------------------ scale warps
@@ -338,7 +376,8 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const uint8_t *b_src = sSfb + stage * C::kSfbStage + lane * 16;
                 // one 16-column store for A's scales and one 16*kNQT-column
                 // store for B's per stage (columns of K-steps a partial last
-                // stage does not have are never read)
+                // stage does not have, and for MXFP4 the two atom slots a stage
+                // does not use, hold stale bytes that are never read)
                 uint32_t av[16], bv[16 * C::kNQT];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -373,10 +412,14 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int quarter = warp & 3;               // TMEM lane quarter this warp may read
         const int half = (warp - 6) >> 2;           // column half of the tile (fast drain)
         const int row = quarter * 32 + lane;        // accumulator row (MMA M index)
-        const float alpha = __fmul_rn(*args.ga, *args.gb);
+        const float alpha = __fmul_rn(args.ga ? *args.ga : 1.0f, args.gb ? *args.gb : 1.0f);   // MXFP4: none
         constexpr bool kFastDrain = !SWAP && sizeof(OutT) == 2 && BN >= 64;
         uint32_t acc = 0, acc_phase = 0;
         uint32_t npart = 0;      // partial (stream-K) work items so far: epi_done/epi_flag phase
+        // Largest |y| this thread stores.  Accumulator rows and columns past P
+        // and Q are exact zeros (their operand rows are zero-filled by the
+        // loads), so folding a whole computed chunk cannot raise it.
+        YMax ym;
         SegIter segs(args, num_tiles, num_kstages);
         Seg sg;
         while (segs.next(sg)) {
@@ -475,16 +518,20 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                                         __nv_bfloat162 hi = __floats2bfloat162_rn(v2, v3);
                                         *reinterpret_cast<uint2 *>(dst) =
                                             make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+                                        ym.bf16x2(*reinterpret_cast<uint32_t *>(&lo));
+                                        ym.bf16x2(*reinterpret_cast<uint32_t *>(&hi));
                                     } else {
                                         *reinterpret_cast<float4 *>(dst) = make_float4(v0, v1, v2, v3);
+                                        ym.f32(v0); ym.f32(v1); ym.f32(v2); ym.f32(v3);
                                     }
                                 } else {
                                     const float vv[4] = {v0, v1, v2, v3};
 #pragma unroll
                                     for (int k = 0; k < 4; ++k)
                                         if (q + k < args.Q) {
-                                            if constexpr (sizeof(OutT) == 2) dst[k] = __float2bfloat16_rn(vv[k]);
-                                            else dst[k] = vv[k];
+                                            const OutT o = to_out<OutT>(vv[k]);
+                                            dst[k] = o;
+                                            ym.add<OutT>(o);
                                         }
                                 }
                             }
@@ -508,10 +555,9 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                                 const int pr = pt * 128 + rr;
                                 const float o = __fmul_rn(v[j][i], alpha);
                                 if (pr < args.P && q < args.Q) {
-                                    if constexpr (sizeof(OutT) == 2)
-                                        y[static_cast<int64_t>(q) * args.ldy + pr] = __float2bfloat16_rn(o);
-                                    else
-                                        y[static_cast<int64_t>(q) * args.ldy + pr] = o;
+                                    const OutT oo = to_out<OutT>(o);
+                                    y[static_cast<int64_t>(q) * args.ldy + pr] = oo;
+                                    ym.add<OutT>(oo);
                                 }
                             }
                         }
@@ -536,6 +582,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[c & 1][2 * k]), alpha),
                                                                   __fmul_rn(__uint_as_float(r[c & 1][2 * k + 1]), alpha));
                         pk[k] = *reinterpret_cast<uint32_t *>(&b2);
+                        ym.bf16x2(pk[k]);
                     }
                     const int q0 = qt * BN + half * HC + c * 32;
                     if (p < args.P) {
@@ -578,6 +625,8 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         float v[CH];
 #pragma unroll
                         for (int i = 0; i < CH; ++i) v[i] = __fmul_rn(__uint_as_float(r[c & 1][i]), alpha);
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) ym.add<OutT>(to_out<OutT>(v[i]));
                         const int q0 = qt * BN + c * CH;
                         if constexpr (SWAP) {
                             // y[q][p]: for each i the warp writes 32 consecutive p
@@ -644,10 +693,20 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 acc_phase ^= 1u;
             }
         }
+        float m = ym.value();
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) s_ymax[warp - 6] = m;
     }
 
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0 && args.ymax_part != nullptr) {
+        float m = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m = fmaxf(m, s_ymax[k]);
+        args.ymax_part[blockIdx.x] = m;
+    }
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (warp == 1) {
         tc_fence_after();
@@ -692,14 +751,15 @@ CUresult encode_tensor_map_u8(CUtensorMap *map, const void *base, uint64_t inner
 }
 
 CUresult encode_scale_map(CUtensorMap *map, const void *scales, uint64_t k_steps, uint64_t row_tiles,
-                          uint32_t box_tiles) {
+                          uint32_t box_tiles, uint32_t box_atoms) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return CUDA_ERROR_NOT_FOUND;
-    // x: 128 words of one 512-byte atom; y: K-step (atom) within a 128-row
-    // tile; z: 128-row tile.  A box holds 4 K-steps of box_tiles row tiles.
+    // x: 128 words of one 512-byte atom; y: atom along K within a 128-row
+    // tile (k_steps of them); z: 128-row tile.  A box holds box_atoms atoms
+    // of box_tiles row tiles.
     cuuint64_t dims[3] = {128, k_steps, row_tiles};
     cuuint64_t strides[2] = {512, k_steps * 512};
-    cuuint32_t box[3] = {128, 4, box_tiles};
+    cuuint32_t box[3] = {128, box_atoms, box_tiles};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void *>(scales), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -746,10 +806,11 @@ static SplitKLayout splitk_layout(int64_t M, int64_t N) {
 
 size_t splitk_ws_bytes(int64_t M, int64_t N) { return splitk_layout(M, N).bytes; }
 
-template <int BN, bool SWAP, typename OutT>
+template <int BN, bool SWAP, typename OutT, bool MX>
 static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, void *y, int64_t ldy,
                             uint32_t *status, uint64_t timeout_ns, int num_sms, int preload,
-                            uint8_t *splitk_ws, const SplitKLayout &skl, cudaStream_t stream) {
+                            uint8_t *splitk_ws, const SplitKLayout &skl, float *ymax_part, int *nparts,
+                            cudaStream_t stream) {
     using C = GemmCfg<BN>;
     CUtensorMap tmA, tmB;
     if (encode_tensor_map_u8(&tmA, pa.codes, K / 2, pa.rows, 128, 128) != CUDA_SUCCESS ||
@@ -772,6 +833,7 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     a.weights_are_a = SWAP ? 1 : 0;
     a.status = status;
     a.timeout_ns = timeout_ns;
+    a.ymax_part = ymax_part;
     const int tiles = a.num_p_tiles * a.num_q_tiles;
     const int64_t units = static_cast<int64_t>(tiles) * ((a.num_k_steps + 3) / 4);
     // Stream-K when the tiles alone would leave at least half of the SMs idle
@@ -788,7 +850,7 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     a.q_pad = a.num_q_tiles * BN;
     a.acc_ws = sk ? reinterpret_cast<float *>(splitk_ws) : nullptr;
     a.tile_cnt = sk ? reinterpret_cast<int32_t *>(splitk_ws + skl.acc_bytes) : nullptr;
-    auto kern = gemm_nvf4_kernel<BN, SWAP, OutT>;
+    auto kern = gemm_nvf4_kernel<BN, SWAP, OutT, MX>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // The stream-K scratch is zero-filled for every call, so it may share a
@@ -797,6 +859,7 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     cudaLaunchConfig_t cfg = {};
     const int64_t work = sk ? units : tiles;
     cfg.gridDim = dim3(static_cast<unsigned>(work < num_sms ? work : num_sms));
+    if (nparts) *nparts = static_cast<int>(cfg.gridDim.x);
     cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
@@ -808,9 +871,11 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
 }
 
-cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
-                        int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
-                        cudaStream_t stream, bool weights_ready, void *splitk_ws) {
+template <bool MX>
+static cudaError_t launch_gemm_fmt(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
+                                   int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
+                                   cudaStream_t stream, bool weights_ready, void *splitk_ws, float *ymax_part,
+                                   int *nparts) {
     // weights_ready: the weights were not written by the kernel launched just
     // before this one, so they may be streamed before the dependent-launch wait.
     const int preload = weights_ready ? 8 : 0;
@@ -821,22 +886,37 @@ cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void 
         // weights on the MMA's M side, activations on N; y[m][n] = acc[n][m]
         const int bn = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
 #define NVFP4_SWAPPED(BNV)                                                                          \
-    return y_bf16 ? run_gemm<BNV, true, __nv_bfloat16>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, stream) \
-                  : run_gemm<BNV, true, float>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, stream);
+    return y_bf16 ? run_gemm<BNV, true, __nv_bfloat16, MX>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream) \
+                  : run_gemm<BNV, true, float, MX>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream);
         if (bn == 16) { NVFP4_SWAPPED(16) }
         if (bn == 32) { NVFP4_SWAPPED(32) }
         NVFP4_SWAPPED(64)
 #undef NVFP4_SWAPPED
     }
     if (pair_gemm_usable(M, N, num_sms))
-        return launch_gemm_pair(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, stream);
+        return launch_gemm_pair(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, stream, ymax_part, nparts, MX);
     const int64_t ptiles = ceil_div(M, 128);
     const bool wide = ptiles * ceil_div(N, 256) >= 2 * num_sms;
     if (wide)
-        return y_bf16 ? run_gemm<256, false, __nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, stream)
-                      : run_gemm<256, false, float>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, stream);
-    return y_bf16 ? run_gemm<128, false, __nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, stream)
-                  : run_gemm<128, false, float>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, stream);
+        return y_bf16 ? run_gemm<256, false, __nv_bfloat16, MX>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream)
+                      : run_gemm<256, false, float, MX>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream);
+    return y_bf16 ? run_gemm<128, false, __nv_bfloat16, MX>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream)
+                  : run_gemm<128, false, float, MX>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream);
+}
+
+cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
+                        int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
+                        cudaStream_t stream, bool weights_ready, void *splitk_ws, float *ymax_part,
+                        int *nparts) {
+    return launch_gemm_fmt<false>(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, num_sms, stream, weights_ready,
+                                  splitk_ws, ymax_part, nparts);
+}
+
+cudaError_t launch_gemm_mx(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
+                           int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
+                           cudaStream_t stream, void *splitk_ws) {
+    return launch_gemm_fmt<true>(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, num_sms, stream, false,
+                                 splitk_ws, nullptr, nullptr);
 }
 
 // ---------------------------------------------------------------------------

@@ -52,6 +52,7 @@ struct PairArgs {
     int32_t num_k_steps;     // K / 64
     int32_t num_pm, num_qn;  // 256-row / 256-column pair tiles
     int32_t tma_store;       // bf16 output written by TMA stores (needs N % 8 == 0)
+    float *ymax_part;        // if set: this CTA's largest |y| as stored, at [blockIdx.x]
     uint32_t *status;
     uint64_t timeout_ns;
 };
@@ -72,15 +73,16 @@ struct PairCfg {
     static constexpr int kTmemWarps = 8;
     static constexpr int kThreads = 32 * (2 + kTmemWarps);
     static constexpr int kStagingBytes = kTmemWarps * 32 * 128;   // per warp: 32 rows x 64 bf16
-    static constexpr int kBarBytes = 8 * (3 * kStages + 4 + 2) + 16;
+    static constexpr int kBarBytes = 8 * (3 * kStages + 4 + 3) + 16;
     static constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + kBarBytes + 1024;
     static_assert(kSfCol + 2 * kSlotCols <= kTmemCols, "tensor memory budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
+// (columns past N are exact zeros: folding them into ym cannot raise it)
 template <typename OutT>
 __device__ __forceinline__ void pair_store_chunk(const uint32_t (&r)[32], float alpha, OutT *yrow,
-                                                 int q0, int N) {
+                                                 int q0, int N, YMax &ym) {
     if constexpr (sizeof(OutT) == 2) {
         uint32_t pk[16];
 #pragma unroll
@@ -88,6 +90,7 @@ __device__ __forceinline__ void pair_store_chunk(const uint32_t (&r)[32], float 
             __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * k]), alpha),
                                                       __fmul_rn(__uint_as_float(r[2 * k + 1]), alpha));
             pk[k] = *reinterpret_cast<uint32_t *>(&b2);
+            ym.bf16x2(pk[k]);
         }
         if (q0 + 32 <= N) {
 #pragma unroll
@@ -105,12 +108,15 @@ __device__ __forceinline__ void pair_store_chunk(const uint32_t (&r)[32], float 
         }
     } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            if (q0 + i < N) yrow[q0 + i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+        for (int i = 0; i < 32; ++i) {
+            const float v = __fmul_rn(__uint_as_float(r[i]), alpha);
+            if (q0 + i < N) yrow[q0 + i] = v;
+            ym.f32(v);
+        }
     }
 }
 
-template <typename OutT>
+template <typename OutT, bool MX>
 __global__ void __launch_bounds__(PairCfg::kThreads, 1)
 gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
@@ -131,8 +137,10 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     uint64_t *sf_free = sf_ready + 2;                                                // each CTA's [2]
     uint64_t *tfull = sf_free + 2;                                                   // each CTA's
     uint64_t *tempty = tfull + 1;                                                    // leader's
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tempty + 1);
+    uint64_t *mma_done = tempty + 1;                                                 // leader's
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile uint32_t *abort_flag = tmem_holder + 1;
+    __shared__ float s_ymax[C::kTmemWarps];               // TMEM warps' largest |stored y|
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -156,6 +164,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         }
         mbar_init(tfull, 1);
         mbar_init(tempty, 2 * C::kTmemWarps);
+        mbar_init(mma_done, 1);
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -178,6 +187,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             const uint64_t pol = policy_evict_normal();
             const uint32_t leader_full0 = mapa_shared(smem_addr(&full[0]), 0);
             uint32_t stage = 0, phase = 0;
+            int issued = 0;
             for (int tile = cid; tile < num_tiles; tile += ncl) {
                 const int pm = tile % args.num_pm;
                 const int qn = tile / args.num_pm;
@@ -193,18 +203,31 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                     if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kABBytes);
                     tma_load_2d_pair(sA + stage * C::kAStage, &tmA, bar, ks * 128, a_rt * 128, pol);
                     tma_load_2d_pair(sB + stage * C::kBStage, &tmB, bar, ks * 128, b_rt * 128, pol);
-                    mbar_arrive_expect_tx(&sfull[stage], C::kSfBytes);
-                    tma_load_3d(sSfa + stage * C::kSfaStage, &tmSA, &sfull[stage], 0, 4 * ks, a_rt, pol);
-                    tma_load_3d(sSfb + stage * C::kSfbStage, &tmSB, &sfull[stage], 0, 4 * ks, 2 * qn, pol);
+                    // scale atoms of this stage: 4 (NVFP4) or 2 (MXFP4) per 128-row tile
+                    mbar_arrive_expect_tx(&sfull[stage], MX ? C::kSfBytes / 2 : C::kSfBytes);
+                    tma_load_3d(sSfa + stage * C::kSfaStage, &tmSA, &sfull[stage], 0, (MX ? 2 : 4) * ks, a_rt, pol);
+                    tma_load_3d(sSfb + stage * C::kSfbStage, &tmSB, &sfull[stage], 0, (MX ? 2 : 4) * ks, 2 * qn, pol);
+                    ++issued;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
+            }
+            // No copy may still be landing when the pair exits: wait (bounded,
+            // also after an abort) for the last loads issued into every stage:
+            // this CTA's scale loads on its own barrier, and in the leader the
+            // operand loads of both CTAs, which complete on the leader's.
+            volatile uint32_t keep_waiting = 0u;
+            for (int j = issued > STAGES ? issued - STAGES : 0; j < issued; ++j) {
+                const uint32_t par = static_cast<uint32_t>(j / STAGES) & 1u;
+                mbar_wait(&sfull[j % STAGES], par, args.timeout_ns, &keep_waiting, args.status);
+                if (leader) mbar_wait(&full[j % STAGES], par, args.timeout_ns, &keep_waiting, args.status);
             }
         }
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // -------------------------------------------------------- MMA issuer
             constexpr uint32_t idesc = make_idesc_nvf4_pair(256);
+            constexpr uint32_t idesc_mx0 = make_idesc_mxf4(256, 256, 0), idesc_mx1 = make_idesc_mxf4(256, 256, 1);
             const uint32_t a_base = smem_addr(sA), b_base = smem_addr(sB);
             uint32_t stage = 0, phase = 0;
             uint32_t gcount = 0;     // groups issued so far (slot = gcount & 1)
@@ -238,15 +261,21 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                         // the descriptors' address field (units of 16 bytes)
                         const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage);
                         const uint64_t bdesc = make_operand_desc(b_base + stage * C::kBStage);
+                        // MXFP4: K step j reads the columns of atom j/2 and
+                        // its bytes {0,1} or {2,3} (descriptor's scale IDs)
+                        auto kstep = [&](int j) {
+                            if constexpr (MX)
+                                mma_mxf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, (j & 1) ? idesc_mx1 : idesc_mx0,
+                                              sf + 4 * (j >> 1), sf + 16 + 8 * (j >> 1), (ks | j) != 0 ? 1u : 0u);
+                            else
+                                mma_nvf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j,
+                                              sf + 16 + 8 * j, (ks | j) != 0 ? 1u : 0u);
+                        };
                         if (nk == 4) {
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                mma_nvf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j,
-                                              sf + 16 + 8 * j, (ks | j) != 0 ? 1u : 0u);
+                            for (int j = 0; j < 4; ++j) kstep(j);
                         } else {
-                            for (int j = 0; j < nk; ++j)
-                                mma_nvf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j,
-                                              sf + 16 + 8 * j, (ks | j) != 0 ? 1u : 0u);
+                            for (int j = 0; j < nk; ++j) kstep(j);
                         }
                         tc_commit_pair(&empty[stage], 0x3);
                         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -255,6 +284,11 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                 }
                 if (ok) tc_commit_pair(tfull, 0x3);
             }
+            // Tensor memory is freed after the final cluster barrier: first let
+            // every MMA this thread issued complete (bounded, also after an abort).
+            tc_commit_pair(mma_done, 0x1);
+            volatile uint32_t keep_waiting = 0u;
+            mbar_wait(mma_done, 0, args.timeout_ns, &keep_waiting, args.status);
         }
     } else {
         // ------------------------------------------------------------ TMEM warps
@@ -266,6 +300,9 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         const uint32_t leader_tempty = mapa_shared(smem_addr(tempty), 0);
         float alpha = 0.0f;
         bool alpha_ready = false;
+        // Largest |y| this thread stores; rows and columns past M and N are
+        // exact zeros (zero-filled operand rows), so folding them is harmless.
+        YMax ym;
         uint32_t gcount = 0;
         int t = 0;
         bool ok = true;
@@ -277,7 +314,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             tc_fence_after();
             if (!alpha_ready) {
                 asm volatile("griddepcontrol.wait;" ::: "memory");
-                alpha = __fmul_rn(*args.ga, *args.gb);
+                alpha = __fmul_rn(args.ga ? *args.ga : 1.0f, args.gb ? *args.gb : 1.0f);   // MXFP4: none
                 alpha_ready = true;
             }
             uint32_t r[4][32];
@@ -310,6 +347,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                             __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(src[2 * k]), alpha),
                                                                       __fmul_rn(__uint_as_float(src[2 * k + 1]), alpha));
                             w[k] = *reinterpret_cast<uint32_t *>(&b2);
+                            ym.bf16x2(w[k]);
                         }
                         st_shared_v4(stg + lane * 128 + ((ch ^ (lane & 7)) * 16), w[0], w[1], w[2], w[3]);
                     }
@@ -327,7 +365,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                     OutT *yrow = static_cast<OutT *>(args.y) + static_cast<int64_t>(p) * args.ldy;
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
-                        pair_store_chunk<OutT>(r[c], alpha, yrow, qn * 256 + half * 128 + c * 32, args.N);
+                        pair_store_chunk<OutT>(r[c], alpha, yrow, qn * 256 + half * 128 + c * 32, args.N, ym);
                 }
             }
             return true;
@@ -354,11 +392,15 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                             const uint8_t *a_src = sSfa + st_i * C::kSfaStage + lane * 16;
                             const uint8_t *b_src = sSfb + st_i * C::kSfbStage + lane * 16;
+                            // the B box holds both row tiles' atoms, tile after tile:
+                            // 4 atoms each (NVFP4) or 2 (MXFP4, whose atom slots 2
+                            // and 3 hold bytes no MMA reads)
+                            constexpr int kTile1 = MX ? 1024 : 2048;
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 const uint4 a = ld_shared_v4(a_src + j * 512);
                                 const uint4 b0 = ld_shared_v4(b_src + j * 512);
-                                const uint4 b1 = ld_shared_v4(b_src + 2048 + j * 512);
+                                const uint4 b1 = ld_shared_v4(b_src + kTile1 + j * 512);
                                 uint32_t *va = v + h * C::kSlabCols + 4 * j;
                                 uint32_t *vb = v + h * C::kSlabCols + 16 + 8 * j;
                                 va[0] = a.x; va[1] = a.y; va[2] = a.z; va[3] = a.w;
@@ -392,10 +434,20 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         }
         if (ok && prev_tile >= 0) epilogue(t - 1, prev_tile);
         if (lane == 0) bulk_wait_group0();   // this warp's output stores are complete
+        float m = ym.value();
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) s_ymax[warp - 2] = m;
     }
 
     tc_fence_before();
     cluster_sync();       // no CTA leaves while its peer may still touch its memory
+    if (threadIdx.x == 0 && args.ymax_part != nullptr) {
+        float m = 0.0f;
+#pragma unroll
+        for (int k = 0; k < C::kTmemWarps; ++k) m = fmaxf(m, s_ymax[k]);
+        args.ymax_part[blockIdx.x] = m;
+    }
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (warp == 1) {
         tc_fence_after();
@@ -407,16 +459,19 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
 // Host side
 // ---------------------------------------------------------------------------
 
-template <typename OutT>
+template <typename OutT, bool MX>
 static cudaError_t run_pair(const Operand &act, const Operand &wgt, int64_t K, void *y, int64_t ldy,
-                            uint32_t *status, uint64_t timeout_ns, int max_clusters, cudaStream_t stream) {
+                            uint32_t *status, uint64_t timeout_ns, int max_clusters, cudaStream_t stream,
+                            float *ymax_part, int *nparts) {
     using C = PairCfg;
     const uint64_t k_steps = static_cast<uint64_t>(K / 64);
+    // 512-byte scale atoms per 128-row tile: one per K step (NVFP4), one per two (MXFP4)
+    const uint64_t atoms_rt = MX ? (k_steps + 1) / 2 : k_steps;
     CUtensorMap tmA, tmB, tmSA, tmSB;
     if (encode_tensor_map_u8(&tmA, act.codes, K / 2, act.rows, 128, 128) != CUDA_SUCCESS ||
         encode_tensor_map_u8(&tmB, wgt.codes, K / 2, wgt.rows, 128, 128) != CUDA_SUCCESS ||
-        encode_scale_map(&tmSA, act.scales, k_steps, ceil_div(act.rows, 128), 1) != CUDA_SUCCESS ||
-        encode_scale_map(&tmSB, wgt.scales, k_steps, ceil_div(wgt.rows, 128), 2) != CUDA_SUCCESS)
+        encode_scale_map(&tmSA, act.scales, atoms_rt, ceil_div(act.rows, 128), 1, MX ? 2 : 4) != CUDA_SUCCESS ||
+        encode_scale_map(&tmSB, wgt.scales, atoms_rt, ceil_div(wgt.rows, 128), 2, MX ? 2 : 4) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     CUtensorMap tmY;
     memset(&tmY, 0, sizeof(tmY));    // unused unless tma_store
@@ -436,15 +491,17 @@ static cudaError_t run_pair(const Operand &act, const Operand &wgt, int64_t K, v
     a.num_pm = static_cast<int32_t>(ceil_div(act.rows, 256));
     a.num_qn = static_cast<int32_t>(ceil_div(wgt.rows, 256));
     a.tma_store = tma_store ? 1 : 0;
+    a.ymax_part = ymax_part;
     a.status = status;
     a.timeout_ns = timeout_ns;
     const int tiles = a.num_pm * a.num_qn;
     const int clusters = tiles < max_clusters ? tiles : max_clusters;
-    cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_pair_kernel<OutT>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_pair_kernel<OutT, MX>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * clusters);
+    if (nparts) *nparts = 2 * clusters;
     cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
@@ -457,7 +514,7 @@ static cudaError_t run_pair(const Operand &act, const Operand &wgt, int64_t K, v
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<OutT>, tmA, tmB, tmSA, tmSB, tmY, a);
+    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<OutT, MX>, tmA, tmB, tmSA, tmSB, tmY, a);
 }
 
 // How many 2-CTA clusters of the pair kernel can be resident at once (0 if
@@ -466,10 +523,8 @@ static cudaError_t run_pair(const Operand &act, const Operand &wgt, int64_t K, v
 static int pair_max_clusters_query() {
     int n = 0;
     bool ok = true;
-    auto kb = gemm_nvf4_pair_kernel<__nv_bfloat16>;
-    auto kf = gemm_nvf4_pair_kernel<float>;
+    auto kb = gemm_nvf4_pair_kernel<__nv_bfloat16, false>;
     ok = ok && cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::kSmemBytes) == cudaSuccess;
-    ok = ok && cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::kSmemBytes) == cudaSuccess;
     if (ok) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2);
@@ -503,11 +558,15 @@ bool pair_gemm_usable(int64_t M, int64_t N, int num_sms) {
 }
 
 cudaError_t launch_gemm_pair(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
-                             int64_t ldy, uint32_t *status, uint64_t timeout_ns, cudaStream_t stream) {
+                             int64_t ldy, uint32_t *status, uint64_t timeout_ns, cudaStream_t stream,
+                             float *ymax_part, int *nparts, bool mx) {
     const int maxc = pair_max_clusters();
     if (maxc <= 0) return cudaErrorLaunchOutOfResources;
-    return y_bf16 ? run_pair<__nv_bfloat16>(act, wgt, K, y, ldy, status, timeout_ns, maxc, stream)
-                  : run_pair<float>(act, wgt, K, y, ldy, status, timeout_ns, maxc, stream);
+    if (mx)
+        return y_bf16 ? run_pair<__nv_bfloat16, true>(act, wgt, K, y, ldy, status, timeout_ns, maxc, stream, ymax_part, nparts)
+                      : run_pair<float, true>(act, wgt, K, y, ldy, status, timeout_ns, maxc, stream, ymax_part, nparts);
+    return y_bf16 ? run_pair<__nv_bfloat16, false>(act, wgt, K, y, ldy, status, timeout_ns, maxc, stream, ymax_part, nparts)
+                  : run_pair<float, false>(act, wgt, K, y, ldy, status, timeout_ns, maxc, stream, ymax_part, nparts);
 }
 
 }  // namespace nvfp4

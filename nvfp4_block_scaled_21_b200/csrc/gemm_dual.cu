@@ -60,7 +60,7 @@ struct DualCfg {
     static constexpr int kSfBase = 256;                       // after the two accumulators
     static constexpr int kTmemCols = 512;
     static constexpr int kThreads = 448;
-    static constexpr int kBarBytes = 8 * (3 * kStages + 2) + 16;
+    static constexpr int kBarBytes = 8 * (3 * kStages + 3) + 16;
     static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;
     static_assert(kSfBase + kStages * kSfCols <= kTmemCols, "tensor memory budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -86,7 +86,8 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     uint64_t *empty = sf_full + STAGES;
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 1;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tempty + 1);
+    uint64_t *mma_done = tempty + 1;                         // every MMA of this CTA has completed
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile uint32_t *abort_flag = tmem_holder + 1;
     __shared__ float warp_max[8];
 
@@ -104,6 +105,7 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         }
         mbar_init(tfull, 1);
         mbar_init(tempty, 8);
+        mbar_init(mma_done, 1);
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -166,6 +168,16 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
+            // No copy may still be landing when the CTA exits: wait (bounded,
+            // also after an abort) for the last load issued into every stage.
+            // On the normal path the MMA thread has consumed them all already.
+            // (Stages counted before a failed empty wait were issued; the
+            // preloaded ones always are.)
+            const int issued = it > pre ? it : pre;
+            volatile uint32_t keep_waiting = 0u;
+            for (int j = issued > STAGES ? issued - STAGES : 0; j < issued; ++j)
+                mbar_wait(&full[j % STAGES], static_cast<uint32_t>(j / STAGES) & 1u, args.timeout_ns,
+                          &keep_waiting, args.status);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -209,6 +221,11 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                 tc_commit(tfull);
                 acc_phase ^= 1u;
             }
+            // Tensor memory is freed below: first let every MMA this thread
+            // issued complete (bounded, also after an abort).
+            tc_commit(mma_done);
+            volatile uint32_t keep_waiting = 0u;
+            mbar_wait(mma_done, 0, args.timeout_ns, &keep_waiting, args.status);
         }
     } else if (warp < 6) {
         // ------------------------------------------------------------ scale warps

@@ -218,6 +218,22 @@ __device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint6
         : "memory");
 }
 
+// The same for MXFP4 operands: E2M1 elements with one UE8M0 scale per 32
+// elements, two scales per row per K = 64 step.  A 32-bit scale column holds
+// four 32-element blocks (K = 128); the instruction descriptor's scale-factor
+// ID fields pick bytes {0,1} or {2,3} of it (see make_idesc_mxf4).
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X"
+        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
 // Arrive once on `bar` when all previously issued tcgen05 async operations of
 // this thread have completed.
 __device__ __forceinline__ void tc_commit(uint64_t *bar) {
@@ -347,6 +363,15 @@ __host__ __device__ constexpr uint32_t make_idesc_nvf4(uint32_t n) {
          | ((128u >> 4) << 24); // M >> 4
 }
 
+// Instruction descriptor of kind::mxf4 (E2M1 A and B, UE8M0 scales, K-major,
+// dense K = 64, M = 128) for K step j of a 128-deep scale column: scale-factor
+// IDs (A: bits 29..30, B: bits 4..5) select the column's bytes {0,1} for even
+// j and {2,3} for odd j.
+__host__ __device__ constexpr uint32_t make_idesc_mxf4(uint32_t n, uint32_t m, uint32_t j) {
+    return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | (1u << 23) | ((m >> 4) << 24) |
+           ((2u * (j & 1u)) << 29) | ((2u * (j & 1u)) << 4);
+}
+
 // ---------------------------------------------------------------------------
 // Two-CTA (cluster of 2) forms: the pair shares one block-scaled MMA
 // (cta_group::2).  Multicast is used only on tcgen05.commit, never on loads.
@@ -412,6 +437,18 @@ __device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t a_desc, 
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X"
+        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X"
         " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
