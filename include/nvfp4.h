@@ -94,7 +94,9 @@ typedef enum {
     NVFP4_OP_DEQUANTIZE = 1,
     NVFP4_OP_GEMM = 2,
     NVFP4_OP_LINEAR_FUSED = 3,           /* nvfp4_linear_fused with NVFP4_EPI_STORE */
-    NVFP4_OP_LINEAR_FUSED_SILU = 4       /* nvfp4_linear_fused with NVFP4_EPI_SILU_MUL_REQUANT */
+    NVFP4_OP_LINEAR_FUSED_SILU = 4,      /* nvfp4_linear_fused with NVFP4_EPI_SILU_MUL_REQUANT */
+    NVFP4_OP_GEMM_REQUANT = 5,           /* nvfp4_gemm_requant */
+    NVFP4_OP_W4A16 = 6                   /* nvfp4_w4a16_linear (the status word only) */
 } nvfp4_op;
 
 typedef enum {
@@ -163,18 +165,46 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor *q, void *y, nvfp4_dt
  * block-scaled FP4 MMAs with fp32 accumulation in tensor memory.  y has row
  * pitch ldy (elements) and dtype yt (BF16 or F32); y may be NULL when M*N == 0
  * (nothing is written), and K == 0 zero-fills y.  W4A4 linear layer: a is
- * the activations, b the weights.
+ * the activations, b the weights.  Both operands stay 4-bit all the way into
+ * the tensor cores, with no dequantize-to-16-bit step (aixq.cc article on
+ * Unsloth Dynamic NVFP4, section "核心差异：W4A4 vs W4A16"); the tensor
+ * cores apply the E4M3 block scales themselves and the two FP32 tensor scales
+ * are applied once per output (NVFP4 wiki page, section "技術原理").
  */
 NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y, nvfp4_dtype yt,
                         int64_t ldy, void *ws, size_t ws_bytes, nvfp4_stream_t stream);
 
 /*
- * The W4A4 linear layer from high-precision activations.
- *   x [M][K] (pitch ldx, dtype xt) is quantized to NVFP4 on the device
- *   ("dynamic" per-call scaling of the activations), then multiplied with the
- *   pre-quantized weights.
+ * nvfp4_gemm, and the output re-quantized to NVFP4 for the next layer:
+ * y_q (y_q->rows == M, y_q->cols == N, N % 16 == 0) receives y AS STORED
+ * (after rounding to y's dtype) quantized with the rules above, with its own
+ * tensor scale over all of y -- the same bytes nvfp4_quantize(y) would give.
+ * Every NVFP4 tensor carries its own two-level scaling (NVFP4 wiki page,
+ * section "技術原理"), so the next layer's activations get a fresh tensor
+ * scale.  The GEMM's epilogue records the largest |y| each CTA stores, so
+ * only the quantizer's encode pass runs afterwards (one more read of y).
+ * K == 0 gives y = 0 and an all-zero y_q with g = 0; M == 0 or N == 0 writes
+ * only y_q's g (0).  Workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM_REQUANT, ...).
+ */
+NVFP4_API nvfp4_status nvfp4_gemm_requant(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y, nvfp4_dtype yt,
+                                          int64_t ldy, const nvfp4_tensor *y_q, void *ws, size_t ws_bytes,
+                                          nvfp4_stream_t stream);
+
+/*
+ * The W4A4 linear layer from high-precision activations (aixq.cc article on
+ * Unsloth Dynamic NVFP4, section "核心差异：W4A4 vs W4A16": weights and
+ * activations both 4-bit, straight into the FP4 tensor cores).
+ *   x [M][K] (pitch ldx, dtype xt) is quantized to NVFP4 on the device on
+ *   every call, its scales derived from this call's values (the mobdome post
+ *   on Qwen3.6-27B-NVFP4, section "第二層：動態縮放（Dynamic Scaling）"), then
+ *   multiplied with the pre-quantized weights.
  *   epilogue == NVFP4_EPI_STORE: y [M][w->rows] = x_q . w^T * gx * gw
- *     (w_up, y_q ignored; y required, dtype yt, pitch ldy).
+ *     (w_up ignored; y required, dtype yt, pitch ldy).  If y_q is not NULL,
+ *     y as stored is also quantized to NVFP4 into y_q (y_q->rows == M,
+ *     y_q->cols == w->rows, a multiple of 16), with its own tensor scale, as
+ *     nvfp4_gemm_requant does; K == 0 then gives an all-zero y_q, N == 0 only
+ *     its g (0).  For M <= 16 (decode) the activation quantizer runs inside
+ *     the GEMM kernel, one launch per call (two with y_q).
  *   epilogue == NVFP4_EPI_SILU_MUL_REQUANT: gate = x_q . w^T, up = x_q . w_up^T
  *     (w_up->rows == w->rows), h = SiLU(gate) * up in fp32, SiLU(z) =
  *     z / (1 + exp(-z)); h is quantized to NVFP4 into y_q (y_q->rows == M,
@@ -211,11 +241,14 @@ NVFP4_API nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t
  *   with NVFP4_ERR_UNSUPPORTED_SHAPE and nothing is launched.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is kept for the rest of the
+ *   process: call from the device's primary context (the CUDA runtime's) only,
+ *   and not after a cudaDeviceReset, after which the array may sit elsewhere.
  *   Every call shares the one array and finds the previous call's contents in
  *   it: calls that overlap on the GPU race on it.  Each call clears the status
  *   word first and rewrites everything else.  Device-side waits give up after
- *   2 s; there is no status readback for this entry point (use
+ *   the bound set by nvfp4_set_wait_timeout_us, like every other entry
+ *   point's; there is no status readback for this entry point (use
  *   nvfp4_linear_fused with a workspace to observe one).
  *   Other arguments, layouts and errors as nvfp4_linear_fused; allocates
  *   nothing (no cudaMalloc, cudaFree or allocating library routine).
@@ -223,6 +256,67 @@ NVFP4_API nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t
 NVFP4_API nvfp4_status nvfp4_linear_noalloc(const void *x, nvfp4_dtype xt, int64_t M, int64_t K,
                                             int64_t ldx, const nvfp4_tensor *w, void *y,
                                             nvfp4_dtype yt, int64_t ldy, nvfp4_stream_t stream);
+
+/*
+ * MXFP4 (eefocus.com article on FP4 vs INT4, section
+ * "FP4被视为下一代AI计算的核心标准"; the OCP MX format): E2M1 elements, 32
+ * consecutive elements along a row share one E8M0 scale (a power of two),
+ * about 4.25 bits per value, no second-level tensor scale.
+ *   scale   X = 2^e, e = ceil(log2(bamax / 6)) clamped to [-127, 127]: the
+ *           smallest power of two with bamax <= 6 X (an all-zero block gets
+ *           byte 0); the page gives no rule, this one never saturates.
+ *   element code = E2M1_rne_satfinite(x / X) (exact division), with the NVFP4
+ *           tie and sign rules.
+ * Layout as nvfp4_tensor, with kb counting 32-element blocks: scale byte of
+ * block kb of row r at ((r/128)*(KB4/4) + kb/4)*512 + (r%32)*16 +
+ * ((r/32)%4)*4 + kb%4, KB4 = roundup(cols/32, 4); one 512-byte atom covers
+ * 128 rows x 128 columns.
+ */
+typedef struct {
+    uint8_t *codes;                      /* [rows][cols/2], element 2j in the low nibble of byte j */
+    uint8_t *scales;                     /* nvfp4_mx_scales_bytes(rows, cols) bytes, tiled as above */
+    int64_t rows;
+    int64_t cols;                        /* a multiple of 32 */
+} nvfp4_mx_tensor;
+
+/* Bytes of the tiled MXFP4 scale array: roundup(rows,128) * roundup(cols/32,4). */
+NVFP4_API size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t cols);
+
+/*
+ * Quantize x [rows][cols] (pitch ld elements, dtype xt; cols % 32 == 0) to
+ * MXFP4 into out.  One pass (no tensor amax, no workspace); padding of the
+ * scale layout is written as 0.
+ */
+NVFP4_API nvfp4_status nvfp4_mx_quantize(const void *x, nvfp4_dtype xt, int64_t rows, int64_t cols,
+                                         int64_t ld, const nvfp4_mx_tensor *out, nvfp4_stream_t stream);
+
+/*
+ * y[M][N] = A . B^T for MXFP4 A [M][K] and B [N][K] (K % 64 == 0) on the
+ * block-scaled FP4 tensor cores (kind::mxf4, one UE8M0 scale per 32
+ * elements), fp32 accumulation; kernels, output dtypes, pitches and
+ * workspace (nvfp4_workspace_bytes(NVFP4_OP_GEMM, M, N, K)) as nvfp4_gemm.
+ */
+NVFP4_API nvfp4_status nvfp4_mx_gemm(const nvfp4_mx_tensor *a, const nvfp4_mx_tensor *b, void *y, nvfp4_dtype yt,
+                                     int64_t ldy, void *ws, size_t ws_bytes, nvfp4_stream_t stream);
+
+/*
+ * W4A16 linear layer: y[M][N] = x . deq(w)^T with 16-bit activations x
+ * [M][K] (xt must be NVFP4_BF16, pitch ldx) and NVFP4 weights w [N][K]
+ * (K % 64 == 0), the scheme the aixq.cc article on Unsloth Dynamic NVFP4
+ * (section "核心差异：W4A4 vs W4A16") compares W4A4 against: the weights are
+ * dequantized to 16 bits before a 16-bit matrix product.  Each weight value
+ * e * s (E2M1 element times E4M3 block scale) is exact in bf16, so the
+ * kernel dequantizes in registers straight into the tensor cores' operand
+ * memory and applies the tensor scale to the fp32 accumulator:
+ *   y = fl32(acc * g_w), acc = sum_k x[m][k] * (e*s)[n][k] accumulated in fp32,
+ * then RNE to bf16 for a bf16 y.  Tiles of 128 weight rows x 16 activation
+ * rows; larger M repeats the weight stream per 16 activation rows (the
+ * decode-shaped path, not a prefill tile).  Workspace: the status word
+ * (nvfp4_workspace_bytes(NVFP4_OP_W4A16, ...) = 256 bytes).
+ */
+NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void *x, nvfp4_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                          const nvfp4_tensor *w, void *y, nvfp4_dtype yt, int64_t ldy, void *ws,
+                                          size_t ws_bytes, nvfp4_stream_t stream);
 
 /*
  * Synchronise `stream`, read the sticky device status word in ws, clear it,

@@ -26,14 +26,15 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_WORKSPACE, ERR_CUDA, \
     ERR_TIMEOUT, ERR_ARCH = range(8)
 F32, BF16 = 0, 1
-OP_QUANTIZE, OP_DEQUANTIZE, OP_GEMM, OP_LINEAR_FUSED, OP_LINEAR_FUSED_SILU = range(5)
+OP_QUANTIZE, OP_DEQUANTIZE, OP_GEMM, OP_LINEAR_FUSED, OP_LINEAR_FUSED_SILU, OP_GEMM_REQUANT, OP_W4A16 = range(7)
 EPI_STORE, EPI_SILU_MUL_REQUANT = 0, 1
 
 EXPORTED = (
     "nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize",
     "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_linear_fused", "nvfp4_get_device_status",
     "nvfp4_selftest_bounded_wait", "nvfp4_set_wait_timeout_us", "nvfp4_status_string",
-    "nvfp4_version", "nvfp4_linear_noalloc",
+    "nvfp4_version", "nvfp4_linear_noalloc", "nvfp4_gemm_requant", "nvfp4_mx_scales_bytes",
+    "nvfp4_mx_quantize", "nvfp4_mx_gemm", "nvfp4_w4a16_linear",
 )
 
 
@@ -44,8 +45,15 @@ class CTensor(ctypes.Structure):
                 ("cols", ctypes.c_int64)]
 
 
+class CMXTensor(ctypes.Structure):
+    """``nvfp4_mx_tensor`` of the C ABI."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64)]
+
+
 _P, _I64, _SZ, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
 _T = ctypes.POINTER(CTensor)
+_TM = ctypes.POINTER(CMXTensor)
 
 _lib.nvfp4_codes_bytes.argtypes = [_I64, _I64]
 _lib.nvfp4_codes_bytes.restype = _SZ
@@ -59,6 +67,16 @@ _lib.nvfp4_dequantize.argtypes = [_T, _P, _I, _I64, _P]
 _lib.nvfp4_dequantize.restype = _I
 _lib.nvfp4_gemm.argtypes = [_T, _T, _P, _I, _I64, _P, _SZ, _P]
 _lib.nvfp4_gemm.restype = _I
+_lib.nvfp4_gemm_requant.argtypes = [_T, _T, _P, _I, _I64, _T, _P, _SZ, _P]
+_lib.nvfp4_gemm_requant.restype = _I
+_lib.nvfp4_mx_scales_bytes.argtypes = [_I64, _I64]
+_lib.nvfp4_mx_scales_bytes.restype = _SZ
+_lib.nvfp4_mx_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _TM, _P]
+_lib.nvfp4_mx_quantize.restype = _I
+_lib.nvfp4_mx_gemm.argtypes = [_TM, _TM, _P, _I, _I64, _P, _SZ, _P]
+_lib.nvfp4_mx_gemm.restype = _I
+_lib.nvfp4_w4a16_linear.argtypes = [_P, _I, _I64, _I64, _I64, _T, _P, _I, _I64, _P, _SZ, _P]
+_lib.nvfp4_w4a16_linear.restype = _I
 _lib.nvfp4_linear_fused.argtypes = [_P, _I, _I64, _I64, _I64, _T, _T, _I, _P, _I, _I64, _T, _T,
                                     _P, _SZ, _P]
 _lib.nvfp4_linear_fused.restype = _I
@@ -151,6 +169,25 @@ class NVFP4Tensor:
                        self.tensor_scale.data_ptr(), self.rows, self.cols)
 
 
+@dataclass
+class MXFP4Tensor:
+    """Device buffers of one MXFP4 tensor [rows][cols] (see ``nvfp4_mx_tensor``)."""
+    codes: "object"          # uint8 [rows, cols/2]
+    scales: "object"         # uint8 [nvfp4_mx_scales_bytes]
+    rows: int
+    cols: int
+
+    @staticmethod
+    def empty(rows: int, cols: int, device="cuda") -> "MXFP4Tensor":
+        torch = _torch()
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+        scales = torch.empty(int(_lib.nvfp4_mx_scales_bytes(rows, cols)), dtype=torch.uint8, device=device)
+        return MXFP4Tensor(codes, scales, rows, cols)
+
+    def c(self) -> CMXTensor:
+        return CMXTensor(self.codes.data_ptr(), self.scales.data_ptr(), self.rows, self.cols)
+
+
 def _rows(*ts) -> None:
     """2-D tensors whose rows are contiguous (any row pitch): the layout the C
     ABI describes with a pointer and a row pitch.  A plain check, not an assert,
@@ -168,6 +205,14 @@ def _buffers(*qs) -> None:
     fp32 tensor scale), or the kernels would read or write past it."""
     for q in qs:
         if q is None:
+            continue
+        if isinstance(q, MXFP4Tensor):
+            for t, need, what in ((q.codes, codes_bytes(q.rows, q.cols), "codes"),
+                                  (q.scales, mx_scales_bytes(q.rows, q.cols), "scales")):
+                have = t.numel() * t.element_size()
+                if not t.is_contiguous() or have < need:
+                    raise ValueError(f"nvfp4: {what} of a {q.rows}x{q.cols} MXFP4 tensor needs {need} contiguous "
+                                     f"bytes; got {have} bytes")
             continue
         if q.tensor_scale.dtype != _torch().float32:
             raise TypeError(f"nvfp4: tensor_scale must be float32, got {q.tensor_scale.dtype}")
@@ -200,7 +245,8 @@ def _on_device(*objs) -> None:
     for o in objs:
         if o is None:
             continue
-        for t in ((o.codes, o.scales, o.tensor_scale) if isinstance(o, NVFP4Tensor) else (o,)):
+        for t in ((o.codes, o.scales, o.tensor_scale) if isinstance(o, NVFP4Tensor) else
+                  (o.codes, o.scales) if isinstance(o, MXFP4Tensor) else (o,)):
             if not t.is_cuda:
                 raise TypeError(f"nvfp4: got a tensor on {t.device}; the library needs CUDA tensors")
             if cur is None:
@@ -215,6 +261,10 @@ def codes_bytes(rows: int, cols: int) -> int:
 
 def scales_bytes(rows: int, cols: int) -> int:
     return int(_lib.nvfp4_scales_bytes(rows, cols))
+
+
+def mx_scales_bytes(rows: int, cols: int) -> int:
+    return int(_lib.nvfp4_mx_scales_bytes(rows, cols))
 
 
 def workspace_bytes(op: int, M: int, N: int, K: int) -> int:
@@ -264,6 +314,21 @@ def nvfp4_gemm(a: NVFP4Tensor, b: NVFP4Tensor, y, ws, stream=None):
     return y
 
 
+def nvfp4_gemm_requant(a: NVFP4Tensor, b: NVFP4Tensor, y, y_q: NVFP4Tensor, ws, stream=None):
+    """y[M][N] = (a . b^T) * ga * gb, and y as stored quantized to NVFP4 into y_q."""
+    _rows(y)
+    _buffers(a, b, y_q)
+    _shape(y, a.rows, b.rows)
+    if (y_q.rows, y_q.cols) != (a.rows, b.rows):
+        raise ValueError(f"nvfp4: y_q is {y_q.rows}x{y_q.cols}, expected {a.rows}x{b.rows}")
+    _on_device(a, b, y, y_q, ws)
+    ca, cb, cq = a.c(), b.c(), y_q.c()
+    st = _lib.nvfp4_gemm_requant(ctypes.byref(ca), ctypes.byref(cb), y.data_ptr(), _dtype_code(y),
+                                 y.stride(0), ctypes.byref(cq), ws.data_ptr(), _ws_bytes(ws), _stream(stream))
+    _check(st, "nvfp4_gemm_requant")
+    return y
+
+
 def nvfp4_linear_fused(x, w: NVFP4Tensor, ws, epilogue: int = EPI_STORE, y=None,
                        w_up: NVFP4Tensor | None = None, y_q: NVFP4Tensor | None = None,
                        x_q: NVFP4Tensor | None = None, stream=None):
@@ -303,6 +368,50 @@ def nvfp4_linear_noalloc(x, w: NVFP4Tensor, y, stream=None):
                                    y.stride(0), _stream(stream))
     _check(st, "nvfp4_linear_noalloc")
     return y
+
+
+def nvfp4_mx_quantize(x, out: MXFP4Tensor, stream=None) -> MXFP4Tensor:
+    """Quantize a 2-D bf16/fp32 CUDA tensor (row pitch x.stride(0)) to MXFP4 into out."""
+    _rows(x)
+    _buffers(out)
+    _on_device(x, out)
+    ct = out.c()
+    st = _lib.nvfp4_mx_quantize(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], x.stride(0),
+                                ctypes.byref(ct), _stream(stream))
+    _check(st, "nvfp4_mx_quantize")
+    return out
+
+
+def nvfp4_mx_gemm(a: MXFP4Tensor, b: MXFP4Tensor, y, ws, stream=None):
+    """y[M][N] = a . b^T for MXFP4 operands (workspace as for OP_GEMM)."""
+    _rows(y)
+    _buffers(a, b)
+    _shape(y, a.rows, b.rows)
+    _on_device(a, b, y, ws)
+    ca, cb = a.c(), b.c()
+    st = _lib.nvfp4_mx_gemm(ctypes.byref(ca), ctypes.byref(cb), y.data_ptr(), _dtype_code(y), y.stride(0),
+                            ws.data_ptr(), _ws_bytes(ws), _stream(stream))
+    _check(st, "nvfp4_mx_gemm")
+    return y
+
+
+def nvfp4_w4a16_linear(x, w: NVFP4Tensor, y, ws, stream=None):
+    """W4A16: y = x . deq(w)^T with bf16 activations x [M][K] and NVFP4 weights."""
+    _rows(x, y)
+    _buffers(w)
+    _shape(y, x.shape[0], w.rows)
+    _on_device(x, w, y, ws)
+    cw = w.c()
+    st = _lib.nvfp4_w4a16_linear(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], x.stride(0), ctypes.byref(cw),
+                                 y.data_ptr(), _dtype_code(y), y.stride(0), ws.data_ptr(), _ws_bytes(ws),
+                                 _stream(stream))
+    _check(st, "nvfp4_w4a16_linear")
+    return y
+
+
+def mx_quantize(x, stream=None) -> MXFP4Tensor:
+    """Allocate an MXFP4Tensor and quantize x into it."""
+    return nvfp4_mx_quantize(x, MXFP4Tensor.empty(x.shape[0], x.shape[1], device=x.device), stream)
 
 
 def nvfp4_get_device_status(ws, stream=None) -> int:

@@ -84,11 +84,13 @@ size_t quantized_bytes(int64_t rows, int64_t cols) {
            align256(static_cast<size_t>(round_up(rows, 128) * kb4_of(cols))) + 256;
 }
 
-uint64_t timeout_ns() { return static_cast<uint64_t>(g_wait_timeout_us.load()) * 1000ull; }
-
 nvfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
 
 }  // namespace
+
+namespace nvfp4 {
+uint64_t wait_timeout_ns() { return static_cast<uint64_t>(g_wait_timeout_us.load()) * 1000ull; }
+}  // namespace nvfp4
 
 extern "C" {
 
@@ -118,6 +120,11 @@ size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K) {
     case NVFP4_OP_LINEAR_FUSED_SILU:
         // status, partials | x_q | h (fp32 [M][N])
         return kQuantizeWs + quantized_bytes(M, K) + align256(static_cast<size_t>(M * N) * sizeof(float));
+    case NVFP4_OP_GEMM_REQUANT:
+        // status, partials (max |y| per GEMM CTA) | stream-K scratch
+        return kQuantizeWs + splitk_ws_bytes(M, N);
+    case NVFP4_OP_W4A16:
+        return kWsStatusBytes;
     }
     return 0;
 }
@@ -176,20 +183,49 @@ static nvfp4_status check_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, voi
     return NVFP4_OK;
 }
 
+// An all-zero NVFP4 tensor: g = 0, and (when it has elements) zero codes and
+// zero scales -- what the quantizer gives for an all-zero or empty input.
+static nvfp4_status zero_quantized(const nvfp4_tensor *q, cudaStream_t stream) {
+    if (cudaMemsetAsync(q->tensor_scale, 0, sizeof(float), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (q->rows * q->cols == 0) return NVFP4_OK;
+    if (cudaMemsetAsync(q->codes, 0, nvfp4_codes_bytes(q->rows, q->cols), stream) != cudaSuccess ||
+        cudaMemsetAsync(q->scales, 0, nvfp4_scales_bytes(q->rows, q->cols), stream) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
+}
+
+// The quantizer's encode pass on y as stored, from the per-CTA maxima the
+// GEMM's epilogue wrote: y_q gets its own tensor scale over all of y.
+static nvfp4_status requant_output(const void *y, nvfp4_dtype yt, int64_t ldy, const nvfp4_tensor *y_q,
+                                   const float *partials, int nparts, int num_sms, cudaStream_t stream) {
+    return from_cuda(launch_encode(y, yt == NVFP4_BF16, y_q->rows, y_q->cols, ldy, partials, nparts,
+                                   y_q->codes, y_q->scales, y_q->tensor_scale, num_sms, stream));
+}
+
 // weights_ready: b was not written by the kernel launched just before (true
 // inside nvfp4_linear_fused, whose first kernel is launched without a
 // programmatic dependency, so every earlier writer of b has finished).
+// y_q (optional): y is also quantized to NVFP4, as stored, with the per-CTA
+// maxima of |y| in `partials` (kMaxAmaxPartials floats).
 static nvfp4_status gemm_impl(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y,
                               nvfp4_dtype yt, int64_t ldy, uint32_t *status, int num_sms,
-                              cudaStream_t stream, bool weights_ready, void *splitk) {
-    if (a->rows == 0 || b->rows == 0) return NVFP4_OK;
-    if (a->cols == 0)   // empty reduction: y = 0
-        return from_cuda(cudaMemset2DAsync(y, ldy * (yt == NVFP4_BF16 ? 2 : 4), 0,
-                                           b->rows * (yt == NVFP4_BF16 ? 2 : 4), a->rows, stream));
+                              cudaStream_t stream, bool weights_ready, void *splitk,
+                              const nvfp4_tensor *y_q = nullptr, float *partials = nullptr) {
+    if (a->rows == 0 || b->rows == 0) return y_q ? zero_quantized(y_q, stream) : NVFP4_OK;
+    if (a->cols == 0) {   // empty reduction: y = 0, so y_q is all zero
+        if (cudaMemset2DAsync(y, ldy * (yt == NVFP4_BF16 ? 2 : 4), 0, b->rows * (yt == NVFP4_BF16 ? 2 : 4),
+                              a->rows, stream) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        return y_q ? zero_quantized(y_q, stream) : NVFP4_OK;
+    }
     Operand act{a->codes, a->scales, a->tensor_scale, a->rows};
     Operand wgt{b->codes, b->scales, b->tensor_scale, b->rows};
-    return from_cuda(launch_gemm(act, wgt, a->cols, y, yt == NVFP4_BF16, ldy, status, timeout_ns(),
-                                 num_sms, stream, weights_ready, splitk));
+    int nparts = 0;
+    const nvfp4_status st = from_cuda(launch_gemm(act, wgt, a->cols, y, yt == NVFP4_BF16, ldy, status,
+                                                  wait_timeout_ns(), num_sms, stream, weights_ready, splitk,
+                                                  y_q ? partials : nullptr, y_q ? &nparts : nullptr));
+    if (st != NVFP4_OK || !y_q) return st;
+    return requant_output(y, yt, ldy, y_q, partials, nparts, num_sms, stream);
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y, nvfp4_dtype yt,
@@ -202,6 +238,21 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y, n
     if ((st = current_device(&dev)) != NVFP4_OK) return st;
     return gemm_impl(a, b, y, yt, ldy, static_cast<uint32_t *>(ws), dev.sms,
                      reinterpret_cast<cudaStream_t>(stream), false, sk ? ws_at(ws, kWsStatusBytes) : nullptr);
+}
+
+nvfp4_status nvfp4_gemm_requant(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y, nvfp4_dtype yt,
+                                int64_t ldy, const nvfp4_tensor *y_q, void *ws, size_t ws_bytes,
+                                nvfp4_stream_t stream) {
+    nvfp4_status st = check_gemm(a, b, y, yt, ldy);
+    if (st != NVFP4_OK) return st;
+    if ((st = check_tensor(y_q, a->rows, b->rows)) != NVFP4_OK) return st;
+    const size_t sk = splitk_ws_bytes(a->rows, b->rows);
+    if ((st = check_ws(ws, ws_bytes, kQuantizeWs + sk)) != NVFP4_OK) return st;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    return gemm_impl(a, b, y, yt, ldy, static_cast<uint32_t *>(ws), dev.sms,
+                     reinterpret_cast<cudaStream_t>(stream), false, sk ? ws_at(ws, kQuantizeWs) : nullptr, y_q,
+                     reinterpret_cast<float *>(ws_at(ws, kPartialsOff)));
 }
 
 nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_t K, int64_t ldx,
@@ -226,6 +277,7 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
             return NVFP4_ERR_INVALID_ARG;
         if (M * N != 0 && (!aligned16(y) || (ldy * (yt == NVFP4_BF16 ? 2 : 4)) % 16))
             return NVFP4_ERR_MISALIGNED;
+        if (y_q && (st = check_tensor(y_q, M, N)) != NVFP4_OK) return st;
     } else {
         if (!w_up || (st = check_tensor(w_up, N, K)) != NVFP4_OK)
             return st != NVFP4_OK ? st : NVFP4_ERR_INVALID_ARG;
@@ -239,6 +291,21 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
     DevInfo dev;
     if ((st = current_device(&dev)) != NVFP4_OK) return st;
     if (M == 0) return NVFP4_OK;
+
+    uint32_t *status = static_cast<uint32_t *>(ws);
+    float *partials = reinterpret_cast<float *>(ws_at(ws, kPartialsOff));
+    // A few activation rows (decode): one kernel quantizes them inside the
+    // GEMM, while the weight stream is already in flight.
+    if (epilogue == NVFP4_EPI_STORE && decode_fused_usable(M, N, K)) {
+        Operand wgt{w->codes, w->scales, w->tensor_scale, N};
+        int nparts = 0;
+        st = from_cuda(launch_gemm_decode(x, xt == NVFP4_BF16, M, K, ldx, wgt, y, yt == NVFP4_BF16, ldy,
+                                          x_q ? x_q->codes : nullptr, x_q ? x_q->scales : nullptr,
+                                          x_q ? x_q->tensor_scale : nullptr, status, wait_timeout_ns(), dev.sms,
+                                          stream, y_q ? partials : nullptr, y_q ? &nparts : nullptr));
+        if (st != NVFP4_OK || !y_q) return st;
+        return requant_output(y, yt, ldy, y_q, partials, nparts, dev.sms, stream);
+    }
 
     // Quantized activations: caller's buffers or carved from the workspace.
     size_t off = kQuantizeWs;
@@ -257,13 +324,15 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
     }
     if (!x_q) off = kQuantizeWs + quantized_bytes(M, K);
     cudaError_t e = launch_quantize(x, xt == NVFP4_BF16, M, K, ldx, xq.codes, xq.scales,
-                                    xq.tensor_scale, reinterpret_cast<float *>(ws_at(ws, kPartialsOff)),
-                                    dev.sms, stream);
+                                    xq.tensor_scale, partials, dev.sms, stream);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
-    uint32_t *status = static_cast<uint32_t *>(ws);
+    // (The GEMM writes its per-CTA maxima of |y| into the same partials only
+    // at its end, after its dependent-launch wait, so the activation encode
+    // pass that reads them has finished by then.)
     if (epilogue == NVFP4_EPI_STORE)
         return gemm_impl(&xq, w, y, yt, ldy, status, dev.sms, stream, true,
-                         splitk_ws_bytes(M, N) != 0 ? ws_at(ws, kQuantizeWs + quantized_bytes(M, K)) : nullptr);
+                         splitk_ws_bytes(M, N) != 0 ? ws_at(ws, kQuantizeWs + quantized_bytes(M, K)) : nullptr,
+                         y_q, partials);
 
     // An empty reduction (K == 0) makes gate = up = 0, so h = SiLU(0) * 0 = 0:
     // y_q gets all-zero codes and scales and g = 0, y (if given) zeros.  With
@@ -285,13 +354,100 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
     Operand act{xq.codes, xq.scales, xq.tensor_scale, M};
     Operand og{w->codes, w->scales, w->tensor_scale, N};
     Operand ou{w_up->codes, w_up->scales, w_up->tensor_scale, N};
-    float *partials = reinterpret_cast<float *>(ws_at(ws, kPartialsOff));
     int nparts = 0;
     if (launch_gemm_dual_silu(act, og, ou, K, h, ldh, partials, kMaxAmaxPartials, &nparts, status,
-                              timeout_ns(), dev.sms, stream, true) != cudaSuccess)
+                              wait_timeout_ns(), dev.sms, stream, true) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     return from_cuda(launch_encode_f32(h, M, N, ldh, partials, nparts, y_q->codes, y_q->scales,
                                        y_q->tensor_scale, dev.sms, stream));
+}
+
+// ---------------------------------------------------------------------------
+// MXFP4
+// ---------------------------------------------------------------------------
+
+static nvfp4_status check_mx_tensor(const nvfp4_mx_tensor *t, int64_t rows, int64_t cols) {
+    if (!t || t->rows != rows || t->cols != cols || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+    if (rows * cols != 0 && (!t->codes || !t->scales)) return NVFP4_ERR_INVALID_ARG;
+    if (cols % 32) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(t->codes) || !aligned16(t->scales)) return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t cols) {
+    if (rows < 0 || cols < 0) return 0;
+    return static_cast<size_t>(round_up(rows, 128) * round_up(cols / 32, 4));
+}
+
+nvfp4_status nvfp4_mx_quantize(const void *x, nvfp4_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                               const nvfp4_mx_tensor *out, nvfp4_stream_t stream) {
+    if ((!x && rows * cols != 0) || (xt != NVFP4_F32 && xt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_mx_tensor(out, rows, cols);
+    if (st != NVFP4_OK) return st;
+    const int eb = xt == NVFP4_BF16 ? 2 : 4;
+    if (rows * cols != 0 && (!aligned16(x) || (ld * eb) % 16)) return NVFP4_ERR_MISALIGNED;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    return from_cuda(launch_mx_quantize(x, xt == NVFP4_BF16, rows, cols, ld, out->codes, out->scales, dev.sms,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_mx_gemm(const nvfp4_mx_tensor *a, const nvfp4_mx_tensor *b, void *y, nvfp4_dtype yt,
+                           int64_t ldy, void *ws, size_t ws_bytes, nvfp4_stream_t stream_) {
+    if (!a || !b || (yt != NVFP4_F32 && yt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if (!y && a->rows * b->rows != 0) return NVFP4_ERR_INVALID_ARG;
+    if (a->cols != b->cols) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_mx_tensor(a, a->rows, a->cols);
+    if (st != NVFP4_OK) return st;
+    if ((st = check_mx_tensor(b, b->rows, b->cols)) != NVFP4_OK) return st;
+    if (a->cols % 64) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (a->rows > kMaxGemmRows || b->rows > kMaxGemmRows || a->cols > kMaxGemmK) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ldy < b->rows) return NVFP4_ERR_INVALID_ARG;
+    const int eb = yt == NVFP4_BF16 ? 2 : 4;
+    if (a->rows * b->rows != 0 && (!aligned16(y) || (ldy * eb) % 16)) return NVFP4_ERR_MISALIGNED;
+    const size_t sk = splitk_ws_bytes(a->rows, b->rows);
+    if ((st = check_ws(ws, ws_bytes, kWsStatusBytes + sk)) != NVFP4_OK) return st;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (a->rows == 0 || b->rows == 0) return NVFP4_OK;
+    if (a->cols == 0)
+        return from_cuda(cudaMemset2DAsync(y, ldy * eb, 0, b->rows * eb, a->rows, stream));
+    Operand act{a->codes, a->scales, nullptr, a->rows};
+    Operand wgt{b->codes, b->scales, nullptr, b->rows};
+    return from_cuda(launch_gemm_mx(act, wgt, a->cols, y, yt == NVFP4_BF16, ldy, static_cast<uint32_t *>(ws),
+                                    wait_timeout_ns(), dev.sms, stream, sk ? ws_at(ws, kWsStatusBytes) : nullptr));
+}
+
+// ---------------------------------------------------------------------------
+// W4A16
+// ---------------------------------------------------------------------------
+
+nvfp4_status nvfp4_w4a16_linear(const void *x, nvfp4_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                const nvfp4_tensor *w, void *y, nvfp4_dtype yt, int64_t ldy, void *ws,
+                                size_t ws_bytes, nvfp4_stream_t stream_) {
+    if ((!x && M * K != 0) || !w || xt != NVFP4_BF16 || (yt != NVFP4_F32 && yt != NVFP4_BF16))
+        return NVFP4_ERR_INVALID_ARG;
+    if (M < 0 || K < 0 || ldx < K) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_tensor(w, w->rows, K);
+    if (st != NVFP4_OK) return st;
+    if (K % 64) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const int64_t N = w->rows;
+    if (M > kMaxGemmRows || N > kMaxGemmRows || K > kMaxGemmK) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if ((!y && M * N != 0) || ldy < N) return NVFP4_ERR_INVALID_ARG;
+    const int yeb = yt == NVFP4_BF16 ? 2 : 4;
+    if ((M * K != 0 && (!aligned16(x) || (ldx * 2) % 16)) || (M * N != 0 && (!aligned16(y) || (ldy * yeb) % 16)))
+        return NVFP4_ERR_MISALIGNED;
+    if ((st = check_ws(ws, ws_bytes, kWsStatusBytes)) != NVFP4_OK) return st;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (M == 0 || N == 0) return NVFP4_OK;
+    if (K == 0) return from_cuda(cudaMemset2DAsync(y, ldy * yeb, 0, N * yeb, M, stream));
+    Operand wgt{w->codes, w->scales, w->tensor_scale, N};
+    return from_cuda(launch_gemm_w4a16(x, M, K, ldx, wgt, y, yt == NVFP4_BF16, ldy, static_cast<uint32_t *>(ws),
+                                       wait_timeout_ns(), dev.sms, stream));
 }
 
 nvfp4_status nvfp4_get_device_status(void *ws, nvfp4_stream_t stream) {

@@ -17,7 +17,11 @@
 // only a host-side stand-in, never a device address, so its device address is
 // looked up per device with cudaGetSymbolAddress, with that device current, on
 // the first call made on that device; make that first call before any stream
-// capture.  Every call shares the one array and finds the previous call's
+// capture.  The address is cached per device ordinal for the life of the
+// process, so it is only valid for the context it was looked up in: call this
+// entry point from the device's primary context (the runtime's own) only, and
+// not after cudaDeviceReset, which unloads the module so that the array may
+// come back at another address.  Every call shares the one array and finds the previous call's
 // contents in it: calls that overlap on the GPU (two streams, two threads, or
 // a second call enqueued on another stream before the first finished) race on
 // it and corrupt each other.  What must start at zero (the device status word)
@@ -124,7 +128,7 @@ extern "C" nvfp4_status nvfp4_linear_noalloc(const void *x, nvfp4_dtype xt, int6
                                                                                     : NVFP4_ERR_CUDA;
     Operand act{xq_codes, xq_scales, xq_g, M};
     Operand wgt{w->codes, w->scales, w->tensor_scale, N};
-    return launch_gemm(act, wgt, K, y, yt == NVFP4_BF16, ldy, status, 2000000000ull, sms, stream) ==
+    return launch_gemm(act, wgt, K, y, yt == NVFP4_BF16, ldy, status, wait_timeout_ns(), sms, stream) ==
                    cudaSuccess
                ? NVFP4_OK
                : NVFP4_ERR_CUDA;
