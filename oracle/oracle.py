@@ -20,6 +20,9 @@ Parity status of each function (what pins it is in ``tests/test_oracle.py``):
                                       tiny case, closed form for constant
                                       operands.
 * ``silu_mul_f64``                   pinned: closed-form identities of SiLU.
+* ``w4a16_gemm_f64`` (16-bit          pinned: exact rational arithmetic from
+  activations x NVFP4 weights)        the code and scale bytes, a closed form
+                                      for constant weights, sign symmetry.
 * ``mx_*`` (MXFP4: 32-value blocks,  pinned: E8M0 decode of all 256 bytes
   E8M0 scales, no tensor scale)      against torch.float8_e8m0fnu; the scale
                                       rule by brute force over every byte;
@@ -270,6 +273,26 @@ def gemm_entries(a: Quantized, b: Quantized, ms, ns):
         _ptr(out), _ptr(na), _ptr(nb))
     assert rc == 0
     return out, na, nb
+
+
+def w4a16_gemm_f64(x: np.ndarray, w: Quantized, nthreads: int | None = None) -> np.ndarray:
+    """W4A16: Y = X . deq(W)^T in fp64 with 16-bit activations X [M][K] taken
+    as they are (bf16 given as uint16 bit patterns, or fp32) and NVFP4 weights
+    W [N][K] dequantized exactly (e * s * g).  The weights are 4-bit, the
+    activations stay 16-bit, and the product uses the dequantized weights
+    (aixq.cc article on Unsloth Dynamic NVFP4, section "核心差异：W4A4 vs
+    W4A16")."""
+    if x.dtype == np.uint16:
+        x = bf16_bits_to_f32(x)
+    xa = np.ascontiguousarray(x, dtype=np.float64)
+    if xa.ndim != 2 or xa.shape[1] != w.cols:
+        raise ValueError("x must be [M][K] with the weights' K")
+    dw = dequantize_f64(w)
+    y = np.empty((xa.shape[0], w.rows), np.float64)
+    nt = nthreads or os.cpu_count() or 1
+    rc = lib().oracle_gemm_f64(_ptr(xa), _ptr(dw), xa.shape[0], w.rows, w.cols, _ptr(y), int(nt))
+    assert rc == 0
+    return y
 
 
 def silu_mul_f64(gate: np.ndarray, up: np.ndarray) -> np.ndarray:

@@ -64,6 +64,9 @@ def test_workspace_sizes_follow_the_kernel_choices():
     M, N = 128, 5120
     xq = a256(M * K // 2) + a256(128 * (K // 16)) + 256
     assert nv.workspace_bytes(nv.OP_LINEAR_FUSED, M, N, K) == 256 + 4096 * 4 + xq + a256(128 * 5120 * 4) + a256(40 * 4)
+    # the re-quantizing GEMM: status + partial maxima of |y|, then the GEMM's stream-K scratch
+    assert nv.workspace_bytes(nv.OP_GEMM_REQUANT, 4096, 17408, 5120) == 256 + 4096 * 4
+    assert nv.workspace_bytes(nv.OP_GEMM_REQUANT, M, N, 17408) == 256 + 4096 * 4 + a256(128 * 5120 * 4) + a256(40 * 4)
 
 
 def test_status_strings():
@@ -104,6 +107,25 @@ def test_gemm_rejects_bad_arguments_without_launch():
     assert g(a, b, 16, nv.BF16, 16, 4096, 256) == nv.ERR_INVALID_ARG                       # ldy < N
     assert g(a, b, 16, nv.BF16, 36, 4096, 256) == nv.ERR_MISALIGNED                        # pitch
     assert g(a, b, 16, nv.BF16, 32, 4096, 8) == nv.ERR_WORKSPACE
+
+
+def test_gemm_requant_rejects_bad_arguments_without_launch():
+    """Each call breaks exactly one rule of nvfp4_gemm_requant and stops at it."""
+    lib = nv.lib()
+    a, b = _t(rows=8, cols=128), _t(rows=32, cols=128)
+
+    def g(a_=a, b_=b, y=16, yt=nv.BF16, ldy=32, yq=_t(rows=8, cols=32), ws=4096, wb=1 << 20):
+        return lib.nvfp4_gemm_requant(ctypes.byref(a_), ctypes.byref(b_), y, yt, ldy,
+                                      ctypes.byref(yq) if yq else None, ws, wb, None)
+
+    assert g(yq=None) == nv.ERR_INVALID_ARG                                         # y_q missing
+    assert g(yq=_t(rows=8, cols=48)) == nv.ERR_INVALID_ARG                          # y_q shape
+    assert g(b_=_t(rows=24, cols=128), ldy=24, yq=_t(rows=8, cols=24)) == nv.ERR_UNSUPPORTED_SHAPE  # N % 16
+    assert g(yq=_t(rows=8, cols=32, scales=24)) == nv.ERR_MISALIGNED
+    assert g(y=None) == nv.ERR_INVALID_ARG
+    assert g(ldy=36) == nv.ERR_MISALIGNED
+    assert g(wb=256) == nv.ERR_WORKSPACE                                            # needs the partials too
+    assert g(ws=None) == nv.ERR_WORKSPACE
 
 
 def test_linear_fused_rejects_bad_arguments_without_launch():
@@ -162,6 +184,8 @@ def test_linear_fused_rejects_more_bad_arguments_without_launch():
     assert f(**{**silu, "y": 24}) == nv.ERR_MISALIGNED
     assert f(**{**silu, "wu_": _t(rows=16, cols=128)}) == nv.ERR_INVALID_ARG        # w_up rows differ
     assert f(xq=_t(rows=8, cols=64)) == nv.ERR_INVALID_ARG                          # x_q shape
+    assert f(yq=_t(rows=8, cols=48)) == nv.ERR_INVALID_ARG                          # STORE y_q shape
+    assert f(yq=_t(rows=8, cols=32, codes=24)) == nv.ERR_MISALIGNED
     assert f(ws=None) == nv.ERR_WORKSPACE
     assert f(wb=64) == nv.ERR_WORKSPACE
     assert f(ws=4100) == nv.ERR_MISALIGNED
@@ -384,3 +408,41 @@ def test_package_fails_loudly_without_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import nvfp4_block_scaled_21_b200"], cwd=tmp_path,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "libnvfp4.so is missing" in r.stderr
+
+
+def _mx(codes=16, scales=16, rows=4, cols=64):
+    return nv.CMXTensor(codes, scales, rows, cols)
+
+
+def test_mx_sizes_and_argument_checks_without_launch():
+    """MXFP4: scale bytes roundup(rows,128) x roundup(cols/32,4); each call
+    below breaks exactly one rule of nvfp4_mx_quantize / nvfp4_mx_gemm."""
+    assert nv.mx_scales_bytes(8192, 5120) == 8192 * 160
+    assert nv.mx_scales_bytes(1, 32) == 128 * 4
+    assert nv.mx_scales_bytes(130, 96) == 256 * 4
+    lib = nv.lib()
+
+    def q(x=16, xt=nv.BF16, r=4, c=64, ld=64, o=_mx()):
+        return lib.nvfp4_mx_quantize(x, xt, r, c, ld, ctypes.byref(o) if o else None, None)
+
+    assert q(x=None) == nv.ERR_INVALID_ARG
+    assert q(xt=3) == nv.ERR_INVALID_ARG
+    assert q(ld=32) == nv.ERR_INVALID_ARG
+    assert q(o=None) == nv.ERR_INVALID_ARG
+    assert q(o=_mx(rows=5)) == nv.ERR_INVALID_ARG
+    assert q(c=48, ld=48, o=_mx(cols=48)) == nv.ERR_UNSUPPORTED_SHAPE            # cols % 32
+    assert q(x=24) == nv.ERR_MISALIGNED
+    assert q(o=_mx(scales=24)) == nv.ERR_MISALIGNED
+
+    a, b = _mx(rows=8, cols=128), _mx(rows=32, cols=128)
+
+    def g(a_=a, b_=b, y=16, yt=nv.BF16, ldy=32, ws=4096, wb=1 << 20):
+        return lib.nvfp4_mx_gemm(ctypes.byref(a_), ctypes.byref(b_), y, yt, ldy, ws, wb, None)
+
+    assert g(y=None) == nv.ERR_INVALID_ARG
+    assert g(b_=_mx(rows=32, cols=64)) == nv.ERR_INVALID_ARG                        # K mismatch
+    assert g(a_=_mx(rows=8, cols=96), b_=_mx(rows=32, cols=96)) == nv.ERR_UNSUPPORTED_SHAPE   # K % 64
+    assert g(ldy=16) == nv.ERR_INVALID_ARG
+    assert g(ldy=36) == nv.ERR_MISALIGNED
+    assert g(wb=8) == nv.ERR_WORKSPACE
+    assert g(yt=4) == nv.ERR_INVALID_ARG

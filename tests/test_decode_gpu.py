@@ -1,0 +1,161 @@
+"""GPU parity of the one-launch decode path (activation quantizer inside the
+GEMM, M <= 16) and of the W4A4 linear layer at full size through the exact
+call the benchmark times.
+
+The decode kernel quantizes x itself in the quantizer's arithmetic, so its
+x_q (codes, tiled scales, tensor scale) must equal the oracle's bit for bit,
+and y must be within the GEMM tolerance of the fp64 oracle product.  It runs
+the same MMAs in the same K order as the two-kernel path (quantizer passes,
+then the swapped GEMM), so the two paths' outputs are also compared bit for
+bit.  The full-size tests call nvfp4_linear_fused twice in a row on different
+rotation slots (different X and weight copies) without a synchronisation in
+between, as the benchmark's captured rotation does, so that a kernel that
+starts before the one before it has finished would show up."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import assert_gemm_close, assert_quantized_equal, bf16_tensor, f32_tensor, to_numpy_f64
+from nvfp4_block_scaled_21_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import nvfp4_block_scaled_21_b200 as nv
+    return nv
+
+
+def quantize_gpu(nv, x):
+    out = nv.NVFP4Tensor.empty(*x.shape)
+    nv.nvfp4_quantize(x, out, nv.workspace(nv.OP_QUANTIZE, x.shape[0], 0, x.shape[1]))
+    return out
+
+
+def norms(q):
+    return np.linalg.norm(oracle.dequantize_f64(q), axis=1)
+
+
+def make_inputs(M, N, K, seed, x_dtype):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[rng.random(x.shape) < 1e-3] *= 50
+    wt = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    if x_dtype == torch.bfloat16:
+        xt = torch.from_numpy(x).to(torch.bfloat16)
+        x_or = xt.view(torch.int16).numpy().view(np.uint16)     # the oracle reads bf16 bits
+    else:
+        xt = torch.from_numpy(x)
+        x_or = x
+    return xt, x_or, wt
+
+
+# M up to 16; partial last K slab (320, 1344), the largest K the kernel
+# takes (5632: 22 slabs), ragged N; bf16 and fp32 in and out.
+CASES = [
+    (1, 4096, 4096, torch.float32, torch.float32),
+    (5, 304, 64, torch.float32, torch.bfloat16),
+    (8, 1024, 1344, torch.bfloat16, torch.bfloat16),
+    (13, 640, 320, torch.bfloat16, torch.float32),
+    (16, 256, 5632, torch.bfloat16, torch.bfloat16),
+    (16, 1000, 320, torch.bfloat16, torch.float32),
+    (9, 128, 5120, torch.bfloat16, torch.bfloat16),
+    (12, 2048, 2048, torch.float32, torch.bfloat16),    # fp32 x, 384 groups: two load rounds
+]
+
+
+@pytest.mark.parametrize("M,N,K,xt,yt", CASES)
+def test_decode_fused_parity(nv, M, N, K, xt, yt):
+    x, x_or, wt = make_inputs(M, N, K, M * 1000 + K, xt)
+    xq_o, wq_o = oracle.quantize(x_or), oracle.quantize(wt)
+    wq = quantize_gpu(nv, f32_tensor(wt))
+    y = torch.full((M, N), float("nan"), dtype=yt, device="cuda")
+    x_q = nv.NVFP4Tensor.empty(M, K)
+    x_q.codes.fill_(0x77)
+    x_q.scales.fill_(0x55)
+    ws = nv.workspace(nv.OP_LINEAR_FUSED, M, N, K)
+    nv.nvfp4_linear_fused(x.cuda(), wq, ws, nv.EPI_STORE, y=y, x_q=x_q)
+    assert nv.nvfp4_get_device_status(ws) == nv.OK
+    assert_quantized_equal(x_q, xq_o)
+    ref = oracle.gemm_f64(xq_o, wq_o)
+    assert_gemm_close(to_numpy_f64(y), ref, norms(xq_o)[:, None], norms(wq_o)[None, :], K,
+                      yt == torch.bfloat16, "decode")
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 1000, 1344), (16, 384, 640), (3, 136, 192)])
+def test_decode_fused_matches_two_kernel_path(nv, M, N, K, monkeypatch):
+    """The one-launch kernel and the quantizer + swapped GEMM path give the
+    same bits; also with a row pitch wider than K and no x_q requested."""
+    x, _, wt = make_inputs(M, N, K, 7 * M + N, torch.bfloat16)
+    buf = torch.zeros((M, K + 40), dtype=torch.bfloat16, device="cuda")
+    buf[:, :K] = x.cuda()
+    wq = quantize_gpu(nv, f32_tensor(wt))
+    outs = []
+    for fused in ("1", "0"):
+        monkeypatch.setenv("NVFP4_DECODE_FUSED", fused)
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ws = nv.workspace(nv.OP_LINEAR_FUSED, M, N, K)
+        nv.nvfp4_linear_fused(buf[:, :K], wq, ws, nv.EPI_STORE, y=y)
+        assert nv.nvfp4_get_device_status(ws) == nv.OK
+        outs.append(y)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+
+
+def _two_slots(nv, w, xt_dtype=torch.bfloat16):
+    """Two rotation slots of a workload: X and W_q copies, as the benchmark
+    keeps them."""
+    X = bf16_tensor(w["X"])
+    wq = quantize_gpu(nv, bf16_tensor(w["W"]))
+    wq2 = nv.NVFP4Tensor(wq.codes.clone(), wq.scales.clone(), wq.tensor_scale.clone(), wq.rows, wq.cols)
+    return [X, X.clone()], [wq, wq2]
+
+
+def test_decode_workload_through_timed_call(nv):
+    """Decode workload at full size (M=8, N=17408, K=5120, seed 2) through
+    nvfp4_linear_fused(STORE, x_q) -- the benchmark's timed call -- twice in a
+    row on two slots: every output of both calls against the fp64 oracle, and
+    both x_q bit-exact."""
+    w = workloads.make("decode")
+    M, N, K = w["M"], w["N"], w["K"]
+    xq_o, wq_o = oracle.quantize(w["X"]), oracle.quantize(w["W"])
+    ref = oracle.gemm_f64(xq_o, wq_o)
+    Xs, Ws = _two_slots(nv, w)
+    ws = nv.workspace(nv.OP_LINEAR_FUSED, M, N, K)
+    ys = [torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    xqs = [nv.NVFP4Tensor.empty(M, K) for _ in range(2)]
+    for r in range(2):
+        nv.nvfp4_linear_fused(Xs[r], Ws[r], ws, nv.EPI_STORE, y=ys[r], x_q=xqs[r])
+    assert nv.nvfp4_get_device_status(ws) == nv.OK
+    for r in range(2):
+        assert_quantized_equal(xqs[r], xq_o)
+        assert_gemm_close(to_numpy_f64(ys[r]), ref, norms(xq_o)[:, None], norms(wq_o)[None, :], K, True,
+                          f"decode slot {r}")
+
+
+def test_prefill_workload_through_timed_call(nv):
+    """Prefill workload at full size (M=4096, N=17408, K=5120, seed 3) through
+    nvfp4_linear_fused(STORE, x_q), twice in a row on two slots: for each call
+    4096 random outputs plus one full row and one full column against the
+    fp64 oracle, and x_q bit-exact."""
+    w = workloads.make("prefill")
+    M, N, K = w["M"], w["N"], w["K"]
+    xq_o, wq_o = oracle.quantize(w["X"]), oracle.quantize(w["W"])
+    Xs, Ws = _two_slots(nv, w)
+    ws = nv.workspace(nv.OP_LINEAR_FUSED, M, N, K)
+    ys = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    xqs = [nv.NVFP4Tensor.empty(M, K) for _ in range(2)]
+    for r in range(2):
+        nv.nvfp4_linear_fused(Xs[r], Ws[r], ws, nv.EPI_STORE, y=ys[r], x_q=xqs[r])
+    assert nv.nvfp4_get_device_status(ws) == nv.OK
+    rng = np.random.default_rng(1)
+    ms = np.concatenate([rng.integers(0, M, 4096), np.full(N, 777), np.arange(M)])
+    ns = np.concatenate([rng.integers(0, N, 4096), np.arange(N), np.full(M, 12345)])
+    ref, na, nb = oracle.gemm_entries(xq_o, wq_o, ms, ns)
+    for r in range(2):
+        assert_quantized_equal(xqs[r], xq_o)
+        yc = ys[r].float().cpu().numpy().astype(np.float64)
+        assert np.isfinite(yc).all()
+        assert_gemm_close(yc[ms, ns], ref, na, nb, K, True, f"prefill slot {r}")
