@@ -31,14 +31,16 @@ sys.path.insert(0, ROOT)
 
 L2_BYTES = 126 * 1024 * 1024
 # DRAM bytes read + written per launch of each workload's dominant kernel(s),
-# from one ncu capture of the current kernels (profiles/*.md, "DRAM read /
-# write"); set an entry to None when its kernel changes.
-# (prefill, decode and mlp: the GEMM kernels changed after their capture, so
-# null until they are captured again)
-NCU_TRAFFIC = {"prefill": None, "decode": None, "quantize": 176_702_976, "mlp": None}
+# from one ncu capture of the current kernels (dram__bytes_read.sum +
+# dram__bytes_write.sum); None where the kernel changed after its capture or
+# the capture did not cover every kernel of the dominant call.
+NCU_TRAFFIC = {"prefill": 158_123_264, "decode": None, "quantize": 174_949_888, "mlp": None,
+               "prefill_requant": None, "mx_prefill": 153_339_392, "w4a16_decode": None,
+               "w4a8_prefill": None}
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP4_PER_BF16 = 4.0          # dense FP4 : dense BF16 on B200 (9 : 2.25 PFLOP/s nominal)
+FP8_PER_BF16 = 2.0          # dense FP8 (and FP8 x FP4) : dense BF16 (4.5 : 2.25 PFLOP/s nominal)
 
 
 def load_peaks():
@@ -110,7 +112,8 @@ class ClockSampler:
                     "samples": 0}
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
                 "reasons": [name for bit, name in _REASONS.items() if self.reasons & bit],
-                "samples": len(self.samples)}
+                "samples": len(self.samples),
+                "window": "the timed region and the per-step replays that follow it"}
 
 
 # ---------------------------------------------------------------------------
@@ -129,9 +132,22 @@ def _clone_q(nv, q, n):
     return out
 
 
+def _workloads():
+    """The seeded input generator, loaded from its file: importing it through
+    the package would load libnvfp4.so, which the reference arm must not map."""
+    import importlib.util
+    mod = sys.modules.get("_nvfp4_workloads")
+    if mod is None:
+        spec = importlib.util.spec_from_file_location(
+            "_nvfp4_workloads", os.path.join(ROOT, "nvfp4_block_scaled_21_b200", "workloads.py"))
+        mod = importlib.util.module_from_spec(spec)
+        sys.modules["_nvfp4_workloads"] = mod
+        spec.loader.exec_module(mod)
+    return mod
+
+
 def _gen(name):
-    from nvfp4_block_scaled_21_b200 import workloads
-    return workloads.make(name)
+    return _workloads().make(name)
 
 
 def _bf16(torch, bits):
@@ -209,12 +225,17 @@ class Decode(Prefill):
         # algorithmic bytes of the step: W codes + W scales, X bf16 in, Y bf16 out
         self.bytes = w_bytes + M * K * 2 + M * N * 2
         self.units = self.bytes / 1e9
-        gemm_bytes = w_bytes + M * K // 2 + M * K // 16 + M * N * 2
-        self.dominant = {"kernel": "gemm_nvf4_kernel (swapped, 128x16 tiles)", "bound": "hbm",
-                         "algorithmic": gemm_bytes, "unit": "GB/s"}
+        # One launch per step: the decode kernel quantizes X itself while the
+        # weight stream is in flight, so the step's kernel is the dominant one.
+        self.launches = 1
+        self.dominant = {"kernel": "gemm_decode_kernel (X quantized in-kernel, swapped 128x16 MMA tiles)",
+                         "bound": "hbm", "algorithmic": self.bytes, "unit": "GB/s"}
         self.config["workload"] = (f"decode W4A4 linear: quantize X bf16 {M}x{K} per call, GEMM with "
                                    f"pre-quantized W {N}x{K}, bf16 out")
         self.config["algorithmic_bytes_per_step"] = self.bytes
+
+    def dominant_call(self, i):
+        self.step(i)
 
 
 class Quantize:
@@ -342,7 +363,222 @@ class Mlp:
         return self.units / seconds_per_step
 
 
-WORKLOADS = {"prefill": Prefill, "decode": Decode, "quantize": Quantize, "mlp": Mlp}
+class PrefillRequant(Prefill):
+    """The prefill linear layer whose bf16 output is also re-quantized to
+    NVFP4 for the next layer (y_q of nvfp4_linear_fused's store form)."""
+    name = "prefill_requant"
+    metric = "NVFP4 GEMM TFLOPS (prefill, output re-quantized)"
+
+    def __init__(self, nv, torch):
+        super().__init__(nv, torch)
+        self.yq = nv.NVFP4Tensor.empty(self.M, self.N)
+        self.launches = 4                       # amax, encode (x); GEMM; encode (y)
+        # y (bf16, 142.6 MB) is read once more by the encode pass, which also
+        # writes y_q's codes and scales
+        self.requant_bytes = self.M * self.N * 2 + self.M * self.N // 2 + self.M * self.N // 16 + 4
+        self.dominant = {"kernel": "the fused call: x quantizer passes, gemm_nvf4_pair_kernel with per-CTA "
+                                   "max |y|, y encode pass", "bound": "tensor", "algorithmic": self.flops,
+                         "unit": "TFLOP/s"}
+        self.config = dict(self.config, workload=f"prefill W4A4 linear with y re-quantized: quantize X bf16 "
+                                                 f"{self.M}x{self.K}, GEMM with W {self.N}x{self.K}, bf16 y "
+                                                 f"and NVFP4 y_q", requant_pass_bytes=self.requant_bytes)
+
+    def step(self, i):
+        r = i % self.R
+        self.nv.nvfp4_linear_fused(self.X[r], self.Wq[r], self.wsl, self.nv.EPI_STORE, y=self.y, y_q=self.yq,
+                                   x_q=self.xq[r])
+
+    dominant_call = step
+
+    def e2e_setup(self):
+        super().e2e_setup()
+        self.c_host = torch_empty_pinned(self.torch, self.yq.codes)
+        self.d2h += self.yq.codes.numel()
+
+    def e2e_step(self, i):
+        r = i % self.R
+        self.X[r].copy_(self.x_host, non_blocking=True)
+        self.nv.nvfp4_linear_fused(self.X[r], self.Wq[r], self.wsl, self.nv.EPI_STORE, y=self.y, y_q=self.yq)
+        self.y_host.copy_(self.y, non_blocking=True)
+        self.c_host.copy_(self.yq.codes, non_blocking=True)
+
+
+class MxPrefill:
+    """MXFP4 variant of the prefill GEMM: one-pass MXFP4 quantize of X
+    (32-value blocks, E8M0 scales, no tensor scale) and the kind::mxf4
+    block-scaled GEMM with pre-quantized MXFP4 weights."""
+    name = "mx_prefill"
+    metric = "MXFP4 GEMM TFLOPS (prefill)"
+    unit = "TFLOP/s"
+
+    def __init__(self, nv, torch):
+        w = _gen("prefill")
+        self.M, self.K, self.N = w["M"], w["K"], w["N"]
+        W = _bf16(torch, w["W"])
+        wq = nv.mx_quantize(W)
+        del W
+        X = _bf16(torch, w["X"])
+        per_step = X.numel() * 2 + wq.codes.numel() + wq.scales.numel()
+        self.R = max(2, -(-2 * L2_BYTES // per_step))
+        self.X = _copies(X, self.R)
+        self.Wq = [wq] + [nv.MXFP4Tensor(wq.codes.clone(), wq.scales.clone(), wq.rows, wq.cols)
+                          for _ in range(self.R - 1)]
+        self.xq = [nv.MXFP4Tensor.empty(self.M, self.K) for _ in range(self.R)]
+        self.y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device="cuda")
+        self.ws = nv.workspace(nv.OP_GEMM, self.M, self.N, self.K)
+        self.nv, self.torch = nv, torch
+        self.flops = 2.0 * self.M * self.N * self.K
+        self.units = self.flops / 1e12
+        self.launches = 2                       # MX quantize, GEMM
+        self.dominant = {"kernel": "gemm_nvf4_pair_kernel<MX> (kind::mxf4, CTA pair, 256x256 tiles)",
+                         "bound": "tensor", "algorithmic": self.flops, "unit": "TFLOP/s"}
+        self.config = {"workload": f"MXFP4 prefill linear: quantize X bf16 {self.M}x{self.K} to MXFP4 per call, "
+                                   f"GEMM with pre-quantized MXFP4 W {self.N}x{self.K}, bf16 out",
+                       "M": self.M, "N": self.N, "K": self.K,
+                       "l2": f"{self.R} rotating copies of X and W_q > 126 MB L2"}
+
+    def step(self, i):
+        r = i % self.R
+        self.nv.nvfp4_mx_quantize(self.X[r], self.xq[r])
+        self.nv.nvfp4_mx_gemm(self.xq[r], self.Wq[r], self.y, self.ws)
+
+    def dominant_call(self, i):
+        r = i % self.R
+        self.nv.nvfp4_mx_gemm(self.xq[r], self.Wq[r], self.y, self.ws)
+
+    def e2e_setup(self):
+        self.x_host = self.X[0].cpu().pin_memory()
+        self.y_host = torch_empty_pinned(self.torch, self.y)
+        self.h2d = self.x_host.numel() * 2
+        self.d2h = self.y.numel() * 2
+
+    def e2e_step(self, i):
+        r = i % self.R
+        self.X[r].copy_(self.x_host, non_blocking=True)
+        self.step(i)
+        self.y_host.copy_(self.y, non_blocking=True)
+
+    def value(self, seconds_per_step):
+        return self.units / seconds_per_step
+
+
+class W4A8Prefill:
+    """W4A8 at the prefill shape: MXFP4 weights times MXFP8 activations (E4M3
+    elements, one E8M0 scale per 32), the activations quantized per call
+    inside nvfp4_w4a8_linear, then the kind::mxf8f6f4 block-scaled GEMM, which
+    runs at the FP8 tensor rate."""
+    name = "w4a8_prefill"
+    metric = "W4A8 GEMM TFLOPS (prefill)"
+    unit = "TFLOP/s"
+
+    def __init__(self, nv, torch):
+        w = _gen("prefill")
+        self.M, self.K, self.N = w["M"], w["K"], w["N"]
+        W = _bf16(torch, w["W"])
+        wq = nv.mx_quantize(W)
+        del W
+        X = _bf16(torch, w["X"])
+        per_step = X.numel() * 2 + wq.codes.numel() + wq.scales.numel()
+        self.R = max(2, -(-2 * L2_BYTES // per_step))
+        self.X = _copies(X, self.R)
+        self.Wq = [wq] + [nv.MXFP4Tensor(wq.codes.clone(), wq.scales.clone(), wq.rows, wq.cols)
+                          for _ in range(self.R - 1)]
+        self.xq = [nv.MXFP8Tensor.empty(self.M, self.K) for _ in range(self.R)]
+        self.y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device="cuda")
+        self.wsl = nv.workspace(nv.OP_W4A8_LINEAR, self.M, self.N, self.K)
+        self.wsg = nv.workspace(nv.OP_GEMM, self.M, self.N, self.K)
+        self.nv, self.torch = nv, torch
+        self.flops = 2.0 * self.M * self.N * self.K
+        self.units = self.flops / 1e12
+        self.launches = 2                       # MXFP8 quantize, GEMM
+        self.dominant = {"kernel": "gemm_nvf4_kernel<W4A8> (kind::mxf8f6f4, one CTA, 128x256 tiles)",
+                         "bound": "tensor", "algorithmic": self.flops, "unit": "TFLOP/s",
+                         "per_bf16": FP8_PER_BF16, "peak_name": "dense FP8"}
+        self.config = {"workload": f"W4A8 prefill linear: quantize X bf16 {self.M}x{self.K} to MXFP8 per call, "
+                                   f"GEMM with pre-quantized MXFP4 W {self.N}x{self.K}, bf16 out",
+                       "M": self.M, "N": self.N, "K": self.K,
+                       "l2": f"{self.R} rotating copies of X and W_q > 126 MB L2"}
+
+    def step(self, i):
+        r = i % self.R
+        self.nv.nvfp4_w4a8_linear(self.X[r], self.Wq[r], self.y, self.wsl, x_q=self.xq[r])
+
+    def dominant_call(self, i):
+        r = i % self.R
+        self.nv.nvfp4_w4a8_gemm(self.xq[r], self.Wq[r], self.y, self.wsg)
+
+    def e2e_setup(self):
+        self.x_host = self.X[0].cpu().pin_memory()
+        self.y_host = torch_empty_pinned(self.torch, self.y)
+        self.h2d = self.x_host.numel() * 2
+        self.d2h = self.y.numel() * 2
+
+    def e2e_step(self, i):
+        r = i % self.R
+        self.X[r].copy_(self.x_host, non_blocking=True)
+        self.step(i)
+        self.y_host.copy_(self.y, non_blocking=True)
+
+    def value(self, seconds_per_step):
+        return self.units / seconds_per_step
+
+
+class W4A16Decode:
+    """The W4A16 comparison scheme at the decode shape: bf16 activations, the
+    same NVFP4 weights dequantized inside the kernel before bf16 MMAs."""
+    name = "w4a16_decode"
+    metric = "W4A16 GEMM GB/s (decode)"
+    unit = "GB/s"
+
+    def __init__(self, nv, torch):
+        w = _gen("decode")
+        self.M, self.K, self.N = w["M"], w["K"], w["N"]
+        M, N, K = self.M, self.N, self.K
+        W = _bf16(torch, w["W"])
+        wq = nv.quantize(W)
+        del W
+        X = _bf16(torch, w["X"])
+        w_bytes = N * K // 2 + N * K // 16
+        self.R = max(2, -(-2 * L2_BYTES // w_bytes))
+        self.X = _copies(X, self.R)
+        self.Wq = _clone_q(nv, wq, self.R)
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        self.ws = nv.workspace(nv.OP_W4A16, M, N, K)
+        self.nv, self.torch = nv, torch
+        self.bytes = w_bytes + M * K * 2 + M * N * 2
+        self.units = self.bytes / 1e9
+        self.launches = 1
+        self.dominant = {"kernel": "gemm_w4a16_kernel (weights dequantized into tensor memory, bf16 MMA)",
+                         "bound": "hbm", "algorithmic": self.bytes, "unit": "GB/s"}
+        self.config = {"workload": f"W4A16 decode linear: bf16 X {M}x{K}, NVFP4 W {N}x{K} dequantized in-kernel, "
+                                   f"bf16 out", "M": M, "N": N, "K": K, "algorithmic_bytes_per_step": self.bytes,
+                       "l2": f"{self.R} rotating copies of W_q > 126 MB L2"}
+
+    def step(self, i):
+        r = i % self.R
+        self.nv.nvfp4_w4a16_linear(self.X[r], self.Wq[r], self.y, self.ws)
+
+    dominant_call = step
+
+    def e2e_setup(self):
+        self.x_host = self.X[0].cpu().pin_memory()
+        self.y_host = torch_empty_pinned(self.torch, self.y)
+        self.h2d = self.x_host.numel() * 2
+        self.d2h = self.y.numel() * 2
+
+    def e2e_step(self, i):
+        r = i % self.R
+        self.X[r].copy_(self.x_host, non_blocking=True)
+        self.step(i)
+        self.y_host.copy_(self.y, non_blocking=True)
+
+    def value(self, seconds_per_step):
+        return self.units / seconds_per_step
+
+
+WORKLOADS = {"prefill": Prefill, "decode": Decode, "quantize": Quantize, "mlp": Mlp,
+             "prefill_requant": PrefillRequant, "mx_prefill": MxPrefill, "w4a16_decode": W4A16Decode,
+             "w4a8_prefill": W4A8Prefill}
 
 
 def torch_empty_pinned(torch, like):
@@ -454,13 +690,17 @@ def measure(wl, torch, K, W, world, local, sample_clocks=False):
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
+    # NVML clocks are sampled from the start of the timed region to the end of
+    # the per-step replays that follow it under the same load (the timed
+    # region alone can be a few milliseconds, shorter than one sample period)
     sampler = ClockSampler(local) if sample_clocks else None
+    if sampler:
+        sampler.__enter__()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with (sampler if sampler else _Null()):
-        start.record()
-        _replay_k(steps, steps_rot, wl.R, K)
-        end.record()
-        torch.cuda.synchronize()
+    start.record()
+    _replay_k(steps, steps_rot, wl.R, K)
+    end.record()
+    torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     elapsed = max_over_ranks(world, start.elapsed_time(end) / 1e3)
@@ -471,6 +711,8 @@ def measure(wl, torch, K, W, world, local, sample_clocks=False):
         steps[(W + i) % wl.R].replay()
         evs[i][1].record()
     torch.cuda.synchronize()
+    if sampler:
+        sampler.__exit__(None, None, None)
     per = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)
     dist = {"median": round(per[K // 2], 2), "p10": round(per[int(0.1 * (K - 1))], 2),
             "p90": round(per[int(0.9 * (K - 1))], 2), "unit": "us", "rank": "local"}
@@ -515,10 +757,11 @@ def measure_e2e(wl, torch, K, world):
 def roofline(wl, kern_us, peaks):
     d = wl.dominant
     if d["bound"] == "tensor":
+        ratio = d.get("per_bf16", FP4_PER_BF16)
         achieved = d["algorithmic"] / (kern_us * 1e-6) / 1e12
-        peak = peaks["bf16_tflops"] * FP4_PER_BF16
+        peak = peaks["bf16_tflops"] * ratio
         unit = "TFLOP/s"
-        peak_note = (f"dense FP4 = {FP4_PER_BF16:g} x {peaks['source']} bf16 burst "
+        peak_note = (f"{d.get('peak_name', 'dense FP4')} = {ratio:g} x {peaks['source']} bf16 burst "
                      f"{peaks['bf16_tflops']:.1f} TFLOP/s")
     else:
         achieved = d["algorithmic"] / (kern_us * 1e-6) / 1e9

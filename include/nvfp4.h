@@ -96,7 +96,8 @@ typedef enum {
     NVFP4_OP_LINEAR_FUSED = 3,           /* nvfp4_linear_fused with NVFP4_EPI_STORE */
     NVFP4_OP_LINEAR_FUSED_SILU = 4,      /* nvfp4_linear_fused with NVFP4_EPI_SILU_MUL_REQUANT */
     NVFP4_OP_GEMM_REQUANT = 5,           /* nvfp4_gemm_requant */
-    NVFP4_OP_W4A16 = 6                   /* nvfp4_w4a16_linear (the status word only) */
+    NVFP4_OP_W4A16 = 6,                  /* nvfp4_w4a16_linear (the status word only) */
+    NVFP4_OP_W4A8_LINEAR = 7             /* nvfp4_w4a8_linear */
 } nvfp4_op;
 
 typedef enum {
@@ -298,6 +299,53 @@ NVFP4_API nvfp4_status nvfp4_mx_quantize(const void *x, nvfp4_dtype xt, int64_t 
  */
 NVFP4_API nvfp4_status nvfp4_mx_gemm(const nvfp4_mx_tensor *a, const nvfp4_mx_tensor *b, void *y, nvfp4_dtype yt,
                                      int64_t ldy, void *ws, size_t ws_bytes, nvfp4_stream_t stream);
+
+/*
+ * W4A8: FP4 weights times FP8 activations, the eefocus.com article's W4A8
+ * (the Zhouyi X3 passage: weights quantized to FP4, activations to FP8).  On
+ * B200 the native mixed FP4 x FP8 tensor-core product is block-scaled with one
+ * UE8M0 scale per 32 elements on both operands (kind::mxf8f6f4), so the
+ * weights are MXFP4 (nvfp4_mx_tensor) and the activations MXFP8:
+ *   scale   X = 2^e, e = ceil(log2(bamax / 448)) clamped to [-127, 127]: the
+ *           smallest power of two with bamax <= 448 X (an all-zero block gets
+ *           byte 0); the page gives no rule, this one never saturates.
+ *   element E4M3 (OCP "fn") RNE of x / X (exact division), sign kept.
+ * Layout: elements [rows][cols] one byte each, scales tiled as MXFP4's.
+ */
+typedef struct {
+    uint8_t *elems;                      /* [rows][cols] E4M3 bytes */
+    uint8_t *scales;                     /* nvfp4_mx_scales_bytes(rows, cols) bytes, tiled */
+    int64_t rows;
+    int64_t cols;                        /* a multiple of 32 */
+} nvfp4_mx8_tensor;
+
+/* Quantize x [rows][cols] (pitch ld, dtype xt; cols % 32 == 0) to MXFP8; one pass. */
+NVFP4_API nvfp4_status nvfp4_mx8_quantize(const void *x, nvfp4_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                                          const nvfp4_mx8_tensor *out, nvfp4_stream_t stream);
+
+/*
+ * y[M][N] = A . B^T with MXFP8 activations A [M][K] and MXFP4 weights B [N][K]
+ * (K % 128 == 0, else NVFP4_ERR_UNSUPPORTED_SHAPE: the copy that unpacks the
+ * weights into 8-bit shared-memory containers moves 128 values per row; the
+ * weights' codes 32-byte aligned, else NVFP4_ERR_MISALIGNED) on the block-scaled
+ * tensor cores (kind::mxf8f6f4, fp32 accumulation; no tensor scales).  Output
+ * dtypes, pitches and workspace (nvfp4_workspace_bytes(NVFP4_OP_GEMM, ...)) as
+ * nvfp4_gemm.
+ */
+NVFP4_API nvfp4_status nvfp4_w4a8_gemm(const nvfp4_mx8_tensor *a, const nvfp4_mx_tensor *b, void *y, nvfp4_dtype yt,
+                                       int64_t ldy, void *ws, size_t ws_bytes, nvfp4_stream_t stream);
+
+/*
+ * The W4A8 linear layer from high-precision activations: x [M][K] (pitch ldx,
+ * dtype xt) is quantized to MXFP8 on the device, then y = x_q . w^T as
+ * nvfp4_w4a8_gemm (same K and alignment rules).  If x_q is not NULL it
+ * receives the quantized activations.
+ * Workspace: nvfp4_workspace_bytes(NVFP4_OP_W4A8_LINEAR, M, N, K).
+ */
+NVFP4_API nvfp4_status nvfp4_w4a8_linear(const void *x, nvfp4_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                         const nvfp4_mx_tensor *w, void *y, nvfp4_dtype yt, int64_t ldy,
+                                         const nvfp4_mx8_tensor *x_q, void *ws, size_t ws_bytes,
+                                         nvfp4_stream_t stream);
 
 /*
  * W4A16 linear layer: y[M][N] = x . deq(w)^T with 16-bit activations x

@@ -26,7 +26,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_WORKSPACE, ERR_CUDA, \
     ERR_TIMEOUT, ERR_ARCH = range(8)
 F32, BF16 = 0, 1
-OP_QUANTIZE, OP_DEQUANTIZE, OP_GEMM, OP_LINEAR_FUSED, OP_LINEAR_FUSED_SILU, OP_GEMM_REQUANT, OP_W4A16 = range(7)
+OP_QUANTIZE, OP_DEQUANTIZE, OP_GEMM, OP_LINEAR_FUSED, OP_LINEAR_FUSED_SILU, OP_GEMM_REQUANT, OP_W4A16, \
+    OP_W4A8_LINEAR = range(8)
 EPI_STORE, EPI_SILU_MUL_REQUANT = 0, 1
 
 EXPORTED = (
@@ -34,7 +35,8 @@ EXPORTED = (
     "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_linear_fused", "nvfp4_get_device_status",
     "nvfp4_selftest_bounded_wait", "nvfp4_set_wait_timeout_us", "nvfp4_status_string",
     "nvfp4_version", "nvfp4_linear_noalloc", "nvfp4_gemm_requant", "nvfp4_mx_scales_bytes",
-    "nvfp4_mx_quantize", "nvfp4_mx_gemm", "nvfp4_w4a16_linear",
+    "nvfp4_mx_quantize", "nvfp4_mx_gemm", "nvfp4_w4a16_linear", "nvfp4_mx8_quantize", "nvfp4_w4a8_gemm",
+    "nvfp4_w4a8_linear",
 )
 
 
@@ -51,9 +53,16 @@ class CMXTensor(ctypes.Structure):
                 ("cols", ctypes.c_int64)]
 
 
+class CMX8Tensor(ctypes.Structure):
+    """``nvfp4_mx8_tensor`` of the C ABI."""
+    _fields_ = [("elems", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64)]
+
+
 _P, _I64, _SZ, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
 _T = ctypes.POINTER(CTensor)
 _TM = ctypes.POINTER(CMXTensor)
+_T8 = ctypes.POINTER(CMX8Tensor)
 
 _lib.nvfp4_codes_bytes.argtypes = [_I64, _I64]
 _lib.nvfp4_codes_bytes.restype = _SZ
@@ -77,6 +86,12 @@ _lib.nvfp4_mx_gemm.argtypes = [_TM, _TM, _P, _I, _I64, _P, _SZ, _P]
 _lib.nvfp4_mx_gemm.restype = _I
 _lib.nvfp4_w4a16_linear.argtypes = [_P, _I, _I64, _I64, _I64, _T, _P, _I, _I64, _P, _SZ, _P]
 _lib.nvfp4_w4a16_linear.restype = _I
+_lib.nvfp4_mx8_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _T8, _P]
+_lib.nvfp4_mx8_quantize.restype = _I
+_lib.nvfp4_w4a8_gemm.argtypes = [_T8, _TM, _P, _I, _I64, _P, _SZ, _P]
+_lib.nvfp4_w4a8_gemm.restype = _I
+_lib.nvfp4_w4a8_linear.argtypes = [_P, _I, _I64, _I64, _I64, _TM, _P, _I, _I64, _T8, _P, _SZ, _P]
+_lib.nvfp4_w4a8_linear.restype = _I
 _lib.nvfp4_linear_fused.argtypes = [_P, _I, _I64, _I64, _I64, _T, _T, _I, _P, _I, _I64, _T, _T,
                                     _P, _SZ, _P]
 _lib.nvfp4_linear_fused.restype = _I
@@ -188,6 +203,25 @@ class MXFP4Tensor:
         return CMXTensor(self.codes.data_ptr(), self.scales.data_ptr(), self.rows, self.cols)
 
 
+@dataclass
+class MXFP8Tensor:
+    """Device buffers of one MXFP8 tensor [rows][cols] (see ``nvfp4_mx8_tensor``)."""
+    elems: "object"          # uint8 [rows, cols] (E4M3 bytes)
+    scales: "object"         # uint8 [nvfp4_mx_scales_bytes]
+    rows: int
+    cols: int
+
+    @staticmethod
+    def empty(rows: int, cols: int, device="cuda") -> "MXFP8Tensor":
+        torch = _torch()
+        elems = torch.empty((rows, cols), dtype=torch.uint8, device=device)
+        scales = torch.empty(int(_lib.nvfp4_mx_scales_bytes(rows, cols)), dtype=torch.uint8, device=device)
+        return MXFP8Tensor(elems, scales, rows, cols)
+
+    def c(self) -> CMX8Tensor:
+        return CMX8Tensor(self.elems.data_ptr(), self.scales.data_ptr(), self.rows, self.cols)
+
+
 def _rows(*ts) -> None:
     """2-D tensors whose rows are contiguous (any row pitch): the layout the C
     ABI describes with a pointer and a row pitch.  A plain check, not an assert,
@@ -205,6 +239,13 @@ def _buffers(*qs) -> None:
     fp32 tensor scale), or the kernels would read or write past it."""
     for q in qs:
         if q is None:
+            continue
+        if isinstance(q, MXFP8Tensor):
+            for t, need, what in ((q.elems, q.rows * q.cols, "elems"), (q.scales, mx_scales_bytes(q.rows, q.cols), "scales")):
+                have = t.numel() * t.element_size()
+                if not t.is_contiguous() or have < need:
+                    raise ValueError(f"nvfp4: {what} of a {q.rows}x{q.cols} MXFP8 tensor needs {need} contiguous "
+                                     f"bytes; got {have} bytes")
             continue
         if isinstance(q, MXFP4Tensor):
             for t, need, what in ((q.codes, codes_bytes(q.rows, q.cols), "codes"),
@@ -246,7 +287,8 @@ def _on_device(*objs) -> None:
         if o is None:
             continue
         for t in ((o.codes, o.scales, o.tensor_scale) if isinstance(o, NVFP4Tensor) else
-                  (o.codes, o.scales) if isinstance(o, MXFP4Tensor) else (o,)):
+                  (o.codes, o.scales) if isinstance(o, MXFP4Tensor) else
+                  (o.elems, o.scales) if isinstance(o, MXFP8Tensor) else (o,)):
             if not t.is_cuda:
                 raise TypeError(f"nvfp4: got a tensor on {t.device}; the library needs CUDA tensors")
             if cur is None:
@@ -406,6 +448,47 @@ def nvfp4_w4a16_linear(x, w: NVFP4Tensor, y, ws, stream=None):
                                  y.data_ptr(), _dtype_code(y), y.stride(0), ws.data_ptr(), _ws_bytes(ws),
                                  _stream(stream))
     _check(st, "nvfp4_w4a16_linear")
+    return y
+
+
+def nvfp4_mx8_quantize(x, out: MXFP8Tensor, stream=None) -> MXFP8Tensor:
+    """Quantize a 2-D bf16/fp32 CUDA tensor to MXFP8 (E4M3 elements, E8M0 scales per 32) into out."""
+    _rows(x)
+    _buffers(out)
+    _on_device(x, out)
+    ct = out.c()
+    st = _lib.nvfp4_mx8_quantize(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], x.stride(0),
+                                 ctypes.byref(ct), _stream(stream))
+    _check(st, "nvfp4_mx8_quantize")
+    return out
+
+
+def nvfp4_w4a8_gemm(a: MXFP8Tensor, b: MXFP4Tensor, y, ws, stream=None):
+    """y[M][N] = a . b^T for MXFP8 activations and MXFP4 weights (workspace as OP_GEMM)."""
+    _rows(y)
+    _buffers(a, b)
+    _shape(y, a.rows, b.rows)
+    _on_device(a, b, y, ws)
+    ca, cb = a.c(), b.c()
+    st = _lib.nvfp4_w4a8_gemm(ctypes.byref(ca), ctypes.byref(cb), y.data_ptr(), _dtype_code(y), y.stride(0),
+                              ws.data_ptr(), _ws_bytes(ws), _stream(stream))
+    _check(st, "nvfp4_w4a8_gemm")
+    return y
+
+
+def nvfp4_w4a8_linear(x, w: MXFP4Tensor, y, ws, x_q: MXFP8Tensor | None = None, stream=None):
+    """W4A8 linear layer: quantize x to MXFP8 on the device, y = x_q . w^T."""
+    _rows(x, y)
+    _buffers(w, x_q)
+    _shape(y, x.shape[0], w.rows)
+    _on_device(x, w, y, ws, x_q)
+    cw = w.c()
+    cq = x_q.c() if x_q is not None else None
+    st = _lib.nvfp4_w4a8_linear(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], x.stride(0), ctypes.byref(cw),
+                                y.data_ptr(), _dtype_code(y), y.stride(0),
+                                ctypes.byref(cq) if cq is not None else None, ws.data_ptr(), _ws_bytes(ws),
+                                _stream(stream))
+    _check(st, "nvfp4_w4a8_linear")
     return y
 
 

@@ -125,6 +125,10 @@ size_t nvfp4_workspace_bytes(nvfp4_op op, int64_t M, int64_t N, int64_t K) {
         return kQuantizeWs + splitk_ws_bytes(M, N);
     case NVFP4_OP_W4A16:
         return kWsStatusBytes;
+    case NVFP4_OP_W4A8_LINEAR:
+        // status | x_q (E4M3 bytes, scales) | stream-K scratch
+        return kWsStatusBytes + align256(static_cast<size_t>(M * K)) + align256(nvfp4_mx_scales_bytes(M, K)) +
+               splitk_ws_bytes(M, N);
     }
     return 0;
 }
@@ -418,6 +422,115 @@ nvfp4_status nvfp4_mx_gemm(const nvfp4_mx_tensor *a, const nvfp4_mx_tensor *b, v
     Operand wgt{b->codes, b->scales, nullptr, b->rows};
     return from_cuda(launch_gemm_mx(act, wgt, a->cols, y, yt == NVFP4_BF16, ldy, static_cast<uint32_t *>(ws),
                                     wait_timeout_ns(), dev.sms, stream, sk ? ws_at(ws, kWsStatusBytes) : nullptr));
+}
+
+// ---------------------------------------------------------------------------
+// W4A8: MXFP8 activations x MXFP4 weights
+// ---------------------------------------------------------------------------
+
+static nvfp4_status check_mx8_tensor(const nvfp4_mx8_tensor *t, int64_t rows, int64_t cols) {
+    if (!t || t->rows != rows || t->cols != cols || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+    if (rows * cols != 0 && (!t->elems || !t->scales)) return NVFP4_ERR_INVALID_ARG;
+    if (cols % 32) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(t->elems) || !aligned16(t->scales)) return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_mx8_quantize(const void *x, nvfp4_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                                const nvfp4_mx8_tensor *out, nvfp4_stream_t stream) {
+    if ((!x && rows * cols != 0) || (xt != NVFP4_F32 && xt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_mx8_tensor(out, rows, cols);
+    if (st != NVFP4_OK) return st;
+    const int eb = xt == NVFP4_BF16 ? 2 : 4;
+    if (rows * cols != 0 && (!aligned16(x) || (ld * eb) % 16)) return NVFP4_ERR_MISALIGNED;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    return from_cuda(launch_mx8_quantize(x, xt == NVFP4_BF16, rows, cols, ld, out->elems, out->scales, dev.sms,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// The weights' codes are read by a copy that unpacks them into 8-bit
+// containers: it moves 128 values of K per row and needs a row length that is
+// a multiple of 128 values and a 32-byte aligned start.
+static nvfp4_status check_w4a8_weights(const nvfp4_mx_tensor *w, int64_t K) {
+    nvfp4_status st = check_mx_tensor(w, w ? w->rows : 0, K);
+    if (st != NVFP4_OK) return st;
+    if (K % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (w->rows * K != 0 && (reinterpret_cast<uintptr_t>(w->codes) & 31u)) return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+static nvfp4_status w4a8_gemm_impl(const nvfp4_mx8_tensor *a, const nvfp4_mx_tensor *b, void *y, nvfp4_dtype yt,
+                                   int64_t ldy, uint32_t *status, int sms, cudaStream_t stream, bool weights_ready,
+                                   void *splitk) {
+    const int eb = yt == NVFP4_BF16 ? 2 : 4;
+    if (a->rows == 0 || b->rows == 0) return NVFP4_OK;
+    if (a->cols == 0) return from_cuda(cudaMemset2DAsync(y, ldy * eb, 0, b->rows * eb, a->rows, stream));
+    Operand act{a->elems, a->scales, nullptr, a->rows};
+    Operand wgt{b->codes, b->scales, nullptr, b->rows};
+    return from_cuda(launch_gemm_w4a8(act, wgt, a->cols, y, yt == NVFP4_BF16, ldy, status, wait_timeout_ns(), sms,
+                                      stream, weights_ready, splitk));
+}
+
+nvfp4_status nvfp4_w4a8_gemm(const nvfp4_mx8_tensor *a, const nvfp4_mx_tensor *b, void *y, nvfp4_dtype yt,
+                             int64_t ldy, void *ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!a || !b || (yt != NVFP4_F32 && yt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if (!y && a->rows * b->rows != 0) return NVFP4_ERR_INVALID_ARG;
+    if (a->cols != b->cols) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_mx8_tensor(a, a->rows, a->cols);
+    if (st != NVFP4_OK) return st;
+    if ((st = check_w4a8_weights(b, a->cols)) != NVFP4_OK) return st;
+    if (a->rows > kMaxGemmRows || b->rows > kMaxGemmRows || a->cols > kMaxGemmK) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ldy < b->rows) return NVFP4_ERR_INVALID_ARG;
+    const int eb = yt == NVFP4_BF16 ? 2 : 4;
+    if (a->rows * b->rows != 0 && (!aligned16(y) || (ldy * eb) % 16)) return NVFP4_ERR_MISALIGNED;
+    const size_t sk = splitk_ws_bytes(a->rows, b->rows);
+    if ((st = check_ws(ws, ws_bytes, kWsStatusBytes + sk)) != NVFP4_OK) return st;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    return w4a8_gemm_impl(a, b, y, yt, ldy, static_cast<uint32_t *>(ws), dev.sms,
+                          reinterpret_cast<cudaStream_t>(stream), false, sk ? ws_at(ws, kWsStatusBytes) : nullptr);
+}
+
+nvfp4_status nvfp4_w4a8_linear(const void *x, nvfp4_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                               const nvfp4_mx_tensor *w, void *y, nvfp4_dtype yt, int64_t ldy,
+                               const nvfp4_mx8_tensor *x_q, void *ws, size_t ws_bytes, nvfp4_stream_t stream_) {
+    if ((!x && M * K != 0) || !w || (xt != NVFP4_F32 && xt != NVFP4_BF16) || (yt != NVFP4_F32 && yt != NVFP4_BF16))
+        return NVFP4_ERR_INVALID_ARG;
+    if (M < 0 || K < 0 || ldx < K) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_w4a8_weights(w, K);
+    if (st != NVFP4_OK) return st;
+    const int64_t N = w->rows;
+    if (M > kMaxGemmRows || N > kMaxGemmRows || K > kMaxGemmK) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if ((!y && M * N != 0) || ldy < N) return NVFP4_ERR_INVALID_ARG;
+    const int xeb = xt == NVFP4_BF16 ? 2 : 4, yeb = yt == NVFP4_BF16 ? 2 : 4;
+    if ((M * K != 0 && (!aligned16(x) || (ldx * xeb) % 16)) || (M * N != 0 && (!aligned16(y) || (ldy * yeb) % 16)))
+        return NVFP4_ERR_MISALIGNED;
+    if (x_q && (st = check_mx8_tensor(x_q, M, K)) != NVFP4_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, nvfp4_workspace_bytes(NVFP4_OP_W4A8_LINEAR, M, N, K))) != NVFP4_OK) return st;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (M == 0) return NVFP4_OK;
+    nvfp4_mx8_tensor xq;
+    size_t off = kWsStatusBytes;
+    if (x_q) {
+        xq = *x_q;
+    } else {
+        xq.elems = ws_at(ws, off);
+        off += align256(static_cast<size_t>(M * K));
+        xq.scales = ws_at(ws, off);
+        xq.rows = M;
+        xq.cols = K;
+    }
+    off = kWsStatusBytes + align256(static_cast<size_t>(M * K)) + align256(nvfp4_mx_scales_bytes(M, K));
+    if (launch_mx8_quantize(x, xt == NVFP4_BF16, M, K, ldx, xq.elems, xq.scales, dev.sms, stream) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    // the quantizer is launched without a programmatic dependency, so the
+    // weights' earlier writers have finished: the GEMM may stream them early
+    return w4a8_gemm_impl(&xq, w, y, yt, ldy, static_cast<uint32_t *>(ws), dev.sms, stream, true,
+                          splitk_ws_bytes(M, N) != 0 ? ws_at(ws, off) : nullptr);
 }
 
 // ---------------------------------------------------------------------------

@@ -110,7 +110,11 @@ struct SegIter {
     }
 };
 
-template <int BN>
+// NACC accumulators per tile: K step j of a stage accumulates into
+// accumulator j % NACC, so that consecutive MMAs do not wait for one another
+// (with few output columns an MMA takes far less time than the latency of the
+// previous one into the same accumulator); the epilogue adds them in order.
+template <int BN, int NACC = 1>
 struct GemmCfg {
     static constexpr int kNQT = (BN + 127) / 128;              // 128-row scale tiles per B tile
     static constexpr int kAStage = 128 * 128;                  // bytes of A per stage
@@ -120,8 +124,9 @@ struct GemmCfg {
     static constexpr int kStageBytes = kAStage + kBStage + kSfaStage + kSfbStage;
     static constexpr int kStages = (BN == 256) ? 4 : (BN == 128 ? 6 : (BN == 64 ? 7 : 8));
     static constexpr int kSfCols = 16 + 16 * kNQT;             // TMEM scale columns per stage
-    static constexpr int kAccStages = (2 * BN + kStages * kSfCols <= 512) ? 2 : 1;
-    static constexpr int kSfBase = kAccStages * BN;            // first scale column
+    static constexpr int kAccCols = NACC * BN;                 // columns of one tile's accumulators
+    static constexpr int kAccStages = (2 * kAccCols + kStages * kSfCols <= 512) ? 2 : 1;
+    static constexpr int kSfBase = kAccStages * kAccCols;      // first scale column
     static constexpr int kColsUsed = kSfBase + kStages * kSfCols;
     static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
@@ -131,37 +136,82 @@ struct GemmCfg {
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kColsUsed <= 512, "tensor memory budget");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+    static_assert(NACC == 1 || NACC == 4, "one accumulator, or one per K step of a stage");
 };
 
-// Scale atoms per 256-deep K stage and per 128-row tile: NVFP4 has one
-// 512-byte atom (4 blocks of 16) per K step of 64; MXFP4 one per two K steps
-// (4 blocks of 32), so a stage holds 4 or 2 atoms.
-template <bool MX> struct ScaleFmt {
-    static constexpr int kAtomsPerStage = MX ? 2 : 4;
-    __host__ __device__ static int atoms_per_row_tile(int k_steps) { return MX ? (k_steps + 1) / 2 : k_steps; }
-    __host__ __device__ static int stage_atoms(int nk) { return MX ? (nk + 1) / 2 : nk; }
-};
+// Swapped tiles (few activation rows on the MMA's N) use four accumulators.
+template <bool SWAP> constexpr int kNumAcc = SWAP ? 4 : 1;
 
-// The block-scaled MMAs of K step j of a stage: NVFP4 reads the stage's
-// scale columns 4j (A) and 4*NQT*j past the A columns (B); MXFP4 reads the
-// columns of atom j/2 and picks their bytes {0,1} or {2,3} by the descriptor.
-template <bool MX, int BN, int NQT>
-__device__ __forceinline__ void mma_kstep(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t sf, int j,
-                                          uint32_t acc) {
-    if constexpr (MX) {
-        const uint32_t idesc = (j & 1) ? make_idesc_mxf4(BN, 128, 1) : make_idesc_mxf4(BN, 128, 0);
-        mma_mxf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * (j >> 1), sf + 16 + 4 * NQT * (j >> 1), acc);
-    } else {
-        mma_nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, make_idesc_nvf4(BN), sf + 4 * j, sf + 16 + 4 * NQT * j, acc);
+// Accumulator columns [taddr, taddr + CH) of a tile, the NACC accumulators
+// (nvalid of them written) added in order ((a0 + a1) + a2) + a3.  Warp-uniform
+// nvalid (tcgen05.ld is .sync.aligned).
+template <int CH, int NACC, int STRIDE>
+__device__ __forceinline__ void tmem_ld_acc(uint32_t taddr, int nvalid, uint32_t (&r)[CH]) {
+    auto ld = [&](uint32_t a, uint32_t (&dst)[CH]) {
+        if constexpr (CH == 32) tmem_ld_32x32b_x32(a, reinterpret_cast<uint32_t(&)[32]>(dst));
+        else tmem_ld_32x32b_x16(a, reinterpret_cast<uint32_t(&)[16]>(dst));
+    };
+    ld(taddr, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int s = 1; s < NACC; ++s) {
+        if (s < nvalid) {
+            uint32_t t[CH];
+            ld(taddr + s * STRIDE, t);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < CH; ++i) r[i] = __float_as_uint(__fadd_rn(__uint_as_float(r[i]), __uint_as_float(t[i])));
+        }
     }
 }
 
-template <int BN, bool SWAP, typename OutT, bool MX>
+// Operand formats of the one-CTA kernel.
+constexpr int kFmtNV = 0;     // NVFP4: E2M1 (packed), UE4M3 per 16, kind::mxf4nvf4 4X, K = 64 per MMA
+constexpr int kFmtMX = 1;     // MXFP4: E2M1 (packed), UE8M0 per 32, kind::mxf4 2X, K = 64 per MMA
+constexpr int kFmtW4A8 = 2;   // MXFP4 weights x MXFP8 activations (8-bit containers in shared memory),
+                              // UE8M0 per 32, kind::mxf8f6f4 1X, K = 32 per MMA
+
+// Scale atoms (512 bytes: 128 rows x 4 blocks) per ring stage and per 128-row
+// tile.  A stage is four MMA K steps: 256 values of K for the FP4 kinds, 128
+// for W4A8, and always 128 bytes per operand row in shared memory.  NVFP4 has
+// one atom per K step (4 blocks of 16), MXFP4 one per two (4 blocks of 32),
+// W4A8 one per four.
+template <int FMT> struct ScaleFmt {
+    static constexpr int kAtomsPerStage = FMT == kFmtNV ? 4 : (FMT == kFmtMX ? 2 : 1);
+    static constexpr int kStepsPerAtom = 4 / kAtomsPerStage;              // MMA K steps one atom covers
+    __host__ __device__ static int atoms_per_row_tile(int k_steps) { return (k_steps + kStepsPerAtom - 1) / kStepsPerAtom; }
+    __host__ __device__ static int stage_atoms(int nk) { return (nk + kStepsPerAtom - 1) / kStepsPerAtom; }
+};
+
+// The block-scaled MMAs of K step j of a stage.  NVFP4 reads the stage's
+// scale columns 4j (A) and 4*NQT*j past the A columns (B); MXFP4 reads the
+// columns of atom j/2 and picks their bytes {0,1} or {2,3} by the
+// descriptor; W4A8 reads atom 0's columns and picks byte j.
+template <int FMT, int BN, int NQT, bool SWAP>
+__device__ __forceinline__ void mma_kstep(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t sf, int j,
+                                          uint32_t acc, uint32_t issue) {
+    if constexpr (FMT == kFmtW4A8) {
+        // the weights are E2M1 (format 5), the activations E4M3 (format 0)
+        constexpr uint32_t fa = SWAP ? 5u : 0u, fb = SWAP ? 0u : 5u;
+        const uint32_t idesc = make_idesc_mxf8f6f4(BN, fa, fb, static_cast<uint32_t>(j));
+        mma_mxf8f6f4(d_tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf, sf + 16, acc, issue);
+    } else if constexpr (FMT == kFmtMX) {
+        const uint32_t idesc = (j & 1) ? make_idesc_mxf4(BN, 128, 1) : make_idesc_mxf4(BN, 128, 0);
+        mma_mxf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * (j >> 1), sf + 16 + 4 * NQT * (j >> 1), acc,
+                 issue);
+    } else {
+        mma_nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, make_idesc_nvf4(BN), sf + 4 * j, sf + 16 + 4 * NQT * j, acc,
+                 issue);
+    }
+}
+
+template <int BN, bool SWAP, typename OutT, int FMT>
 __global__ void __launch_bounds__(448, 1)
 gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ GemmArgs args) {
-    using C = GemmCfg<BN>;
-    using F = ScaleFmt<MX>;
+    constexpr int NACC = kNumAcc<SWAP>;
+    using C = GemmCfg<BN, NACC>;
+    using F = ScaleFmt<FMT>;
     constexpr int STAGES = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -211,10 +261,18 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
     const int num_tiles = args.num_p_tiles * args.num_q_tiles;
     const int num_kstages = (args.num_k_steps + 3) / 4;
+    // Bytes the operand copies of one stage signal on its barrier.  The
+    // unpacking copy of the W4A8 weights counts the packed bytes it reads
+    // (64 per row), not the 128 it writes.
+    constexpr uint32_t kOperandTxBytes =
+        FMT != kFmtW4A8 ? C::kAStage + C::kBStage : (SWAP ? C::kAStage / 2 + C::kBStage : C::kAStage + C::kBStage / 2);
 
     if (warp == 0) {
-        if (lane == 0) {
+        {
             // -------------------------------------------------------- producer
+            // The whole warp walks the loop (its waits are warp-uniform); one
+            // elected lane issues the copies.
+            const bool issue = elect_one_sync();
             const uint64_t pol_a = SWAP ? policy_evict_first() : policy_evict_normal();
             const uint64_t pol_b = SWAP ? policy_evict_last() : policy_evict_normal();
             // The weights may be streamed before the dependent-launch wait for
@@ -248,12 +306,13 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             auto finish_preload = [&]() {
                 asm volatile("griddepcontrol.wait;" ::: "memory");
                 waited = true;
-                for (int p = 0; p < pre; ++p) {
+                for (int p = 0; p < pre && issue; ++p) {
                     const int ks = first.ks0 + p;
                     const int nk = min(4, args.num_k_steps - 4 * ks);
                     if (args.weights_are_a) load_b(static_cast<uint32_t>(p), qt0, ks, nk);
                     else load_a(static_cast<uint32_t>(p), pt0, ks, nk);
                 }
+                __syncwarp();
             };
             uint32_t stage = 0, phase = 0;
             int it = 0;   // stage index within this CTA's work
@@ -267,22 +326,28 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 for (int q = 0; q < C::kNQT; ++q) nq_loaded += (qt * C::kNQT + q < args.q_row_tiles);
                 for (int ks = sg.ks0; ks < sg.ks1; ++ks, ++it) {
                     const int nk = min(4, args.num_k_steps - 4 * ks);
-                    const uint32_t bytes = C::kAStage + C::kBStage + F::stage_atoms(nk) * 512 * (1 + nq_loaded);
+                    const uint32_t bytes = kOperandTxBytes + F::stage_atoms(nk) * 512 * (1 + nq_loaded);
                     if (it < pre) {
                         // fresh stage (first pass over the ring): no empty wait needed
-                        mbar_arrive_expect_tx(&full[stage], bytes);
-                        if (args.weights_are_a) load_a(stage, pt, ks, nk);
-                        else load_b(stage, qt, ks, nk);
+                        if (issue) {
+                            mbar_arrive_expect_tx(&full[stage], bytes);
+                            if (args.weights_are_a) load_a(stage, pt, ks, nk);
+                            else load_b(stage, qt, ks, nk);
+                        }
                     } else {
                         if (!waited) finish_preload();
-                        if (!mbar_wait(&empty[stage], phase ^ 1u, args.timeout_ns, abort_flag, args.status)) {
+                        if (!__all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1u, args.timeout_ns,
+                                                               abort_flag, args.status))) {
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(&full[stage], bytes);
-                        load_a(stage, pt, ks, nk);
-                        load_b(stage, qt, ks, nk);
+                        if (issue) {
+                            mbar_arrive_expect_tx(&full[stage], bytes);
+                            load_a(stage, pt, ks, nk);
+                            load_b(stage, qt, ks, nk);
+                        }
                     }
+                    __syncwarp();
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
@@ -296,20 +361,26 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                           &keep_waiting, args.status);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        {
             // -------------------------------------------------------- MMA issuer
+            // The whole warp walks the loop; one elected lane issues the MMAs
+            // and commits.
+            const uint32_t issue = elect_one_sync() ? 1u : 0u;
             const uint32_t a_base = smem_addr(sA), b_base = smem_addr(sB);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             SegIter segs(args, num_tiles, num_kstages);
             Seg sg;
             while (segs.next(sg)) {
-                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.timeout_ns, abort_flag, args.status)) break;
+                if (!__all_sync(0xffffffffu, mbar_wait(&tempty[acc], acc_phase ^ 1u, args.timeout_ns, abort_flag,
+                                                       args.status)))
+                    break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * BN;
+                const uint32_t d_tmem = tmem_base + acc * C::kAccCols;
                 bool ok = true;
                 for (int ks = sg.ks0; ks < sg.ks1; ++ks) {
-                    if (!mbar_wait(&full[stage], phase, args.timeout_ns, abort_flag, args.status) ||
-                        !mbar_wait(&sf_full[stage], phase, args.timeout_ns, abort_flag, args.status)) {
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait(&full[stage], phase, args.timeout_ns, abort_flag, args.status) &&
+                                    mbar_wait(&sf_full[stage], phase, args.timeout_ns, abort_flag, args.status))) {
                         ok = false;
                         break;
                     }
@@ -320,19 +391,22 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage);
                     const uint64_t bdesc = make_operand_desc(b_base + stage * C::kBStage);
                     const uint32_t acc0 = ks != sg.ks0 ? 1u : 0u;
+                    // K step j -> accumulator j % NACC; its first MMA of the
+                    // tile overwrites it
+                    auto accf = [&](int j) -> uint32_t { return NACC == 1 ? ((acc0 | j) != 0 ? 1u : 0u) : acc0; };
                     if (nk == 4) {
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
-                            mma_kstep<MX, BN, C::kNQT>(d_tmem, adesc, bdesc, sf, j, (acc0 | j) != 0 ? 1u : 0u);
+                            mma_kstep<FMT, BN, C::kNQT, SWAP>(d_tmem + (j % NACC) * BN, adesc, bdesc, sf, j, accf(j), issue);
                     } else {
                         for (int j = 0; j < nk; ++j)
-                            mma_kstep<MX, BN, C::kNQT>(d_tmem, adesc, bdesc, sf, j, (acc0 | j) != 0 ? 1u : 0u);
+                            mma_kstep<FMT, BN, C::kNQT, SWAP>(d_tmem + (j % NACC) * BN, adesc, bdesc, sf, j, accf(j), issue);
                     }
-                    tc_commit(&empty[stage]);
+                    tc_commit(&empty[stage], issue);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                tc_commit(&tfull[acc]);
+                tc_commit(&tfull[acc], issue);
                 if (C::kAccStages == 2) {
                     acc ^= 1u;
                     if (acc == 0) acc_phase ^= 1u;
@@ -340,9 +414,9 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     acc_phase ^= 1u;
                 }
             }
-            // Tensor memory is freed below: first let every MMA this thread
+            // Tensor memory is freed below: first let every MMA this warp
             // issued complete (bounded, also after an abort).
-            tc_commit(mma_done);
+            tc_commit(mma_done, issue);
             volatile uint32_t keep_waiting = 0u;
             mbar_wait(mma_done, 0, args.timeout_ns, &keep_waiting, args.status);
         }
@@ -430,7 +504,9 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const int p = pt * 128 + row;
-            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::kAccCols;
+            // accumulators this work item wrote: one per K step it has, at most NACC
+            const int nvalid = min(NACC, min(4 * sg.ks1, args.num_k_steps) - 4 * sg.ks0);
             // (stream-K is never chosen for 256-wide tiles; keep that path out of them)
             const bool partial = BN <= 128 && (sg.ks0 != 0 || sg.ks1 != num_kstages);
             if (partial) {
@@ -446,11 +522,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
                     for (int c = 0; c < WC / CH; ++c) {
                         uint32_t r[CH];
-                        if constexpr (CH == 32)
-                            tmem_ld_32x32b_x32(tbase + c0 + c * CH, reinterpret_cast<uint32_t(&)[32]>(r));
-                        else
-                            tmem_ld_32x32b_x16(tbase + c0 + c * CH, reinterpret_cast<uint32_t(&)[16]>(r));
-                        tmem_ld_wait();
+                        tmem_ld_acc<CH, NACC, BN>(tbase + c0 + c * CH, nvalid, r);
 #pragma unroll
                         for (int i = 0; i < CH; i += 4)
                             red_add_v4_f32(accrow + c * CH + i, __uint_as_float(r[i]), __uint_as_float(r[i + 1]),
@@ -617,11 +689,16 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         else
                             tmem_ld_32x32b_x16(tbase + c * CH, reinterpret_cast<uint32_t(&)[16]>(dst));
                     };
-                    ld(0, r[0]);
-                    tmem_ld_wait();
+                    if constexpr (NACC == 1) {
+                        ld(0, r[0]);
+                        tmem_ld_wait();
+                    }
 #pragma unroll
                     for (int c = 0; c < NCH; ++c) {
-                        if (c + 1 < NCH) ld(c + 1, r[(c + 1) & 1]);       // next chunk in flight
+                        if constexpr (NACC > 1)
+                            tmem_ld_acc<CH, NACC, BN>(tbase + c * CH, nvalid, r[c & 1]);   // summed, not prefetched
+                        else if (c + 1 < NCH)
+                            ld(c + 1, r[(c + 1) & 1]);       // next chunk in flight
                         float v[CH];
 #pragma unroll
                         for (int i = 0; i < CH; ++i) v[i] = __fmul_rn(__uint_as_float(r[c & 1][i]), alpha);
@@ -679,7 +756,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                                 }
                             }
                         }
-                        if (c + 1 < NCH) tmem_ld_wait();
+                        if (NACC == 1 && c + 1 < NCH) tmem_ld_wait();
                     }
                 }
                 tc_fence_before();
@@ -750,6 +827,23 @@ CUresult encode_tensor_map_u8(CUtensorMap *map, const void *base, uint64_t inner
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+CUresult encode_tensor_map_fp4_unpacked(CUtensorMap *map, const void *base, uint64_t k_elems, uint64_t rows,
+                                        uint32_t box_rows) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return CUDA_ERROR_NOT_FOUND;
+    // packed E2M1 rows of k_elems values (k_elems / 2 bytes apart); each box
+    // of 128 values x box_rows rows lands as 128-byte rows in shared memory,
+    // 16 values per 16-byte chunk (8 bytes of values, 8 bytes of gap), the
+    // operand form of the mixed FP4 x FP8 MMA
+    cuuint64_t dims[2] = {k_elems, rows};
+    cuuint64_t strides[1] = {k_elems / 2};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 CUresult encode_scale_map(CUtensorMap *map, const void *scales, uint64_t k_steps, uint64_t row_tiles,
                           uint32_t box_tiles, uint32_t box_atoms) {
     EncodeTiledFn fn = get_encode_fn();
@@ -806,16 +900,27 @@ static SplitKLayout splitk_layout(int64_t M, int64_t N) {
 
 size_t splitk_ws_bytes(int64_t M, int64_t N) { return splitk_layout(M, N).bytes; }
 
-template <int BN, bool SWAP, typename OutT, bool MX>
+template <int BN, bool SWAP, typename OutT, int FMT>
 static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, void *y, int64_t ldy,
                             uint32_t *status, uint64_t timeout_ns, int num_sms, int preload,
                             uint8_t *splitk_ws, const SplitKLayout &skl, float *ymax_part, int *nparts,
                             cudaStream_t stream) {
-    using C = GemmCfg<BN>;
+    using C = GemmCfg<BN, kNumAcc<SWAP>>;
     CUtensorMap tmA, tmB;
-    if (encode_tensor_map_u8(&tmA, pa.codes, K / 2, pa.rows, 128, 128) != CUDA_SUCCESS ||
-        encode_tensor_map_u8(&tmB, qb.codes, K / 2, qb.rows, 128, BN) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
+    if constexpr (FMT == kFmtW4A8) {
+        // 128 values of K per 128-byte shared-memory row: the MXFP4 weights
+        // unpacked by the copy into 8-bit containers, the E4M3 activations as
+        // they are
+        const Operand &w = SWAP ? pa : qb, &x = SWAP ? qb : pa;
+        CUtensorMap &tw = SWAP ? tmA : tmB, &tx = SWAP ? tmB : tmA;
+        if (encode_tensor_map_fp4_unpacked(&tw, w.codes, K, w.rows, SWAP ? 128 : BN) != CUDA_SUCCESS ||
+            encode_tensor_map_u8(&tx, x.codes, K, x.rows, 128, SWAP ? BN : 128) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    } else {
+        if (encode_tensor_map_u8(&tmA, pa.codes, K / 2, pa.rows, 128, 128) != CUDA_SUCCESS ||
+            encode_tensor_map_u8(&tmB, qb.codes, K / 2, qb.rows, 128, BN) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
     GemmArgs a;
     a.sfa = pa.scales;
     a.sfb = qb.scales;
@@ -825,7 +930,7 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     a.ldy = ldy;
     a.P = static_cast<int32_t>(pa.rows);
     a.Q = static_cast<int32_t>(qb.rows);
-    a.num_k_steps = static_cast<int32_t>(K / 64);
+    a.num_k_steps = static_cast<int32_t>(FMT == kFmtW4A8 ? K / 32 : K / 64);   // MMA K steps
     a.num_p_tiles = static_cast<int32_t>(ceil_div(pa.rows, 128));
     a.num_q_tiles = static_cast<int32_t>(ceil_div(qb.rows, BN));
     a.q_row_tiles = static_cast<int32_t>(ceil_div(qb.rows, 128));
@@ -850,7 +955,7 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     a.q_pad = a.num_q_tiles * BN;
     a.acc_ws = sk ? reinterpret_cast<float *>(splitk_ws) : nullptr;
     a.tile_cnt = sk ? reinterpret_cast<int32_t *>(splitk_ws + skl.acc_bytes) : nullptr;
-    auto kern = gemm_nvf4_kernel<BN, SWAP, OutT, MX>;
+    auto kern = gemm_nvf4_kernel<BN, SWAP, OutT, FMT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // The stream-K scratch is zero-filled for every call, so it may share a
@@ -871,7 +976,7 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
 }
 
-template <bool MX>
+template <int FMT>
 static cudaError_t launch_gemm_fmt(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
                                    int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
                                    cudaStream_t stream, bool weights_ready, void *splitk_ws, float *ymax_part,
@@ -886,37 +991,45 @@ static cudaError_t launch_gemm_fmt(const Operand &act, const Operand &wgt, int64
         // weights on the MMA's M side, activations on N; y[m][n] = acc[n][m]
         const int bn = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
 #define NVFP4_SWAPPED(BNV)                                                                          \
-    return y_bf16 ? run_gemm<BNV, true, __nv_bfloat16, MX>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream) \
-                  : run_gemm<BNV, true, float, MX>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream);
+    return y_bf16 ? run_gemm<BNV, true, __nv_bfloat16, FMT>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream) \
+                  : run_gemm<BNV, true, float, FMT>(wgt, act, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream);
         if (bn == 16) { NVFP4_SWAPPED(16) }
         if (bn == 32) { NVFP4_SWAPPED(32) }
         NVFP4_SWAPPED(64)
 #undef NVFP4_SWAPPED
     }
-    if (pair_gemm_usable(M, N, num_sms))
-        return launch_gemm_pair(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, stream, ymax_part, nparts, MX);
+    if (FMT != kFmtW4A8 && pair_gemm_usable(M, N, num_sms))
+        return launch_gemm_pair(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, stream, ymax_part, nparts,
+                                FMT == kFmtMX);
     const int64_t ptiles = ceil_div(M, 128);
     const bool wide = ptiles * ceil_div(N, 256) >= 2 * num_sms;
     if (wide)
-        return y_bf16 ? run_gemm<256, false, __nv_bfloat16, MX>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream)
-                      : run_gemm<256, false, float, MX>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream);
-    return y_bf16 ? run_gemm<128, false, __nv_bfloat16, MX>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream)
-                  : run_gemm<128, false, float, MX>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream);
+        return y_bf16 ? run_gemm<256, false, __nv_bfloat16, FMT>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream)
+                      : run_gemm<256, false, float, FMT>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream);
+    return y_bf16 ? run_gemm<128, false, __nv_bfloat16, FMT>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream)
+                  : run_gemm<128, false, float, FMT>(act, wgt, K, y, ldy, status, timeout_ns, num_sms, preload, skw, skl, ymax_part, nparts, stream);
 }
 
 cudaError_t launch_gemm(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
                         int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
                         cudaStream_t stream, bool weights_ready, void *splitk_ws, float *ymax_part,
                         int *nparts) {
-    return launch_gemm_fmt<false>(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, num_sms, stream, weights_ready,
+    return launch_gemm_fmt<kFmtNV>(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, num_sms, stream, weights_ready,
                                   splitk_ws, ymax_part, nparts);
 }
 
 cudaError_t launch_gemm_mx(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
                            int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
                            cudaStream_t stream, void *splitk_ws) {
-    return launch_gemm_fmt<true>(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, num_sms, stream, false,
-                                 splitk_ws, nullptr, nullptr);
+    return launch_gemm_fmt<kFmtMX>(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, num_sms, stream, false,
+                                   splitk_ws, nullptr, nullptr);
+}
+
+cudaError_t launch_gemm_w4a8(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
+                             int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
+                             cudaStream_t stream, bool weights_ready, void *splitk_ws) {
+    return launch_gemm_fmt<kFmtW4A8>(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, num_sms, stream,
+                                     weights_ready, splitk_ws, nullptr, nullptr);
 }
 
 // ---------------------------------------------------------------------------

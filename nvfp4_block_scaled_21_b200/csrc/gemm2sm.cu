@@ -181,8 +181,11 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     const int num_groups = (num_kstages + 1) / 2;
 
     if (warp == 0) {
-        if (lane == 0) {
+        {
             // -------------------------------------------------------- producer
+            // The whole warp walks the loop (its waits are warp-uniform); one
+            // elected lane issues the copies.
+            const bool issue = elect_one_sync();
             asm volatile("griddepcontrol.wait;" ::: "memory");
             const uint64_t pol = policy_evict_normal();
             const uint32_t leader_full0 = mapa_shared(smem_addr(&full[0]), 0);
@@ -195,18 +198,24 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                 const int b_rt = 2 * qn + static_cast<int>(rank);   // this CTA's half of B
                 bool ok = true;
                 for (int ks = 0; ks < num_kstages; ++ks) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, args.timeout_ns, abort_flag, args.status)) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1u, args.timeout_ns, abort_flag,
+                                                           args.status))) {
                         ok = false;
                         break;
                     }
                     const uint32_t bar = leader_full0 + 8u * stage;
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kABBytes);
-                    tma_load_2d_pair(sA + stage * C::kAStage, &tmA, bar, ks * 128, a_rt * 128, pol);
-                    tma_load_2d_pair(sB + stage * C::kBStage, &tmB, bar, ks * 128, b_rt * 128, pol);
-                    // scale atoms of this stage: 4 (NVFP4) or 2 (MXFP4) per 128-row tile
-                    mbar_arrive_expect_tx(&sfull[stage], MX ? C::kSfBytes / 2 : C::kSfBytes);
-                    tma_load_3d(sSfa + stage * C::kSfaStage, &tmSA, &sfull[stage], 0, (MX ? 2 : 4) * ks, a_rt, pol);
-                    tma_load_3d(sSfb + stage * C::kSfbStage, &tmSB, &sfull[stage], 0, (MX ? 2 : 4) * ks, 2 * qn, pol);
+                    if (issue) {
+                        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kABBytes);
+                        tma_load_2d_pair(sA + stage * C::kAStage, &tmA, bar, ks * 128, a_rt * 128, pol);
+                        tma_load_2d_pair(sB + stage * C::kBStage, &tmB, bar, ks * 128, b_rt * 128, pol);
+                        // scale atoms of this stage: 4 (NVFP4) or 2 (MXFP4) per 128-row tile
+                        mbar_arrive_expect_tx(&sfull[stage], MX ? C::kSfBytes / 2 : C::kSfBytes);
+                        tma_load_3d(sSfa + stage * C::kSfaStage, &tmSA, &sfull[stage], 0, (MX ? 2 : 4) * ks, a_rt,
+                                    pol);
+                        tma_load_3d(sSfb + stage * C::kSfbStage, &tmSB, &sfull[stage], 0, (MX ? 2 : 4) * ks, 2 * qn,
+                                    pol);
+                    }
+                    __syncwarp();
                     ++issued;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -224,8 +233,11 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             }
         }
     } else if (warp == 1) {
-        if (lane == 0 && leader) {
+        if (leader) {
             // -------------------------------------------------------- MMA issuer
+            // The whole warp walks the loop; one elected lane issues the MMAs
+            // and commits.
+            const uint32_t issue = elect_one_sync() ? 1u : 0u;
             constexpr uint32_t idesc = make_idesc_nvf4_pair(256);
             constexpr uint32_t idesc_mx0 = make_idesc_mxf4(256, 256, 0), idesc_mx1 = make_idesc_mxf4(256, 256, 1);
             const uint32_t a_base = smem_addr(sA), b_base = smem_addr(sB);
@@ -235,14 +247,14 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             bool ok = true;
             for (int tile = cid; tile < num_tiles && ok; tile += ncl, ++t) {
                 // the previous tile's accumulator has been read out of TMEM
-                if (t > 0 && !mbar_wait(tempty, static_cast<uint32_t>(t - 1) & 1u, args.timeout_ns,
-                                                abort_flag, args.status))
+                if (t > 0 && !__all_sync(0xffffffffu, mbar_wait(tempty, static_cast<uint32_t>(t - 1) & 1u,
+                                                                 args.timeout_ns, abort_flag, args.status)))
                     break;
                 tc_fence_after();
                 for (int g = 0; g < num_groups && ok; ++g, ++gcount) {
                     const uint32_t slot = gcount & 1u;
-                    if (!mbar_wait(&sf_ready[slot], (gcount >> 1) & 1u, args.timeout_ns, abort_flag,
-                                           args.status)) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&sf_ready[slot], (gcount >> 1) & 1u, args.timeout_ns,
+                                                           abort_flag, args.status))) {
                         ok = false;
                         break;
                     }
@@ -250,7 +262,8 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                     for (int h = 0; h < 2; ++h) {
                         const int ks = 2 * g + h;
                         if (ks >= num_kstages) break;
-                        if (!mbar_wait(&full[stage], phase, args.timeout_ns, abort_flag, args.status)) {
+                        if (!__all_sync(0xffffffffu,
+                                        mbar_wait(&full[stage], phase, args.timeout_ns, abort_flag, args.status))) {
                             ok = false;
                             break;
                         }
@@ -266,10 +279,10 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                         auto kstep = [&](int j) {
                             if constexpr (MX)
                                 mma_mxf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, (j & 1) ? idesc_mx1 : idesc_mx0,
-                                              sf + 4 * (j >> 1), sf + 16 + 8 * (j >> 1), (ks | j) != 0 ? 1u : 0u);
+                                              sf + 4 * (j >> 1), sf + 16 + 8 * (j >> 1), (ks | j) != 0 ? 1u : 0u, issue);
                             else
                                 mma_nvf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j,
-                                              sf + 16 + 8 * j, (ks | j) != 0 ? 1u : 0u);
+                                              sf + 16 + 8 * j, (ks | j) != 0 ? 1u : 0u, issue);
                         };
                         if (nk == 4) {
 #pragma unroll
@@ -277,16 +290,16 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                         } else {
                             for (int j = 0; j < nk; ++j) kstep(j);
                         }
-                        tc_commit_pair(&empty[stage], 0x3);
+                        tc_commit_pair(&empty[stage], 0x3, issue);
                         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                     }
-                    if (ok) tc_commit_pair(&sf_free[slot], 0x3);
+                    if (ok) tc_commit_pair(&sf_free[slot], 0x3, issue);
                 }
-                if (ok) tc_commit_pair(tfull, 0x3);
+                if (ok) tc_commit_pair(tfull, 0x3, issue);
             }
             // Tensor memory is freed after the final cluster barrier: first let
-            // every MMA this thread issued complete (bounded, also after an abort).
-            tc_commit_pair(mma_done, 0x1);
+            // every MMA this warp issued complete (bounded, also after an abort).
+            tc_commit_pair(mma_done, 0x1, issue);
             volatile uint32_t keep_waiting = 0u;
             mbar_wait(mma_done, 0, args.timeout_ns, &keep_waiting, args.status);
         }

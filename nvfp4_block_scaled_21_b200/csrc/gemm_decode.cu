@@ -72,12 +72,17 @@ struct DecodeCfg {
     static constexpr int kThreads = 320;                   // 10 warps
     static constexpr int kQThreads = 256;                  // quantizer warps 2..9
     static constexpr int kEarlyStages = 2;                 // weight stages in flight while x loads
-    static constexpr uint32_t kSfbCol = 2 * kN;            // x scales after two accumulators
+    // Each K step of a slab accumulates into its own accumulator (four
+    // independent chains of dependent MMAs instead of one), summed in a
+    // fixed order in the epilogue; two tiles' worth, double-buffered.
+    static constexpr int kAcc = 4;
+    static constexpr uint32_t kAccCols = kAcc * kN;        // 64 columns per tile buffer
+    static constexpr uint32_t kSlotCol = 2 * kAccCols;     // stage scale slots after the accumulators
+    static constexpr uint32_t kSlotCols = 32;              // weight scales 16 | x scales 16
     static constexpr uint32_t kTmemCols = 512;
-    // tensor memory: 2*16 accumulator columns + 16 per K slab of x scales +
-    // 16 per stage of weight scales
-    static constexpr int kMaxSlabs = (512 - 2 * kN - 16 * kStages) / 16;   // S = 8: 22; S = 10: 20
+    static constexpr int kMaxSlabs = 22;                   // x codes in shared memory: K <= 5632
     static constexpr int kBarriers = 3 * kStages + 8;
+    static_assert(kSlotCol + kStages * kSlotCols <= kTmemCols, "tensor memory budget");
     static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
     static_assert(kEarlyStages <= kStages, "early stages fit the ring");
 };
@@ -145,7 +150,6 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
-    const uint32_t sfa_col = C::kSfbCol + 16u * static_cast<uint32_t>(kslabs);
     const int my_tiles = static_cast<int>(blockIdx.x) < args.num_tiles
                              ? (args.num_tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
                              : 0;
@@ -207,21 +211,22 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                     break;
                 tc_fence_after();
                 const int nk = min(4, ksteps - 4 * ks);
-                const uint32_t d_tmem = tmem_base + acc * C::kN;
-                const uint32_t sfa = tmem_base + sfa_col + 16u * st;
-                const uint32_t sfb = tmem_base + C::kSfbCol + 16u * static_cast<uint32_t>(ks);
+                // K step q of the slab into accumulator q (the first slab overwrites)
+                const uint32_t d_tmem = tmem_base + acc * C::kAccCols;
+                const uint32_t sfa = tmem_base + C::kSlotCol + C::kSlotCols * st;
+                const uint32_t sfb = sfa + 16;
                 // K-step q: +32 bytes = +2 in the descriptors' address field
                 const uint64_t adesc = make_operand_desc(ring_base + st * C::kStageBytes);
                 const uint64_t bdesc = make_operand_desc(x_base + ks * C::kXSlab);
                 if (nk == 4) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        mma_nvf4(d_tmem, adesc + 2 * q, bdesc + 2 * q, idesc, sfa + 4 * q, sfb + 4 * q,
-                                 (ks | q) != 0 ? 1u : 0u);
+                        mma_nvf4(d_tmem + q * C::kN, adesc + 2 * q, bdesc + 2 * q, idesc, sfa + 4 * q, sfb + 4 * q,
+                                 ks != 0 ? 1u : 0u);
                 } else {
                     for (int q = 0; q < nk; ++q)
-                        mma_nvf4(d_tmem, adesc + 2 * q, bdesc + 2 * q, idesc, sfa + 4 * q, sfb + 4 * q,
-                                 (ks | q) != 0 ? 1u : 0u);
+                        mma_nvf4(d_tmem + q * C::kN, adesc + 2 * q, bdesc + 2 * q, idesc, sfa + 4 * q, sfb + 4 * q,
+                                 ks != 0 ? 1u : 0u);
                 }
                 tc_commit(&empty[st]);
                 if (ks == kslabs - 1) {
@@ -307,7 +312,6 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         const float inv6g = __frcp_rn(six_g);
         const bool exact_only = !(six_g > 0.0f) || isinf(inv6g);
         const bool write_xq = args.xq_codes != nullptr && blockIdx.x == 0;
-        const int64_t kb4 = ksteps * 4;                      // K % 64 == 0: no block padding
         // reciprocal of every possible decoded block scale, one per thread
         if (qt < 128) rcp_table[qt] = block_rcp(static_cast<uint32_t>(qt), g);
         __syncwarp();
@@ -347,11 +351,8 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                         *reinterpret_cast<uint2 *>(xc + (gq >> 2) * C::kXSlab + r * 128 + ((c ^ (r & 7)) << 4) +
                                                    8 * (kb & 1)) = cw;
                         if ((lane & 3) == 0) sfw[gq * 16 + r] = word;
-                        if (write_xq) {
+                        if (write_xq)
                             *reinterpret_cast<uint2 *>(args.xq_codes + static_cast<int64_t>(r) * (args.K / 2) + kb * 8) = cw;
-                            if ((lane & 3) == 0)
-                                *reinterpret_cast<uint32_t *>(args.xq_scales + scale_offset(r, kb, kb4)) = word;
-                        }
                     }
                 }
             }
@@ -364,51 +365,41 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                 st_shared_v4(row + ((c0 ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
                 st_shared_v4(row + (((c0 + 1) ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
             }
-            if (write_xq) {
-                // x_q's tensor scale, and the zero padding of its tiled scale
-                // layout: rows M .. roundup(M, 128) - 1
-                if (qt == 0) *args.xq_g = g;
-                for (int i = qt; i < (128 - args.M) * ksteps; i += C::kQThreads) {
-                    const int r = args.M + i / ksteps, gq = i % ksteps;
-                    *reinterpret_cast<uint32_t *>(args.xq_scales + scale_offset(r, 4 * gq, kb4)) = 0u;
-                }
-            }
+            if (write_xq && qt == 0) *args.xq_g = g;
         }
         fence_proxy_async_smem();          // the codes, for the tensor cores' operand reads
         __syncwarp();
         if (lane == 0) mbar_arrive(red);
         ok = ok && __all_sync(0xffffffffu, mbar_wait(red, 0, args.timeout_ns, abort_flag, args.status));
 
-        // (3) x scales into tensor memory, replicated in every lane quarter: the
-        // word of row l < 16 at K-step g goes to lane l, column kSfbCol + 4g;
-        // the other three columns of each K-step and lanes 16..31 are zero.
-        // One 16-column store per slab; the two warps of a quarter split them.
-        if (ok) {
-            const int per = (kslabs + 1) / 2;
-            const int i1 = min(kslabs, (half + 1) * per);
-            for (int i = half * per; i < i1; ++i) {
-                uint32_t sv[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const int gk = 4 * i + (k >> 2);
-                    sv[k] = ((k & 3) == 0 && lane < 16 && gk < ksteps) ? sfw[gk * 16 + lane] : 0u;
-                }
-                tmem_st_32x32b_x16(lane_base + C::kSfbCol + 16u * static_cast<uint32_t>(i), sv);
+        // The x codes are in shared memory and the x scale words in sfw: the
+        // MMA may read the codes; the scale warps copy each slab's x scale words
+        // into tensor memory together with its weight scales.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(xready);
+        if (ok && write_xq) {
+            // x_q's tiled scales, whole 16-byte chunks: chunk l of K step gq's
+            // atom holds rows l, l + 32, l + 64, l + 96; only row l < M <= 16
+            // is data, the rest (and rows M .. 15 of sfw) is zero padding
+            for (int i = qt; i < ksteps * 32; i += C::kQThreads) {
+                const int gq = i >> 5, l = i & 31;
+                const uint32_t w0 = l < C::kN ? sfw[gq * 16 + l] : 0u;
+                *reinterpret_cast<uint4 *>(args.xq_scales + static_cast<int64_t>(gq) * 512 + l * 16) =
+                    make_uint4(w0, 0u, 0u, 0u);
             }
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(xready);
         }
 
         if (half == 0) {
-            // ------------------------------------------------------------ weight-scale warps
-            // Lane l of every quarter receives the 16 bytes at l*16 of each
-            // 512-byte atom (columns c = 0..3 hold rows 32c + l, bytes = the
-            // 4 K-blocks), into the TMEM scale slot of the stage; stages are
-            // handed to the MMA two at a time (one store-completion wait per
-            // pair).  A partial last slab's missing atoms are stale bytes no
-            // MMA reads.
+            // ------------------------------------------------------------ scale warps
+            // Per slab, one 32-column store into the stage's TMEM slot:
+            // the weight scales (lane l of every quarter receives the 16 bytes
+            // at l*16 of each 512-byte atom: columns c = 0..3 hold rows 32c + l,
+            // bytes = the 4 K-blocks), then the x scales (replicated in every
+            // quarter: the word of row l < 16 at K step q of the slab goes to
+            // lane l, column 16 + 4q; the other columns and lanes are zero).
+            // Stages are handed to the MMA two at a time (one store-completion
+            // wait per pair).  A partial last slab's missing atoms and K steps
+            // are bytes no MMA reads.
             uint32_t pend[2];
             int npend = 0;
             auto flush = [&]() {
@@ -425,13 +416,19 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                 const bool got = mbar_wait(&full[st], par, args.timeout_ns, abort_flag, args.status);
                 if (!__all_sync(0xffffffffu, got)) break;
                 const uint8_t *src = ring + st * C::kStageBytes + C::kAStage + lane * 16;
-                uint32_t av[16];
+                const int ks = i % kslabs;
+                uint32_t av[32];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const uint4 a = ld_shared_v4(src + j * 512);
                     av[4 * j] = a.x; av[4 * j + 1] = a.y; av[4 * j + 2] = a.z; av[4 * j + 3] = a.w;
+                    const int gk = 4 * ks + j;
+                    av[16 + 4 * j] = (lane < 16 && gk < ksteps) ? sfw[gk * 16 + lane] : 0u;
+                    av[17 + 4 * j] = 0u;
+                    av[18 + 4 * j] = 0u;
+                    av[19 + 4 * j] = 0u;
                 }
-                tmem_st_32x32b_x16(lane_base + sfa_col + 16u * st, av);
+                tmem_st_32x32b_x32(lane_base + C::kSlotCol + C::kSlotCols * st, av);
                 pend[npend++] = st;
                 if (npend == 2) flush();
             }
@@ -446,19 +443,31 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                 const bool got = mbar_wait(&tfull[acc], acc_phase, args.timeout_ns, abort_flag, args.status);
                 if (!__all_sync(0xffffffffu, got)) break;
                 tc_fence_after();
-                uint32_t r[16];
-                tmem_ld_32x32b_x16(lane_base + acc * C::kN, r);
+                uint32_t r4[C::kAcc][16];
+#pragma unroll
+                for (int a = 0; a < C::kAcc; ++a) tmem_ld_32x32b_x16(lane_base + acc * C::kAccCols + a * C::kN, r4[a]);
                 tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[acc]);
+                // acc0 + acc1 + acc2 + acc3 in that order; accumulators that
+                // no K step reached (K < 256) hold no data and are skipped
+                float r[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float v = __uint_as_float(r4[0][i]);
+#pragma unroll
+                    for (int a = 1; a < C::kAcc; ++a)
+                        if (a < ksteps) v = __fadd_rn(v, __uint_as_float(r4[a][i]));
+                    r[i] = v;
+                }
                 const int p = t * 128 + quarter * 32 + lane;     // weight row = output column
                 if (p < args.N) {
                     OutT *y = static_cast<OutT *>(args.y);
 #pragma unroll
                     for (int i = 0; i < C::kN; ++i) {
                         if (i < args.M) {
-                            const OutT o = to_out<OutT>(__fmul_rn(__uint_as_float(r[i]), alpha));
+                            const OutT o = to_out<OutT>(__fmul_rn(r[i], alpha));
                             y[static_cast<int64_t>(i) * args.ldy + p] = o;
                             ym.add<OutT>(o);
                         }

@@ -25,11 +25,14 @@
 //           64-column chunks of the 16 activation rows (bf16, 128-byte
 //           swizzle), S-deep ring.
 //   1       TMEM allocator and MMA issuer: 16 MMAs (M = 128, N = 16, K = 16,
-//           A from tensor memory) per slab.
+//           A from tensor memory) per slab, MMA i of a slab into accumulator
+//           i % 8 (an MMA this small takes far less time than the latency of
+//           the previous one into the same accumulator).
 //   2..9    converters: two warps per TMEM lane quarter (one weight row per
 //           thread), each dequantizing two of the slab's four 64-wide K steps
 //           into one of two tensor-memory A slots.
-//   10..13  epilogue: y = acc * gw, stored as y[m][n].
+//   10..13  epilogue: acc = the 8 accumulators added in order, y = acc * gw,
+//           stored as y[m][n].
 // Every wait is bounded; a timeout sets the status word and winds the CTA
 // down after its copies and MMAs in flight have landed.
 #include <cstdlib>
@@ -61,7 +64,8 @@ struct W16Cfg {
     static constexpr int kStageBytes = kWStage + kSfStage + kXStage;   // 26 KB
     static constexpr int kN = 16;
     static constexpr int kThreads = 448;
-    static constexpr uint32_t kASlotCol = 2 * kN;          // A slots after two accumulators
+    static constexpr int kNumAcc = 8;                      // accumulators, kN columns each
+    static constexpr uint32_t kASlotCol = kNumAcc * kN;    // A slots after the accumulators
     static constexpr uint32_t kASlotCols = 128;            // 256 bf16 per row
     static constexpr uint32_t kTmemCols = 512;
     static constexpr int kBarBytes = 8 * (2 * kStages + 8) + 16;
@@ -245,9 +249,14 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
                 for (int c = 0; c < nk; ++c) {
                     const uint64_t bdesc = make_operand_desc(x0 + c * C::kXChunk);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)   // K = 16 per MMA: 8 TMEM columns, 32 bytes of a row
-                        mma_bf16_ts(tmem_base, a0 + 32 * c + 8 * q, bdesc + 2 * q, idesc,
-                                    (ks | c | q) != 0 ? 1u : 0u);
+                    for (int q = 0; q < 4; ++q) {   // K = 16 per MMA: 8 TMEM columns, 32 bytes of a row
+                        // MMA 4c + q of the slab -> accumulator (4c + q) % 8,
+                        // overwritten by its first MMA of the tile (slab 0:
+                        // K % 64 == 0, so every slab has K steps 0 and 1)
+                        const int a = (4 * c + q) % C::kNumAcc;
+                        mma_bf16_ts(tmem_base + a * C::kN, a0 + 32 * c + 8 * q, bdesc + 2 * q, idesc,
+                                    (ks != 0 || 4 * c + q >= C::kNumAcc) ? 1u : 0u);
+                    }
                 }
                 tc_commit(&empty[st]);
                 tc_commit(&a_empty[slot]);
@@ -316,9 +325,21 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
             if (!__all_sync(0xffffffffu, got)) break;
             tphase ^= 1u;
             tc_fence_after();
+            // ((a0 + a1) + a2) + ... in fp32, over the accumulators written:
+            // four MMAs per K step, so K = 64 (one K step) writes a0..a3 only
+            const uint32_t lb = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+            const int nacc = min(C::kNumAcc, 4 * min(4, ksteps));
             uint32_t acc[16];
-            tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16), acc);
+            tmem_ld_32x32b_x16(lb, acc);
             tmem_ld_wait();
+            for (int a = 1; a < nacc; ++a) {
+                uint32_t t[16];
+                tmem_ld_32x32b_x16(lb + a * C::kN, t);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    acc[i] = __float_as_uint(__fadd_rn(__uint_as_float(acc[i]), __uint_as_float(t[i])));
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty);

@@ -60,6 +60,21 @@ cudaError_t launch_gemm_w4a16(const void *x, int64_t M, int64_t K, int64_t ldx, 
                               bool y_bf16, int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
                               cudaStream_t stream);
 
+// W4A8: y[M][N] = A . B^T with MXFP8 activations (E4M3 bytes [M][K], UE8M0
+// scales per 32, tiled) and MXFP4 weights, kind::mxf8f6f4 (one-CTA kernel).
+cudaError_t launch_gemm_w4a8(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
+                             int64_t ldy, uint32_t *status, uint64_t timeout_ns, int num_sms,
+                             cudaStream_t stream, bool weights_ready, void *splitk_ws);
+
+// Tensor map over packed E2M1 rows that unpacks them into the 8-bit-container
+// shared-memory form (16 values per 16-byte chunk), boxes of 128 values.
+CUresult encode_tensor_map_fp4_unpacked(CUtensorMap *map, const void *base, uint64_t k_elems, uint64_t rows,
+                                        uint32_t box_rows);
+
+// MXFP8 quantizer (one pass): E4M3 bytes [rows][cols], UE8M0 scales tiled.
+cudaError_t launch_mx8_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld, uint8_t *elems,
+                                uint8_t *scales, int num_sms, cudaStream_t stream);
+
 // MXFP4 quantizer (one pass): codes [rows][cols/2], UE8M0 scales tiled.
 cudaError_t launch_mx_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld, uint8_t *codes,
                                uint8_t *scales, int num_sms, cudaStream_t stream);

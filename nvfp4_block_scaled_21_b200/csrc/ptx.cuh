@@ -208,13 +208,14 @@ __device__ __forceinline__ void tc_fence_after() {
 // (descriptors), block scales UE4M3 per 16 elements in tensor memory.
 __device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                         uint32_t accumulate) {
+                                         uint32_t accumulate, uint32_t issue = 1u) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
+        "setp.ne.b32 q, %7, 0;\n\t"
+        "@q " "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
         " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem), "r"(issue)
         : "memory");
 }
 
@@ -224,23 +225,52 @@ __device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint6
 // ID fields pick bytes {0,1} or {2,3} of it (see make_idesc_mxf4).
 __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                         uint32_t accumulate) {
+                                         uint32_t accumulate, uint32_t issue = 1u) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X"
+        "setp.ne.b32 q, %7, 0;\n\t"
+        "@q " "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X"
         " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem), "r"(issue)
+        : "memory");
+}
+
+// The W4A8 product: E2M1 and E4M3 operands (8-bit containers in shared
+// memory), one UE8M0 scale per 32 elements, K = 32 per MMA; a 32-bit scale
+// column holds four K steps' scales, picked by the descriptor's scale IDs.
+__device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                             uint32_t accumulate, uint32_t issue = 1u) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, %7, 0;\n\t"
+        "@q " "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X"
+        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem), "r"(issue)
         : "memory");
 }
 
 // Arrive once on `bar` when all previously issued tcgen05 async operations of
-// this thread have completed.
-__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+// this thread have completed.  (The MMA wrappers and the commits take an
+// optional `issue` flag: a whole warp may walk an issue loop with one elected
+// lane executing them.)
+__device__ __forceinline__ void tc_commit(uint64_t *bar, uint32_t issue = 1u) {
     asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_addr(bar))
+        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
+        "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+            smem_addr(bar)), "r"(issue)
         : "memory");
+}
+
+// One lane of the converged warp: the issuer of single-thread instructions in
+// loops the whole warp walks.  Elect once and keep the flag, so that a commit
+// comes from the lane that issued the MMAs it tracks.
+__device__ __forceinline__ bool elect_one_sync() {
+    uint32_t pred = 0;
+    asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}" : "=r"(pred));
+    return pred != 0;
 }
 
 // Each thread of the warp writes 16 (32) consecutive 32-bit columns of its lane.
@@ -372,6 +402,13 @@ __host__ __device__ constexpr uint32_t make_idesc_mxf4(uint32_t n, uint32_t m, u
            ((2u * (j & 1u)) << 29) | ((2u * (j & 1u)) << 4);
 }
 
+// Instruction descriptor of kind::mxf8f6f4 with the given A and B element
+// formats (E4M3 = 0, E2M1 = 5), UE8M0 scales, K-major, M = 128, the given N,
+// and scale ID j (0..3) for both operands: byte j of their scale columns.
+__host__ __device__ constexpr uint32_t make_idesc_mxf8f6f4(uint32_t n, uint32_t a_fmt, uint32_t b_fmt, uint32_t j) {
+    return (a_fmt << 7) | (b_fmt << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24) | (j << 29) | (j << 4);
+}
+
 // ---------------------------------------------------------------------------
 // Two-CTA (cluster of 2) forms: the pair shares one block-scaled MMA
 // (cta_group::2).  Multicast is used only on tcgen05.commit, never on loads.
@@ -432,35 +469,38 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 // memory and tensor memory, B split by N halves, scales in each CTA's TMEM.
 __device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                               uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                              uint32_t accumulate) {
+                                              uint32_t accumulate, uint32_t issue = 1u) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X"
+        "setp.ne.b32 q, %7, 0;\n\t"
+        "@q " "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X"
         " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem), "r"(issue)
         : "memory");
 }
 
 __device__ __forceinline__ void mma_mxf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                               uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                              uint32_t accumulate) {
+                                              uint32_t accumulate, uint32_t issue = 1u) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X"
+        "setp.ne.b32 q, %7, 0;\n\t"
+        "@q " "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X"
         " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem), "r"(issue)
         : "memory");
 }
 
 // Arrive once on the mbarrier at this shared offset in every CTA of `mask`
 // when the pair's previously issued tcgen05 operations have completed.
-__device__ __forceinline__ void tc_commit_pair(uint64_t *bar, uint16_t mask) {
+__device__ __forceinline__ void tc_commit_pair(uint64_t *bar, uint16_t mask, uint32_t issue = 1u) {
     asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-        " [%0], %1;" ::"r"(smem_addr(bar)),
-        "h"(mask)
+        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t"
+        "@q tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;\n\t}" ::"r"(smem_addr(bar)),
+        "h"(mask), "r"(issue)
         : "memory");
 }
 

@@ -44,6 +44,10 @@ __global__ void __launch_bounds__(256) amax_partials_kernel(const T *__restrict_
                                                             int64_t cols, int64_t ld,
                                                             float *__restrict__ partials) {
     constexpr int EPI = Elem<T>::kPerItem;
+    // Launched as a programmatic dependent of the previous kernel in the
+    // stream (which may have written x or still read the partials): resident
+    // early, it starts work the moment that kernel completes.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // let the encode pass queue up
     float m = 0.0f;
     if (ld == cols && rows * cols / EPI < (int64_t(1) << 31)) {
@@ -356,22 +360,25 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
     // pass 2 runs one thread per 16-value block
     const int g2 = quantize_grid(rows, cols, 1, num_sms, occ_encode[bf16]);
     if (g1 > kMaxAmaxPartials) g1 = kMaxAmaxPartials;
-    if (bf16)
-        amax_partials_kernel<__nv_bfloat16><<<g1, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16 *>(x), rows, cols, ld, partials);
-    else
-        amax_partials_kernel<float><<<g1, 256, 0, stream>>>(static_cast<const float *>(x), rows,
-                                                             cols, ld, partials);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg1 = {};
+    cfg1.gridDim = dim3(g1);
+    cfg1.blockDim = dim3(256);
+    cfg1.stream = stream;
+    cfg1.attrs = attr;
+    cfg1.numAttrs = 1;
+    cudaError_t e = bf16 ? cudaLaunchKernelEx(&cfg1, amax_partials_kernel<__nv_bfloat16>,
+                                              static_cast<const __nv_bfloat16 *>(x), rows, cols, ld, partials)
+                         : cudaLaunchKernelEx(&cfg1, amax_partials_kernel<float>, static_cast<const float *>(x), rows,
+                                              cols, ld, partials);
     if (e != cudaSuccess) return e;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(g2);
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (bf16)

@@ -520,3 +520,94 @@ int64_t oracle_mx_storage_bytes(int64_t rows, int64_t cols)
 {
     return rows * cols / 2 + rows * cols / 32;
 }
+
+
+/* ------------------------------------------------------------------------ */
+/* MXFP8 activations for the W4A8 product ([EEF]: the Zhouyi X3 passage,    */
+/* FP4 weights with activations quantized to FP8; on hardware whose native  */
+/* mixed FP4 x FP8 product is block-scaled, both operands carry MX scales). */
+/* Readings taken (the page gives no formula):                               */
+/*   X1  block scale: 32 consecutive values share an E8M0 scale X = 2^e,     */
+/*       e = ceil(log2(bamax / 448)): the smallest power of two that brings  */
+/*       the block's largest magnitude into the E4M3 range (bamax <= 448 X), */
+/*       clamped to [-127, 127]; an all-zero block gets byte 0 (M1 with      */
+/*       E4M3's largest value in place of E2M1's).                           */
+/*   X2  element: E4M3 RNE (ties to even, OCP "fn" grid) of x / X, which is  */
+/*       exact; the sign is kept, also for values that round to zero.       */
+/* ------------------------------------------------------------------------ */
+
+/* X1.  bamax / 448 = f * 2^p with f in [0.5, 1); the quotient is a power of
+ * two exactly when f == 0.5 (bamax = 448 * 2^k = 7 * 2^(k+6) is exact in
+ * fp32, and any other fp32 bamax is relatively at least 2^-24 away from it,
+ * far more than the fp64 rounding of the quotient), and then
+ * ceil(log2) = p - 1; otherwise it is p. */
+unsigned oracle_mx8_block_scale(float bamax)
+{
+    int p, e;
+    double f;
+    if (!(bamax > 0.0f))
+        return 0u;
+    f = frexp((double)bamax / 448.0, &p);
+    e = (f == 0.5) ? p - 1 : p;
+    if (e < -127)
+        e = -127;
+    if (e > 127)
+        e = 127;
+    return (unsigned)(e + 127);
+}
+
+/* X2: signed E4M3 byte of v, |v| <= 448 by construction (satfinite beyond). */
+unsigned oracle_e4m3_encode_signed(float v)
+{
+    unsigned mag = oracle_e4m3_encode(fabsf(v));
+    return signbit(v) ? (mag | 0x80u) : mag;
+}
+
+/* Quantize the logical [rows][cols] window (cols % 32 == 0) of a row-major
+ * fp32 matrix with leading dimension ld to MXFP8: E4M3 bytes [rows][cols]
+ * and E8M0 scale bytes [rows][cols/32].  Returns 0, or -1 on bad arguments or
+ * a non-finite input. */
+int oracle_mx8_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld,
+                        uint8_t *elems, uint8_t *scales)
+{
+    int64_t nblk = cols / 32;
+    if (rows < 0 || cols < 0 || cols % 32 != 0 || ld < cols)
+        return -1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            if (!isfinite(x[r * ld + c]))
+                return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nblk; ++b) {
+            const float *blk = x + r * ld + b * 32;
+            float bamax = 0.0f;
+            unsigned s;
+            double scale;
+            for (int i = 0; i < 32; ++i) {
+                float a = fabsf(blk[i]);
+                if (a > bamax)
+                    bamax = a;
+            }
+            s = oracle_mx8_block_scale(bamax);
+            scales[r * nblk + b] = (uint8_t)s;
+            scale = oracle_e8m0_value(s);
+            for (int i = 0; i < 32; ++i)
+                elems[r * cols + b * 32 + i] =
+                    (uint8_t)oracle_e4m3_encode_signed((float)((double)blk[i] / scale));
+        }
+    }
+    return 0;
+}
+
+/* fp64 dequantization of an MXFP8 [rows][cols]: e4m3 * 2^(s - 127), exact. */
+int oracle_mx8_dequantize_f64(const uint8_t *elems, const uint8_t *scales,
+                              int64_t rows, int64_t cols, double *y)
+{
+    if (rows < 0 || cols < 0 || cols % 32 != 0)
+        return -1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            y[r * cols + c] = oracle_e4m3_value(elems[r * cols + c]) *
+                              oracle_e8m0_value(scales[r * (cols / 32) + c / 32]);
+    return 0;
+}

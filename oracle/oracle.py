@@ -29,6 +29,10 @@ Parity status of each function (what pins it is in ``tests/test_oracle.py``):
                                       exact round trip; nearest-code check;
                                       block granularity; 4.25-bit storage;
                                       closed-form GEMM.
+* ``mx8_*``, ``w4a8_gemm_f64``       pinned: the scale rule by brute force over
+  (MXFP8 activations, W4A8)           every byte; elements against torch's E4M3
+                                      conversion; exact round trip; closed-form
+                                      W4A8 product.
 * tiled scale layout, nibble order   parity unpinned by the pages: fixed by the
                                       tensor-core operand format and checked only
                                       through GPU GEMM parity.
@@ -121,6 +125,14 @@ def _declare(L):
     L.oracle_mx_dequantize_f64.restype = ctypes.c_int
     L.oracle_mx_storage_bytes.argtypes = [_I64, _I64]
     L.oracle_mx_storage_bytes.restype = _I64
+    L.oracle_mx8_block_scale.argtypes = [ctypes.c_float]
+    L.oracle_mx8_block_scale.restype = ctypes.c_uint
+    L.oracle_e4m3_encode_signed.argtypes = [ctypes.c_float]
+    L.oracle_e4m3_encode_signed.restype = ctypes.c_uint
+    L.oracle_mx8_quantize.argtypes = [_P, _I64, _I64, _I64, _P, _P]
+    L.oracle_mx8_quantize.restype = ctypes.c_int
+    L.oracle_mx8_dequantize_f64.argtypes = [_P, _P, _I64, _I64, _P]
+    L.oracle_mx8_dequantize_f64.restype = ctypes.c_int
 
 
 def _ptr(a: np.ndarray):
@@ -380,3 +392,66 @@ def mx_gemm_f64(a: QuantizedMX, b: QuantizedMX, nthreads: int | None = None) -> 
 
 def mx_storage_bytes(rows: int, cols: int) -> int:
     return int(lib().oracle_mx_storage_bytes(rows, cols))
+
+
+# --------------------------------------------------------------------------
+# MXFP8 activations and the W4A8 product (readings X1-X2 in nvfp4_oracle.c):
+# FP4 weights (MXFP4) times FP8 activations (E4M3 elements, one E8M0 scale per
+# 32 values), the eefocus.com article's W4A8 (section on the Zhouyi X3 NPU).
+# --------------------------------------------------------------------------
+
+class QuantizedMX8:
+    """One MXFP8 tensor as the oracle emits it.
+
+    elems:  uint8 [rows][cols], E4M3 bytes
+    scales: uint8 [rows][cols/32], row-major E8M0 block scales
+    """
+
+    def __init__(self, elems, scales, rows, cols):
+        self.elems, self.scales, self.rows, self.cols = elems, scales, rows, cols
+
+
+def mx8_block_scale(bamax: float) -> int:
+    return lib().oracle_mx8_block_scale(float(bamax))
+
+
+def e4m3_encode_signed(v: float) -> int:
+    return lib().oracle_e4m3_encode_signed(float(v))
+
+
+def mx8_quantize(x: np.ndarray) -> QuantizedMX8:
+    """Quantize a 2-D fp32 array (or bf16 given as its uint16 bit patterns) to MXFP8."""
+    if x.dtype == np.uint16:
+        x = bf16_bits_to_f32(x)
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if x.ndim != 2:
+        raise ValueError("mx8_quantize expects a 2-D array")
+    rows, cols = x.shape
+    if cols % 32:
+        raise ValueError("cols must be a multiple of 32")
+    elems = np.zeros((rows, cols), np.uint8)
+    scales = np.zeros((rows, cols // 32), np.uint8)
+    rc = lib().oracle_mx8_quantize(_ptr(x), rows, cols, cols, _ptr(elems), _ptr(scales))
+    if rc != 0:
+        raise ValueError("oracle_mx8_quantize rejected the input (non-finite?)")
+    return QuantizedMX8(elems, scales, rows, cols)
+
+
+def mx8_dequantize_f64(q: QuantizedMX8) -> np.ndarray:
+    y = np.empty((q.rows, q.cols), np.float64)
+    rc = lib().oracle_mx8_dequantize_f64(_ptr(q.elems), _ptr(q.scales), q.rows, q.cols, _ptr(y))
+    assert rc == 0
+    return y
+
+
+def w4a8_gemm_f64(x: QuantizedMX8, w: QuantizedMX, nthreads: int | None = None) -> np.ndarray:
+    """W4A8: Y = deq(X) . deq(W)^T in fp64, X MXFP8 [M][K], W MXFP4 [N][K]."""
+    if x.cols != w.cols:
+        raise ValueError("K mismatch")
+    dx = mx8_dequantize_f64(x)
+    dw = mx_dequantize_f64(w)
+    y = np.empty((x.rows, w.rows), np.float64)
+    nt = nthreads or os.cpu_count() or 1
+    rc = lib().oracle_gemm_f64(_ptr(dx), _ptr(dw), x.rows, w.rows, x.cols, _ptr(y), int(nt))
+    assert rc == 0
+    return y

@@ -446,3 +446,44 @@ def test_mx_sizes_and_argument_checks_without_launch():
     assert g(ldy=36) == nv.ERR_MISALIGNED
     assert g(wb=8) == nv.ERR_WORKSPACE
     assert g(yt=4) == nv.ERR_INVALID_ARG
+
+
+def test_w4a8_argument_checks_without_launch():
+    """MXFP8 quantizer and W4A8 GEMM / linear layer: each call below breaks
+    exactly one rule (K a multiple of 128 and 32-byte aligned weight codes,
+    which the unpacking copy of the weights needs)."""
+    lib = nv.lib()
+
+    def mx8(elems=16, scales=16, rows=4, cols=128):
+        return nv.CMX8Tensor(elems, scales, rows, cols)
+
+    def q(x=16, xt=nv.BF16, r=4, c=128, ld=128, o=mx8()):
+        return lib.nvfp4_mx8_quantize(x, xt, r, c, ld, ctypes.byref(o) if o else None, None)
+
+    assert q(x=None) == nv.ERR_INVALID_ARG
+    assert q(xt=3) == nv.ERR_INVALID_ARG
+    assert q(ld=64) == nv.ERR_INVALID_ARG
+    assert q(o=mx8(rows=5)) == nv.ERR_INVALID_ARG
+    assert q(c=48, ld=48, o=mx8(cols=48)) == nv.ERR_UNSUPPORTED_SHAPE          # cols % 32
+    assert q(x=24) == nv.ERR_MISALIGNED
+    assert q(o=mx8(elems=24)) == nv.ERR_MISALIGNED
+
+    def g(a_=mx8(rows=8), b_=_mx(codes=32, rows=32, cols=128), y=16, yt=nv.BF16, ldy=32, ws=4096, wb=1 << 20):
+        return lib.nvfp4_w4a8_gemm(ctypes.byref(a_), ctypes.byref(b_), y, yt, ldy, ws, wb, None)
+
+    assert g(y=None) == nv.ERR_INVALID_ARG
+    assert g(b_=_mx(codes=32, rows=32, cols=256)) == nv.ERR_INVALID_ARG                       # K mismatch
+    assert g(a_=mx8(rows=8, cols=192), b_=_mx(codes=32, rows=32, cols=192)) == nv.ERR_UNSUPPORTED_SHAPE
+    assert g(b_=_mx(codes=48, rows=32, cols=128)) == nv.ERR_MISALIGNED                        # codes % 32
+    assert g(ldy=36) == nv.ERR_MISALIGNED
+    assert g(wb=8) == nv.ERR_WORKSPACE
+
+    def lin(x=16, K=128, w=_mx(codes=32, rows=32, cols=128), ldy=32, xq=None, wb=1 << 20):
+        return lib.nvfp4_w4a8_linear(x, nv.BF16, 8, K, K, ctypes.byref(w), 16, nv.BF16, ldy,
+                                     ctypes.byref(xq) if xq else None, 4096, wb, None)
+
+    assert lin(x=None) == nv.ERR_INVALID_ARG
+    assert lin(K=192, w=_mx(codes=32, rows=32, cols=192)) == nv.ERR_UNSUPPORTED_SHAPE          # K % 128
+    assert lin(w=_mx(codes=48, rows=32, cols=128)) == nv.ERR_MISALIGNED
+    assert lin(xq=mx8(rows=7)) == nv.ERR_INVALID_ARG
+    assert lin(wb=8) == nv.ERR_WORKSPACE

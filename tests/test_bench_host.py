@@ -92,3 +92,15 @@ def test_device_info_never_raises():
     import torch
     info = bench.device_info(torch, 0)
     assert set(info) == {"name", "cc", "cuda_runtime", "driver"}
+
+
+def test_reference_arm_inputs_do_not_load_the_library():
+    """The reference arm builds its inputs with the seeded generator loaded
+    from its file, so the process never maps libnvfp4.so."""
+    import subprocess
+    import sys
+    code = ("import sys; sys.path.insert(0, '.'); import bench; bench._gen('tiny'); "
+            "maps = open('/proc/self/maps').read(); print('libnvfp4' in maps, 'nvfp4_block_scaled_21_b200' in sys.modules)")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.split() == ["False", "False"], r.stdout

@@ -4,10 +4,8 @@ call the benchmark times.
 
 The decode kernel quantizes x itself in the quantizer's arithmetic, so its
 x_q (codes, tiled scales, tensor scale) must equal the oracle's bit for bit,
-and y must be within the GEMM tolerance of the fp64 oracle product.  It runs
-the same MMAs in the same K order as the two-kernel path (quantizer passes,
-then the swapped GEMM), so the two paths' outputs are also compared bit for
-bit.  The full-size tests call nvfp4_linear_fused twice in a row on different
+and y must be within the GEMM tolerance of the fp64 oracle product, as must
+the two-kernel path (quantizer passes, then the swapped GEMM) it replaces.  The full-size tests call nvfp4_linear_fused twice in a row on different
 rotation slots (different X and weight copies) without a synchronisation in
 between, as the benchmark's captured rotation does, so that a kernel that
 starts before the one before it has finished would show up."""
@@ -85,23 +83,25 @@ def test_decode_fused_parity(nv, M, N, K, xt, yt):
 
 
 @pytest.mark.parametrize("M,N,K", [(8, 1000, 1344), (16, 384, 640), (3, 136, 192)])
-def test_decode_fused_matches_two_kernel_path(nv, M, N, K, monkeypatch):
-    """The one-launch kernel and the quantizer + swapped GEMM path give the
-    same bits; also with a row pitch wider than K and no x_q requested."""
-    x, _, wt = make_inputs(M, N, K, 7 * M + N, torch.bfloat16)
+def test_decode_fused_and_two_kernel_paths(nv, M, N, K, monkeypatch):
+    """The one-launch kernel and the quantizer + swapped GEMM path, with a row
+    pitch wider than K and no x_q requested, both within tolerance of the
+    oracle.  (They sum the fp32 partial products in different orders: the
+    one-launch kernel keeps one accumulator per K step of a slab.)"""
+    x, x_or, wt = make_inputs(M, N, K, 7 * M + N, torch.bfloat16)
+    xq_o, wq_o = oracle.quantize(x_or), oracle.quantize(wt)
+    ref = oracle.gemm_f64(xq_o, wq_o)
     buf = torch.zeros((M, K + 40), dtype=torch.bfloat16, device="cuda")
     buf[:, :K] = x.cuda()
     wq = quantize_gpu(nv, f32_tensor(wt))
-    outs = []
     for fused in ("1", "0"):
         monkeypatch.setenv("NVFP4_DECODE_FUSED", fused)
         y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         ws = nv.workspace(nv.OP_LINEAR_FUSED, M, N, K)
         nv.nvfp4_linear_fused(buf[:, :K], wq, ws, nv.EPI_STORE, y=y)
         assert nv.nvfp4_get_device_status(ws) == nv.OK
-        outs.append(y)
-    torch.cuda.synchronize()
-    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+        assert_gemm_close(to_numpy_f64(y), ref, norms(xq_o)[:, None], norms(wq_o)[None, :], K, True,
+                          f"decode fused={fused}")
 
 
 def _two_slots(nv, w, xt_dtype=torch.bfloat16):

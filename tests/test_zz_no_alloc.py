@@ -62,6 +62,13 @@ def test_noalloc_matches_workspace_entry_point_twice(M, K, N):
         err = np.abs(got - ref)
         assert np.isfinite(got).all(), f"call {call}: non-finite output"
         assert (err <= tol).all(), f"call {call}: max err/tol {(err / tol).max():.3f}"
+        # and against the fp64 oracle itself, on sampled outputs
+        rng = np.random.default_rng(call)
+        ms, ns = rng.integers(0, M, 512), rng.integers(0, N, 512)
+        ref_o, na_o, nb_o = oracle.gemm_entries(x_o, w_o, ms, ns)
+        tol_o = gemm_tolerance(ref_o, na_o, nb_o, K, True)
+        err_o = np.abs(got[ms, ns] - ref_o)
+        assert (err_o <= tol_o).all(), f"call {call}: vs oracle max err/tol {(err_o / tol_o).max():.3f}"
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
