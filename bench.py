@@ -34,9 +34,9 @@ L2_BYTES = 126 * 1024 * 1024
 # from one ncu capture of the current kernels (dram__bytes_read.sum +
 # dram__bytes_write.sum); None where the kernel changed after its capture or
 # the capture did not cover every kernel of the dominant call.
-NCU_TRAFFIC = {"prefill": 158_123_264, "decode": None, "quantize": 174_949_888, "mlp": None,
-               "prefill_requant": None, "mx_prefill": 153_339_392, "w4a16_decode": None,
-               "w4a8_prefill": None}
+NCU_TRAFFIC = {"prefill": 157_946_112, "decode": 50_256_896, "quantize": None, "mlp": None,
+               "prefill_requant": 402_010_112, "mx_prefill": None, "w4a16_decode": 50_272_000,
+               "w4a8_prefill": 162_502_656}
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP4_PER_BF16 = 4.0          # dense FP4 : dense BF16 on B200 (9 : 2.25 PFLOP/s nominal)
@@ -225,17 +225,16 @@ class Decode(Prefill):
         # algorithmic bytes of the step: W codes + W scales, X bf16 in, Y bf16 out
         self.bytes = w_bytes + M * K * 2 + M * N * 2
         self.units = self.bytes / 1e9
-        # One launch per step: the decode kernel quantizes X itself while the
-        # weight stream is in flight, so the step's kernel is the dominant one.
-        self.launches = 1
-        self.dominant = {"kernel": "gemm_decode_kernel (X quantized in-kernel, swapped 128x16 MMA tiles)",
-                         "bound": "hbm", "algorithmic": self.bytes, "unit": "GB/s"}
+        # Per step: the quantizer's two passes over X, then the swapped GEMM
+        # (weights on the MMA's M, the 8 tokens on N = 16), which streams its
+        # first weight stages before the quantizer has finished.
+        self.launches = 3
+        self.dominant = {"kernel": "gemm_nvf4_kernel<16, swapped> (128x16 MMA tiles, four accumulators)",
+                         "bound": "hbm", "algorithmic": w_bytes + M * K // 2 + M * K // 16 + M * N * 2,
+                         "unit": "GB/s"}
         self.config["workload"] = (f"decode W4A4 linear: quantize X bf16 {M}x{K} per call, GEMM with "
                                    f"pre-quantized W {N}x{K}, bf16 out")
         self.config["algorithmic_bytes_per_step"] = self.bytes
-
-    def dominant_call(self, i):
-        self.step(i)
 
 
 class Quantize:
@@ -318,14 +317,15 @@ class Mlp:
         hq_bytes = M * N // 2 + M * N // 16
         self.bytes = per_step + M * K * 2 + M * K * 2 + 2 * hq_bytes
         self.units = self.bytes / 1e9
-        self.launches = 5                       # amax, encode (x); gate+up GEMM; encode (h); down GEMM
-        # The largest share of the step is the gate+up kernel (ncu: 33.4 us
+        # amax and encode passes on x; gate+up GEMM, which re-quantizes h in
+        # its epilogue (its 136 tiles fit the SMs); down GEMM
+        self.launches = 4
+        # The largest share of the step is the gate+up kernel (ncu: 33.0 us
         # against 27.5 us for the down projection).  It runs inside the
-        # fused call together with the two quantizer passes on x and the encode
-        # pass on h, so the roofline is taken over that call: gate and up
-        # weights, x in, h_q out.
-        self.dominant = {"kernel": "gemm_nvf4_dual_kernel (gate+up, SiLU*up epilogue) in the fused call "
-                                   "with the quantizer passes on x and h",
+        # fused call together with the two quantizer passes on x, so the
+        # roofline is taken over that call: gate and up weights, x in, h_q out.
+        self.dominant = {"kernel": "gemm_nvf4_dual_kernel (gate+up, SiLU*up epilogue re-quantizing h) in the "
+                                   "fused call with the quantizer passes on x",
                          "bound": "hbm",
                          "algorithmic": 2 * (N * K // 2 + N * K // 16) + M * K * 2 + hq_bytes,
                          "unit": "GB/s"}

@@ -74,7 +74,9 @@ uint8_t *ws_at(void *ws, size_t off) { return static_cast<uint8_t *>(ws) + off; 
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// Workspace carving (offsets in bytes).
+// Workspace carving (offsets in bytes).  The first kWsStatusBytes hold the
+// status word (offset 0) and the fused MLP's CTA arrival counter (offset 128).
+constexpr size_t kGridBarOff = 128;
 constexpr size_t kPartialsOff = kWsStatusBytes;
 constexpr size_t kPartialsBytes = kMaxAmaxPartials * sizeof(float);
 constexpr size_t kQuantizeWs = kPartialsOff + kPartialsBytes;
@@ -327,6 +329,14 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
         xq.cols = K;
     }
     if (!x_q) off = kQuantizeWs + quantized_bytes(M, K);
+    // MLP with one gate/up tile per SM: h is re-quantized inside the GEMM's
+    // epilogue, whose CTAs meet on a counter zeroed here (before the
+    // activation quantizer, so that the GEMM stays its dependent launch).
+    const bool fused_requant = epilogue == NVFP4_EPI_SILU_MUL_REQUANT && N != 0 && K != 0 &&
+                               dual_fused_requant_usable(M, N, dev.sms, static_cast<int>(kMaxAmaxPartials));
+    uint32_t *grid_bar = reinterpret_cast<uint32_t *>(ws_at(ws, kGridBarOff));
+    if (fused_requant && cudaMemsetAsync(grid_bar, 0, sizeof(uint32_t), stream) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
     cudaError_t e = launch_quantize(x, xt == NVFP4_BF16, M, K, ldx, xq.codes, xq.scales,
                                     xq.tensor_scale, partials, dev.sms, stream);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -351,16 +361,21 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
         return NVFP4_OK;
     }
 
-    // Gate and up in one GEMM whose epilogue writes h = SiLU(gate) * up and the
-    // per-CTA max |h|; then the quantizer's encode pass turns h into NVFP4.
-    float *h = y ? static_cast<float *>(y) : reinterpret_cast<float *>(ws_at(ws, off));
-    const int64_t ldh = y ? ldy : N;
+    // Gate and up in one GEMM whose epilogue forms h = SiLU(gate) * up and the
+    // per-CTA max |h|; h_q either in the same epilogue (fused_requant) or by
+    // the quantizer's encode pass over h written to memory.
     Operand act{xq.codes, xq.scales, xq.tensor_scale, M};
     Operand og{w->codes, w->scales, w->tensor_scale, N};
     Operand ou{w_up->codes, w_up->scales, w_up->tensor_scale, N};
     int nparts = 0;
+    if (fused_requant)
+        return from_cuda(launch_gemm_dual_silu(act, og, ou, K, static_cast<float *>(y), y ? ldy : N, partials,
+                                               kMaxAmaxPartials, &nparts, status, wait_timeout_ns(), dev.sms, stream,
+                                               true, y_q->codes, y_q->scales, y_q->tensor_scale, grid_bar));
+    float *h = y ? static_cast<float *>(y) : reinterpret_cast<float *>(ws_at(ws, off));
+    const int64_t ldh = y ? ldy : N;
     if (launch_gemm_dual_silu(act, og, ou, K, h, ldh, partials, kMaxAmaxPartials, &nparts, status,
-                              wait_timeout_ns(), dev.sms, stream, true) != cudaSuccess)
+                              wait_timeout_ns(), dev.sms, stream, true, nullptr, nullptr, nullptr, nullptr) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     return from_cuda(launch_encode_f32(h, M, N, ldh, partials, nparts, y_q->codes, y_q->scales,
                                        y_q->tensor_scale, dev.sms, stream));

@@ -11,8 +11,16 @@
 //     h = fl32(fl32(gate / fl32(1 + expf(-gate))) * up)
 // -- the same fp32 operations, in the same order, as the separate GEMMs and
 // the elementwise SiLU * up would -- plus, per CTA, max |h| in the format of
-// the quantizer's first pass, so that only the quantizer's encode pass has to
-// run on h afterwards.
+// the quantizer's first pass.
+//
+// Re-quantizing h (each NVFP4 tensor carries its own two-level scaling:
+// NVFP4 wiki page, section "技術原理") needs max |h| over the whole tensor
+// before the first block can be encoded.  When every CTA holds exactly one
+// tile (a cooperative launch, tiles <= SMs), the epilogue does it in place:
+// each CTA publishes its max |h|, waits (bounded) until every CTA has, and
+// encodes the tile it still holds in registers with the quantizer's own
+// arithmetic (encode.cuh), so h never goes to memory unless asked for.
+// Otherwise h is written and the quantizer's encode pass runs on it.
 //
 // Roles (one persistent CTA per SM, 14 warps), as in gemm.cu:
 //   warp 0      TMA producer: per 256-deep K slab the A tile (128 activation
@@ -25,8 +33,11 @@
 //               lane quarter (tcgen05.st), two stages per handshake.
 //   warps 6..13 epilogue: two warps per lane quarter, 64 columns each.
 // Every wait is bounded; a timeout sets the status word and winds down.
+#include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include "common.cuh"
+#include "encode.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -39,9 +50,14 @@ struct DualArgs {
     const uint8_t *sfbg;      // tiled scales of Wg (N rows)
     const uint8_t *sfbu;      // tiled scales of Wu
     const float *gx, *gwg, *gwu;
-    float *h;                 // [M][ldh] fp32
+    float *h;                 // [M][ldh] fp32, or null (fused re-quantization only)
     int64_t ldh;
     float *partials;          // max |h| per CTA (gridDim.x values)
+    uint8_t *hq_codes;        // fused re-quantization (null: off): h_q codes [M][N/2],
+    uint8_t *hq_scales;       // tiled scales,
+    float *hq_g;              // tensor scale,
+    uint32_t *grid_bar;       // CTA arrival counter, zero at launch
+    int32_t kb4;              // h_q scale blocks per row, rounded up to 4
     int32_t M, N;
     int32_t num_k_steps;      // K / 64
     int32_t num_p_tiles, num_q_tiles;
@@ -277,6 +293,10 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         const int row = quarter * 32 + lane;
         const float ag = __fmul_rn(*args.gx, *args.gwg);
         const float au = __fmul_rn(*args.gx, *args.gwu);
+        const bool fuse = args.hq_codes != nullptr;    // then this CTA has exactly one tile
+        float hv[2][32];                               // that tile's h for this thread
+        int tile_pt = 0, tile_qt = 0;
+        bool have_tile = false;
         float amax = 0.0f;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -288,20 +308,23 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             const int p = pt * 128 + row;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + half * 64;
             float *hrow = args.h + static_cast<int64_t>(p) * args.ldh;
+            tile_pt = pt;
+            tile_qt = qt;
+            have_tile = true;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t g[32], u[32];
                 tmem_ld_32x32b_x32(tb + c * 32, g);
                 tmem_ld_32x32b_x32(tb + 128 + c * 32, u);
                 tmem_ld_wait();
-                float h[32];
+                float *h = hv[c];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     h[i] = silu_mul(__fmul_rn(__uint_as_float(g[i]), ag), __fmul_rn(__uint_as_float(u[i]), au));
                     amax = fmaxf(amax, fabsf(h[i]));
                 }
                 const int q0 = qt * 128 + half * 64 + c * 32;
-                if (p < args.M) {
+                if (args.h != nullptr && p < args.M) {
                     if (q0 + 32 <= args.N) {
 #pragma unroll
                         for (int i = 0; i < 32; i += 4)
@@ -322,6 +345,77 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         if (lane == 0) warp_max[warp - 6] = amax;
+
+        if (fuse) {
+            // ---- grid-wide max |h|, then encode this thread's 4 blocks of 16
+            __shared__ float s_amax;
+            __shared__ uint32_t s_go;
+            asm volatile("bar.sync 1, 256;" ::: "memory");        // the 8 epilogue warps
+            if (warp == 6 && lane == 0) {
+                float m = 0.0f;
+                for (int i = 0; i < 8; ++i) m = fmaxf(m, warp_max[i]);
+                args.partials[blockIdx.x] = m;
+                __threadfence();
+                atomicAdd(args.grid_bar, 1u);
+                // every CTA of the cooperative launch is resident, so the
+                // count reaches gridDim.x unless one of them gave up; bounded
+                uint32_t go = 1u;
+                const uint64_t start = global_timer_ns();
+                for (uint32_t spin = 1;; ++spin) {
+                    uint32_t n;
+                    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(n) : "l"(args.grid_bar) : "memory");
+                    if (n >= gridDim.x) break;
+                    if ((spin & 63u) == 0) {
+                        if (*abort_flag) { go = 0u; break; }
+                        if (global_timer_ns() - start > args.timeout_ns) {
+                            atomicOr(args.status, kStatusTimeoutBit);
+                            *abort_flag = 1u;
+                            go = 0u;
+                            break;
+                        }
+                    }
+                }
+                float gmax = 0.0f;
+                if (go)
+                    for (int i = 0; i < static_cast<int>(gridDim.x); ++i) gmax = fmaxf(gmax, __ldcg(args.partials + i));
+                s_amax = gmax;
+                s_go = go && have_tile && !*abort_flag;
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (s_go) {
+                // the quantizer's arithmetic: g, 6g, its reciprocal, per block
+                // the E4M3 scale byte and the E2M1 codes
+                const float g = __fdiv_rn(s_amax, kTensorScaleDiv);
+                const float six_g = __fmul_rn(6.0f, g);
+                const float inv6g = __frcp_rn(six_g);
+                const bool exact_only = !(six_g > 0.0f) || isinf(inv6g);
+                if (blockIdx.x == 0 && warp == 6 && lane == 0) *args.hq_g = g;
+                const int p = tile_pt * 128 + row;
+                const int kb0 = (tile_qt * 128 + half * 64) / kBlock;   // first of this thread's 4 blocks
+                const int nblk = args.N / kBlock;
+                uint32_t word = 0;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(hv[b >> 1][(b & 1) * 16 + i]);
+                    const uint32_t sb = block_scale_byte(block_absmax(w, static_cast<float *>(nullptr)), six_g, inv6g,
+                                                         exact_only);
+                    const uint2 cw = block_codes<float, 16>(w, block_rcp(sb, g));
+                    word |= sb << (8 * b);
+                    if (p < args.M && kb0 + b < nblk)
+                        *reinterpret_cast<uint2 *>(args.hq_codes + static_cast<int64_t>(p) * (args.N / 2) +
+                                                   (kb0 + b) * 8) = cw;
+                }
+                // rows past M and blocks past N/16 are zero blocks: byte 0, the
+                // layout's padding value; blocks past kb4 are outside it
+                if (kb0 < args.kb4) {
+                    const int64_t off = (static_cast<int64_t>(p >> 7) * (args.kb4 / 4) + (kb0 >> 2)) * 512 +
+                                        (p & 31) * 16 + ((p >> 5) & 3) * 4;
+                    *reinterpret_cast<uint32_t *>(args.hq_scales + off) = word;
+                }
+            }
+        }
     }
 
     tc_fence_before();
@@ -340,10 +434,19 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
 
 }  // namespace
 
+bool dual_fused_requant_usable(int64_t M, int64_t N, int num_sms, int max_partials) {
+    // NVFP4_MLP_FUSED_REQUANT=0 keeps the separate encode pass on h.
+    const char *opt = getenv("NVFP4_MLP_FUSED_REQUANT");
+    if (opt != nullptr && opt[0] == '0') return false;
+    const int64_t tiles = ceil_div(M, 128) * ceil_div(N, 128);
+    return tiles >= 1 && tiles <= num_sms && tiles <= max_partials;
+}
+
 cudaError_t launch_gemm_dual_silu(const Operand &act, const Operand &wg, const Operand &wu, int64_t K,
                                   float *h, int64_t ldh, float *partials, int max_partials, int *num_partials,
                                   uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t stream,
-                                  bool weights_ready) {
+                                  bool weights_ready, uint8_t *hq_codes, uint8_t *hq_scales, float *hq_g,
+                                  uint32_t *grid_bar) {
     using C = DualCfg;
     CUtensorMap tmA, tmBg, tmBu;
     if (encode_tensor_map_u8(&tmA, act.codes, K / 2, act.rows, 128, 128) != CUDA_SUCCESS ||
@@ -360,6 +463,11 @@ cudaError_t launch_gemm_dual_silu(const Operand &act, const Operand &wg, const O
     a.h = h;
     a.ldh = ldh;
     a.partials = partials;
+    a.hq_codes = hq_codes;
+    a.hq_scales = hq_scales;
+    a.hq_g = hq_g;
+    a.grid_bar = grid_bar;
+    a.kb4 = static_cast<int32_t>(kb4_of(wg.rows));
     a.M = static_cast<int32_t>(act.rows);
     a.N = static_cast<int32_t>(wg.rows);
     a.num_k_steps = static_cast<int32_t>(K / 64);
@@ -373,6 +481,7 @@ cudaError_t launch_gemm_dual_silu(const Operand &act, const Operand &wg, const O
     if (grid > max_partials) grid = max_partials;
     if (grid < 1) grid = 1;
     *num_partials = grid;
+    if (hq_codes != nullptr && grid != tiles) return cudaErrorInvalidValue;   // one tile per CTA
     cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_dual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -381,10 +490,29 @@ cudaError_t launch_gemm_dual_silu(const Operand &act, const Operand &wg, const O
     cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;        // the fused form's CTAs wait for one another
+    attr[1].val.cooperative = 1;
     cfg.attrs = attr;
+    if (hq_codes == nullptr) {
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, gemm_nvf4_dual_kernel, tmA, tmBg, tmBu, a);
+    }
+    // Cooperative, and a programmatic dependent of the quantizer if the
+    // driver takes both; cooperative alone otherwise (remembered).
+    static std::atomic<int> coop_pdl{1};
+    if (coop_pdl.load()) {
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        e = cudaLaunchKernelEx(&cfg, gemm_nvf4_dual_kernel, tmA, tmBg, tmBu, a);
+        if (e == cudaSuccess) return e;
+        if (e != cudaErrorInvalidValue && e != cudaErrorNotSupported) return e;
+        (void)cudaGetLastError();      // a refused configuration, not a failed launch
+        coop_pdl.store(0);
+    }
+    cfg.attrs = attr + 1;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, gemm_nvf4_dual_kernel, tmA, tmBg, tmBu, a);
 }

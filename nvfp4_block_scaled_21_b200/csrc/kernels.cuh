@@ -93,10 +93,15 @@ cudaError_t launch_encode(const void *x, bool bf16, int64_t rows, int64_t cols, 
 // both products per tile), and max |h| per CTA into partials (the quantizer's
 // first-pass format); *num_partials receives how many were written
 // (<= max_partials).
+// h_q non-null: the fused form (one tile per CTA, cooperative launch; see
+// dual_fused_requant_usable) re-quantizes h in the epilogue; h may then be null.
+// grid_bar: a 32-bit counter that is zero when the kernel starts.
 cudaError_t launch_gemm_dual_silu(const Operand &act, const Operand &wg, const Operand &wu, int64_t K,
                                   float *h, int64_t ldh, float *partials, int max_partials, int *num_partials,
                                   uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t stream,
-                                  bool weights_ready);
+                                  bool weights_ready, uint8_t *hq_codes, uint8_t *hq_scales, float *hq_g,
+                                  uint32_t *grid_bar);
+bool dual_fused_requant_usable(int64_t M, int64_t N, int num_sms, int max_partials);
 
 
 // The W4A4 linear layer for M <= 16 activation rows with the activation

@@ -1,11 +1,11 @@
-"""GPU parity of the one-launch decode path (activation quantizer inside the
-GEMM, M <= 16) and of the W4A4 linear layer at full size through the exact
-call the benchmark times.
+"""GPU parity of the two decode paths of nvfp4_linear_fused (M <= 16): the
+default quantizer passes + swapped GEMM, and the opt-in one-launch kernel
+(NVFP4_DECODE_FUSED=1) that quantizes x inside the GEMM; and of the W4A4
+linear layer at full size through the exact call the benchmark times.
 
-The decode kernel quantizes x itself in the quantizer's arithmetic, so its
-x_q (codes, tiled scales, tensor scale) must equal the oracle's bit for bit,
-and y must be within the GEMM tolerance of the fp64 oracle product, as must
-the two-kernel path (quantizer passes, then the swapped GEMM) it replaces.  The full-size tests call nvfp4_linear_fused twice in a row on different
+Both paths quantize x in the quantizer's arithmetic, so x_q (codes, tiled
+scales, tensor scale) must equal the oracle's bit for bit, and y must be
+within the GEMM tolerance of the fp64 oracle product.  The full-size tests call nvfp4_linear_fused twice in a row on different
 rotation slots (different X and weight copies) without a synchronisation in
 between, as the benchmark's captured rotation does, so that a kernel that
 starts before the one before it has finished would show up."""
@@ -64,8 +64,10 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("fused", ["0", "1"])
 @pytest.mark.parametrize("M,N,K,xt,yt", CASES)
-def test_decode_fused_parity(nv, M, N, K, xt, yt):
+def test_decode_parity(nv, M, N, K, xt, yt, fused, monkeypatch):
+    monkeypatch.setenv("NVFP4_DECODE_FUSED", fused)
     x, x_or, wt = make_inputs(M, N, K, M * 1000 + K, xt)
     xq_o, wq_o = oracle.quantize(x_or), oracle.quantize(wt)
     wq = quantize_gpu(nv, f32_tensor(wt))
@@ -79,7 +81,7 @@ def test_decode_fused_parity(nv, M, N, K, xt, yt):
     assert_quantized_equal(x_q, xq_o)
     ref = oracle.gemm_f64(xq_o, wq_o)
     assert_gemm_close(to_numpy_f64(y), ref, norms(xq_o)[:, None], norms(wq_o)[None, :], K,
-                      yt == torch.bfloat16, "decode")
+                      yt == torch.bfloat16, f"decode fused={fused}")
 
 
 @pytest.mark.parametrize("M,N,K", [(8, 1000, 1344), (16, 384, 640), (3, 136, 192)])

@@ -113,18 +113,61 @@ def check_mlp(nv, X, Wg, Wu, Wd, M, K, N):
     assert_gemm_close(to_numpy_f64(y), ref, norms(hq_o)[:, None], norms(wd_o)[None, :], N, True, "down")
 
 
-def test_mlp_small(nv):
+# h_q is formed either inside the gate/up kernel's epilogue (one tile per SM:
+# the default when the tiles fit) or by the quantizer's encode pass over h
+# (NVFP4_MLP_FUSED_REQUANT=0, and always when the tiles outnumber the SMs).
+@pytest.mark.parametrize("fused", ["1", "0"])
+def test_mlp_small(nv, fused, monkeypatch):
+    monkeypatch.setenv("NVFP4_MLP_FUSED_REQUANT", fused)
     M, K, N = 32, 512, 384
     w = workloads.make("mlp", M=M, K=K, N=N, seed=40)
     check_mlp(nv, w["X"], w["Wg"], w["Wu"], w["Wd"], M, K, N)
 
 
-def test_mlp_ragged_tiles(nv):
+@pytest.mark.parametrize("fused", ["1", "0"])
+def test_mlp_ragged_tiles(nv, fused, monkeypatch):
     """Two 128-row tiles with a partial second one, a partial last 128-column
     tile of h and a partial last K slab, through the fused gate/up kernel."""
+    monkeypatch.setenv("NVFP4_MLP_FUSED_REQUANT", fused)
     M, K, N = 200, 320, 320
     w = workloads.make("mlp", M=M, K=K, N=N, seed=41)
     check_mlp(nv, w["X"], w["Wg"], w["Wu"], w["Wd"], M, K, N)
+
+
+def test_mlp_more_tiles_than_sms(nv):
+    """9 x 18 = 162 gate/up tiles, more than the SMs: the encode pass path."""
+    M, K, N = 1100, 256, 2304
+    w = workloads.make("mlp", M=M, K=K, N=N, seed=42)
+    check_mlp(nv, w["X"], w["Wg"], w["Wu"], w["Wd"], M, K, N)
+
+
+def test_mlp_fused_requant_without_h(nv, monkeypatch):
+    """The in-epilogue re-quantization with h not requested (h never written)
+    gives the same h_q bytes (padding included) and tensor scale as with h
+    requested, and as the separate encode pass; also against the oracle's
+    quantization of the GPU's h.  N = 1040: 65 blocks per row, so the scale
+    rows are padded to 68 and the last tile's second half lies past them."""
+    M, K, N = 160, 1024, 1040
+    w = workloads.make("mlp", M=M, K=K, N=N, seed=43)
+    wg, wu = quantize_gpu(nv, bf16_tensor(w["Wg"])), quantize_gpu(nv, bf16_tensor(w["Wu"]))
+    x = bf16_tensor(w["X"])
+    ws = nv.workspace(nv.OP_LINEAR_FUSED_SILU, M, N, K)
+    outs = []
+    h = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    for fused, with_h in (("1", False), ("1", True), ("0", True)):
+        monkeypatch.setenv("NVFP4_MLP_FUSED_REQUANT", fused)
+        h_q = nv.NVFP4Tensor.empty(M, N)
+        h_q.codes.fill_(0x77)
+        h_q.scales.fill_(0x55)
+        nv.nvfp4_linear_fused(x, wg, ws, nv.EPI_SILU_MUL_REQUANT, y=h if with_h else None, w_up=wu, y_q=h_q)
+        assert nv.nvfp4_get_device_status(ws) == nv.OK
+        torch.cuda.synchronize()
+        outs.append(h_q)
+    assert_quantized_equal(outs[0], oracle.quantize(h.cpu().numpy()))
+    for q in outs[1:]:
+        assert torch.equal(q.codes, outs[0].codes)
+        assert torch.equal(q.scales, outs[0].scales)
+        assert torch.equal(q.tensor_scale, outs[0].tensor_scale)
 
 
 def test_linear_degenerate_shapes(nv):
