@@ -34,8 +34,8 @@ L2_BYTES = 126 * 1024 * 1024
 # from one ncu capture of the current kernels (dram__bytes_read.sum +
 # dram__bytes_write.sum); None where the kernel changed after its capture or
 # the capture did not cover every kernel of the dominant call.
-NCU_TRAFFIC = {"prefill": 157_946_112, "decode": 50_256_896, "quantize": None, "mlp": None,
-               "prefill_requant": 402_010_112, "mx_prefill": None, "w4a16_decode": 50_272_000,
+NCU_TRAFFIC = {"prefill": 157_946_112, "decode": 50_256_896, "quantize": 172_076_288, "mlp": 112_434_688,
+               "prefill_requant": 402_010_112, "mx_prefill": 153_014_272, "w4a16_decode": 50_272_000,
                "w4a8_prefill": 162_502_656}
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -317,15 +317,14 @@ class Mlp:
         hq_bytes = M * N // 2 + M * N // 16
         self.bytes = per_step + M * K * 2 + M * K * 2 + 2 * hq_bytes
         self.units = self.bytes / 1e9
-        # amax and encode passes on x; gate+up GEMM, which re-quantizes h in
-        # its epilogue (its 136 tiles fit the SMs); down GEMM
-        self.launches = 4
-        # The largest share of the step is the gate+up kernel (ncu: 33.0 us
-        # against 27.5 us for the down projection).  It runs inside the
-        # fused call together with the two quantizer passes on x, so the
-        # roofline is taken over that call: gate and up weights, x in, h_q out.
-        self.dominant = {"kernel": "gemm_nvf4_dual_kernel (gate+up, SiLU*up epilogue re-quantizing h) in the "
-                                   "fused call with the quantizer passes on x",
+        self.launches = 5                       # amax, encode (x); gate+up GEMM; encode (h); down GEMM
+        # The largest share of the step is the gate+up kernel (ncu: 33.6 us
+        # against 26.6 us for the down projection).  It runs inside the
+        # fused call together with the two quantizer passes on x and the encode
+        # pass on h, so the roofline is taken over that call: gate and up
+        # weights, x in, h_q out.
+        self.dominant = {"kernel": "gemm_nvf4_dual_kernel (gate+up, SiLU*up epilogue) in the fused call "
+                                   "with the quantizer passes on x and h",
                          "bound": "hbm",
                          "algorithmic": 2 * (N * K // 2 + N * K // 16) + M * K * 2 + hq_bytes,
                          "unit": "GB/s"}

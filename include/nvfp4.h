@@ -41,16 +41,22 @@
  *     There is no CPU fallback.
  *   - Workspace: `ws` points to at least nvfp4_workspace_bytes(...) bytes of
  *     device memory.  Zero-fill it once after allocating; the library keeps a
- *     sticky status word in its first 16 bytes and uses the rest as scratch.
+ *     sticky status word in its first 16 bytes and the grid-wide meeting
+ *     point of its cooperative kernels at bytes 128..135 (back at zero after
+ *     every completed call), and uses the rest as scratch.  After a device-side
+ *     give-up (NVFP4_ERR_TIMEOUT) zero-fill it again before reusing it.
  *     GEMMs with few output tiles split K across SMs and add fp32 partial
  *     sums in the scratch (zero-filled by the call itself, so workspaces may
  *     be shared between operations and shapes that do not overlap in time).
  *     Calls that share one workspace must not overlap on the GPU.
- *   - Kernel choice is automatic.  Two environment switches, read at each
- *     call, exist for A/B measurements: NVFP4_GEMM_CTA_PAIR=0 keeps large-M
- *     GEMMs on the one-CTA kernel; NVFP4_GEMM_STREAMK=0 disables the split-K
- *     (stream-K) path for GEMMs with few output tiles.  Results stay within
- *     the same tolerance either way.
+ *   - Kernel choice is automatic.  Environment switches, read at each call,
+ *     exist for A/B measurements: NVFP4_GEMM_CTA_PAIR=0 keeps large-M GEMMs
+ *     on the one-CTA kernel; NVFP4_GEMM_STREAMK=0 disables the split-K
+ *     (stream-K) path for GEMMs with few output tiles; NVFP4_DECODE_FUSED=1
+ *     runs nvfp4_linear_fused's STORE form for M <= 16 as one kernel that
+ *     quantizes x itself; NVFP4_MLP_FUSED_REQUANT=1 re-quantizes h inside the
+ *     gate/up kernel of the SiLU form when its tiles fit one per SM.  Results
+ *     stay within the same tolerance either way (x_q and y_q bit-identical).
  */
 #ifndef NVFP4_H
 #define NVFP4_H

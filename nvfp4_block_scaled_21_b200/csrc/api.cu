@@ -75,7 +75,9 @@ uint8_t *ws_at(void *ws, size_t off) { return static_cast<uint8_t *>(ws) + off; 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace carving (offsets in bytes).  The first kWsStatusBytes hold the
-// status word (offset 0) and the fused MLP's CTA arrival counter (offset 128).
+// status word (offset 0) and the grid meeting point of the cooperative
+// kernels (offset 128: arrival count, generation; back at zero after every
+// completed meeting).
 constexpr size_t kGridBarOff = 128;
 constexpr size_t kPartialsOff = kWsStatusBytes;
 constexpr size_t kPartialsBytes = kMaxAmaxPartials * sizeof(float);
@@ -330,13 +332,10 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
     }
     if (!x_q) off = kQuantizeWs + quantized_bytes(M, K);
     // MLP with one gate/up tile per SM: h is re-quantized inside the GEMM's
-    // epilogue, whose CTAs meet on a counter zeroed here (before the
-    // activation quantizer, so that the GEMM stays its dependent launch).
+    // epilogue, whose CTAs meet at the workspace's grid meeting point.
     const bool fused_requant = epilogue == NVFP4_EPI_SILU_MUL_REQUANT && N != 0 && K != 0 &&
                                dual_fused_requant_usable(M, N, dev.sms, static_cast<int>(kMaxAmaxPartials));
     uint32_t *grid_bar = reinterpret_cast<uint32_t *>(ws_at(ws, kGridBarOff));
-    if (fused_requant && cudaMemsetAsync(grid_bar, 0, sizeof(uint32_t), stream) != cudaSuccess)
-        return NVFP4_ERR_CUDA;
     cudaError_t e = launch_quantize(x, xt == NVFP4_BF16, M, K, ldx, xq.codes, xq.scales,
                                     xq.tensor_scale, partials, dev.sms, stream);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;

@@ -95,7 +95,7 @@ cudaError_t launch_encode(const void *x, bool bf16, int64_t rows, int64_t cols, 
 // (<= max_partials).
 // h_q non-null: the fused form (one tile per CTA, cooperative launch; see
 // dual_fused_requant_usable) re-quantizes h in the epilogue; h may then be null.
-// grid_bar: a 32-bit counter that is zero when the kernel starts.
+// grid_bar: the two-word grid meeting point (see grid_meet), zero-filled once.
 cudaError_t launch_gemm_dual_silu(const Operand &act, const Operand &wg, const Operand &wu, int64_t K,
                                   float *h, int64_t ldh, float *partials, int max_partials, int *num_partials,
                                   uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t stream,

@@ -78,6 +78,41 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     }
 }
 
+// Grid-wide meeting point of a cooperative launch, run by one thread per CTA
+// after its CTA's writes that the others will read (each writer fenced them).
+// bar[0] counts arrivals, bar[1] is the generation: the last CTA to arrive
+// resets the count and advances the generation, the others wait (bounded) for
+// the generation to move.  The count is back at zero after every completed
+// meeting, so a zero-filled pair serves any sequence of launches and grid
+// sizes that do not overlap in time.  Returns false on a timeout or an abort
+// (the timeout is recorded as mbar_wait does).
+__device__ __forceinline__ bool grid_meet(uint32_t *bar, uint64_t timeout_ns, volatile uint32_t *abort_flag,
+                                          uint32_t *status) {
+    uint32_t gen;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(gen) : "l"(bar + 1) : "memory");
+    __threadfence();
+    if (atomicAdd(bar, 1u) == gridDim.x - 1) {
+        atomicExch(bar, 0u);
+        __threadfence();
+        atomicAdd(bar + 1, 1u);
+        return true;
+    }
+    const uint64_t start = global_timer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        uint32_t now;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(now) : "l"(bar + 1) : "memory");
+        if (now != gen) return true;
+        if ((spin & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - start > timeout_ns) {
+                atomicOr(status, kStatusTimeoutBit);
+                *abort_flag = 1u;
+                return false;
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // TMA and bulk copies (global -> shared, completion on an mbarrier)
 // ---------------------------------------------------------------------------
