@@ -34,7 +34,7 @@ L2_BYTES = 126 * 1024 * 1024
 # from one ncu capture of the current kernels (dram__bytes_read.sum +
 # dram__bytes_write.sum); None where the kernel changed after its capture or
 # the capture did not cover every kernel of the dominant call.
-NCU_TRAFFIC = {"prefill": 157_946_112, "decode": 50_256_896, "quantize": 172_076_288, "mlp": 112_434_688,
+NCU_TRAFFIC = {"prefill": 157_946_112, "decode": 50_256_896, "quantize": 172_076_288, "mlp": 103_521_536,
                "prefill_requant": 402_010_112, "mx_prefill": 153_014_272, "w4a16_decode": 50_272_000,
                "w4a8_prefill": 162_502_656}
 FALLBACK_HBM_GBS = 6650.0
@@ -253,9 +253,9 @@ class Quantize:
         self.nv, self.torch = nv, torch
         n = self.M * self.K
         # The two-pass method reads x twice (amax pass, encode pass: x is 84 MB
-        # and measured L2 reuse between the passes is negligible) and writes the
-        # codes, the scales and the tensor scale.  The one-read lower bound of a
-        # hypothetical single-pass quantizer is reported beside it.
+        # and the second read comes from DRAM again) and writes the codes, the
+        # scales and the tensor scale.  The one-read lower bound is reported
+        # beside it.
         self.bytes_one_read = n * 2 + n // 2 + n // 16 + 4
         self.bytes = self.bytes_one_read + n * 2
         self.units = self.bytes / 1e9
@@ -317,14 +317,15 @@ class Mlp:
         hq_bytes = M * N // 2 + M * N // 16
         self.bytes = per_step + M * K * 2 + M * K * 2 + 2 * hq_bytes
         self.units = self.bytes / 1e9
-        self.launches = 5                       # amax, encode (x); gate+up GEMM; encode (h); down GEMM
-        # The largest share of the step is the gate+up kernel (ncu: 33.6 us
-        # against 26.6 us for the down projection).  It runs inside the
-        # fused call together with the two quantizer passes on x and the encode
-        # pass on h, so the roofline is taken over that call: gate and up
-        # weights, x in, h_q out.
-        self.dominant = {"kernel": "gemm_nvf4_dual_kernel (gate+up, SiLU*up epilogue) in the fused call "
-                                   "with the quantizer passes on x and h",
+        # amax and encode passes on x; gate+up GEMM, which re-quantizes h in
+        # its epilogue (its 136 tiles fit the SMs); down GEMM
+        self.launches = 4
+        # The largest share of the step is the gate+up kernel (ncu: 40.4 us
+        # against 27.8 us for the down projection).  It runs inside the
+        # fused call together with the two quantizer passes on x, so the
+        # roofline is taken over that call: gate and up weights, x in, h_q out.
+        self.dominant = {"kernel": "gemm_nvf4_dual_kernel (gate+up, SiLU*up epilogue re-quantizing h) in the "
+                                   "fused call with the quantizer passes on x",
                          "bound": "hbm",
                          "algorithmic": 2 * (N * K // 2 + N * K // 16) + M * K * 2 + hq_bytes,
                          "unit": "GB/s"}

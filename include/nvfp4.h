@@ -54,9 +54,14 @@
  *     on the one-CTA kernel; NVFP4_GEMM_STREAMK=0 disables the split-K
  *     (stream-K) path for GEMMs with few output tiles; NVFP4_DECODE_FUSED=1
  *     runs nvfp4_linear_fused's STORE form for M <= 16 as one kernel that
- *     quantizes x itself; NVFP4_MLP_FUSED_REQUANT=1 re-quantizes h inside the
- *     gate/up kernel of the SiLU form when its tiles fit one per SM.  Results
- *     stay within the same tolerance either way (x_q and y_q bit-identical).
+ *     quantizes x itself; NVFP4_MLP_FUSED_REQUANT=0 keeps the SiLU form's
+ *     re-quantization of h in a separate encode pass (by default the gate/up
+ *     kernel does it in its epilogue when its tiles fit one per SM);
+ *     NVFP4_QUANTIZE_ONEPASS=1 quantizes large contiguous tensors with one
+ *     cooperative kernel that reads x once (slower than the two passes on
+ *     B200 as measured; kept for A/B runs).
+ *     Results stay within the same tolerance either way (x_q and y_q
+ *     bit-identical).
  */
 #ifndef NVFP4_H
 #define NVFP4_H

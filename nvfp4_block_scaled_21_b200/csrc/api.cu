@@ -153,7 +153,9 @@ nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype xt, int64_t rows, int64_t
     return from_cuda(launch_quantize(x, xt == NVFP4_BF16, rows, cols, ld, out->codes, out->scales,
                                      out->tensor_scale,
                                      reinterpret_cast<float *>(ws_at(ws, kPartialsOff)), dev.sms,
-                                     reinterpret_cast<cudaStream_t>(stream)));
+                                     reinterpret_cast<cudaStream_t>(stream),
+                                     reinterpret_cast<uint32_t *>(ws_at(ws, kGridBarOff)),
+                                     static_cast<uint32_t *>(ws), wait_timeout_ns()));
 }
 
 nvfp4_status nvfp4_dequantize(const nvfp4_tensor *q, void *y, nvfp4_dtype yt, int64_t ldy,
@@ -337,7 +339,8 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
                                dual_fused_requant_usable(M, N, dev.sms, static_cast<int>(kMaxAmaxPartials));
     uint32_t *grid_bar = reinterpret_cast<uint32_t *>(ws_at(ws, kGridBarOff));
     cudaError_t e = launch_quantize(x, xt == NVFP4_BF16, M, K, ldx, xq.codes, xq.scales,
-                                    xq.tensor_scale, partials, dev.sms, stream);
+                                    xq.tensor_scale, partials, dev.sms, stream, grid_bar, status,
+                                    wait_timeout_ns());
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     // (The GEMM writes its per-CTA maxima of |y| into the same partials only
     // at its end, after its dependent-launch wait, so the activation encode

@@ -15,9 +15,9 @@
 //
 // Re-quantizing h (each NVFP4 tensor carries its own two-level scaling:
 // NVFP4 wiki page, section "技術原理") needs max |h| over the whole tensor
-// before the first block can be encoded.  In the fused form (opt-in, see
-// dual_fused_requant_usable), when every CTA holds exactly one tile (a
-// cooperative launch, tiles <= SMs), the epilogue does it in place:
+// before the first block can be encoded.  When every CTA holds exactly one
+// tile (a cooperative launch, tiles <= SMs: dual_fused_requant_usable), the
+// epilogue does it in place:
 // each CTA publishes its max |h|, meets the others at a bounded grid-wide
 // meeting point (grid_meet), and encodes the tile it still holds in
 // registers with the quantizer's own arithmetic (encode.cuh), so h never
@@ -353,19 +353,29 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             __shared__ float s_amax;
             __shared__ uint32_t s_go;
             asm volatile("bar.sync 1, 256;" ::: "memory");        // the 8 epilogue warps
-            if (warp == 6 && lane == 0) {
-                float m = 0.0f;
-                for (int i = 0; i < 8; ++i) m = fmaxf(m, warp_max[i]);
-                args.partials[blockIdx.x] = m;
-                // every CTA of the cooperative launch is resident and arrives
-                // exactly once (also after a give-up of its own), so the wait
-                // ends unless one of them gave up; bounded either way
-                const uint32_t go = grid_meet(args.grid_bar, args.timeout_ns, abort_flag, args.status) ? 1u : 0u;
+            if (warp == 6) {
+                uint32_t go = 0u;
+                if (lane == 0) {
+                    float m = 0.0f;
+                    for (int i = 0; i < 8; ++i) m = fmaxf(m, warp_max[i]);
+                    args.partials[blockIdx.x] = m;
+                    // every CTA of the cooperative launch is resident and
+                    // arrives exactly once (also after a give-up of its own),
+                    // so the wait ends unless one of them gave up; bounded
+                    go = grid_meet(args.grid_bar, args.timeout_ns, abort_flag, args.status) ? 1u : 0u;
+                }
+                go = __shfl_sync(0xffffffffu, go, 0);
+                // the grid's maxima, read by the whole warp at once
                 float gmax = 0.0f;
                 if (go)
-                    for (int i = 0; i < static_cast<int>(gridDim.x); ++i) gmax = fmaxf(gmax, __ldcg(args.partials + i));
-                s_amax = gmax;
-                s_go = go && have_tile && !*abort_flag;
+                    for (int i = lane; i < static_cast<int>(gridDim.x); i += 32)
+                        gmax = fmaxf(gmax, __ldcg(args.partials + i));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+                if (lane == 0) {
+                    s_amax = gmax;
+                    s_go = go && have_tile && !*abort_flag;
+                }
             }
             asm volatile("bar.sync 1, 256;" ::: "memory");
             if (s_go) {
@@ -421,14 +431,11 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
 }  // namespace
 
 bool dual_fused_requant_usable(int64_t M, int64_t N, int num_sms, int max_partials) {
-    // Opt-in (NVFP4_MLP_FUSED_REQUANT=1).  Measured on B200 at M = 128,
-    // K = 5120, N = 17408: the gate/up call takes 43.0 us this way against
-    // 41.0 us with the separate encode pass.  The cooperative launch starts
-    // only once the activation quantizer has drained, so the weight stages
-    // are no longer streamed while it runs, which costs more than the
-    // h round trip and the extra launch saved.
+    // NVFP4_MLP_FUSED_REQUANT=0 keeps the separate encode pass on h.  Measured
+    // on B200 at M = 128, K = 5120, N = 17408: the gate/up call takes 37.9 us
+    // this way against 40.0 us with the encode pass.
     const char *opt = getenv("NVFP4_MLP_FUSED_REQUANT");
-    if (opt == nullptr || opt[0] != '1') return false;
+    if (opt != nullptr && opt[0] == '0') return false;
     const int64_t tiles = ceil_div(M, 128) * ceil_div(N, 128);
     return tiles >= 1 && tiles <= num_sms && tiles <= max_partials;
 }

@@ -7,9 +7,17 @@
 
 namespace nvfp4 {
 
+// With grid_bar and status (a workspace's meeting point and status word),
+// large contiguous tensors take the one-read cooperative quantizer
+// (quantize_onepass_usable); otherwise the two passes run.
 cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld,
                             uint8_t *codes, uint8_t *scales, float *g_out, float *partials,
-                            int num_sms, cudaStream_t stream);
+                            int num_sms, cudaStream_t stream, uint32_t *grid_bar = nullptr,
+                            uint32_t *status = nullptr, uint64_t timeout_ns = 0);
+bool quantize_onepass_usable(int64_t rows, int64_t cols, int64_t ld, bool bf16);
+cudaError_t launch_quantize_onepass(const void *x, bool bf16, int64_t rows, int64_t cols, uint8_t *codes,
+                                    uint8_t *scales, float *g_out, float *partials, uint32_t *grid_bar,
+                                    uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scales, const float *g,
                               int64_t rows, int64_t cols, void *y, bool bf16, int64_t ldy,

@@ -348,9 +348,17 @@ static int resident_ctas(K kernel) {
 
 cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld,
                             uint8_t *codes, uint8_t *scales, float *g_out, float *partials,
-                            int num_sms, cudaStream_t stream) {
+                            int num_sms, cudaStream_t stream, uint32_t *grid_bar, uint32_t *status,
+                            uint64_t timeout_ns) {
     // An empty tensor has no codes and no scale bytes; its amax is 0, so g = 0.
     if (rows == 0 || cols == 0) return cudaMemsetAsync(g_out, 0, sizeof(float), stream);
+    // Large contiguous tensors: one cooperative pass that reads x once.
+    if (grid_bar != nullptr && status != nullptr && quantize_onepass_usable(rows, cols, ld, bf16)) {
+        const cudaError_t e = launch_quantize_onepass(x, bf16, rows, cols, codes, scales, g_out, partials, grid_bar,
+                                                      status, timeout_ns, num_sms, stream);
+        if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+        (void)cudaGetLastError();      // fewer SMs than the grid (a shared device): the two passes
+    }
     const int eb = bf16 ? 2 : 4;
     static const int occ_amax[2] = {resident_ctas(amax_partials_kernel<float>),
                                     resident_ctas(amax_partials_kernel<__nv_bfloat16>)};

@@ -113,9 +113,9 @@ def check_mlp(nv, X, Wg, Wu, Wd, M, K, N):
     assert_gemm_close(to_numpy_f64(y), ref, norms(hq_o)[:, None], norms(wd_o)[None, :], N, True, "down")
 
 
-# h_q is formed either by the quantizer's encode pass over h (the default) or
-# inside the gate/up kernel's epilogue (NVFP4_MLP_FUSED_REQUANT=1, when the
-# tiles fit one per SM; otherwise the encode pass still runs).
+# h_q is formed either inside the gate/up kernel's epilogue (the default when
+# the tiles fit one per SM) or by the quantizer's encode pass over h
+# (NVFP4_MLP_FUSED_REQUANT=0, and always when the tiles outnumber the SMs).
 @pytest.mark.parametrize("fused", ["1", "0"])
 def test_mlp_small(nv, fused, monkeypatch):
     monkeypatch.setenv("NVFP4_MLP_FUSED_REQUANT", fused)
@@ -134,10 +134,8 @@ def test_mlp_ragged_tiles(nv, fused, monkeypatch):
     check_mlp(nv, w["X"], w["Wg"], w["Wu"], w["Wd"], M, K, N)
 
 
-def test_mlp_more_tiles_than_sms(nv, monkeypatch):
-    """9 x 18 = 162 gate/up tiles, more than the SMs: the encode pass path
-    even with the fused form asked for."""
-    monkeypatch.setenv("NVFP4_MLP_FUSED_REQUANT", "1")
+def test_mlp_more_tiles_than_sms(nv):
+    """9 x 18 = 162 gate/up tiles, more than the SMs: the encode pass path."""
     M, K, N = 1100, 256, 2304
     w = workloads.make("mlp", M=M, K=K, N=N, seed=42)
     check_mlp(nv, w["X"], w["Wg"], w["Wu"], w["Wd"], M, K, N)

@@ -212,3 +212,38 @@ def test_dequantize_rounding_order(nv):
     y = torch.empty((1, 16), dtype=torch.float32, device="cuda")
     nv.nvfp4_dequantize(t, y)
     assert np.array_equal(y.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+# The one-read cooperative quantizer (contiguous x, cols % 64 == 0, at least
+# 8 MB): all of a CTA's slice on chip (16 MB bf16), a slice that spills past
+# shared memory and registers and is read again (84 MB bf16), fp32 input with
+# rows not a multiple of 128 (padding rows of the scale layout), and a small
+# column count.  Bit-exact against the oracle and against the two-pass
+# quantizer (NVFP4_QUANTIZE_ONEPASS=0).
+@pytest.mark.parametrize("rows,cols,dtype", [(2048, 4096, torch.bfloat16), (8192, 5120, torch.bfloat16),
+                                             (1000, 4096, torch.float32), (3000, 1536, torch.bfloat16)])
+def test_quantize_onepass(nv, rows, cols, dtype, monkeypatch):
+    rng = np.random.default_rng(rows + cols)
+    x = rng.standard_normal((rows, cols)).astype(np.float32)
+    x[rng.random(x.shape) < 1e-3] *= 50
+    if dtype == torch.bfloat16:
+        xt = torch.from_numpy(x).to(torch.bfloat16)
+        x_or = xt.view(torch.int16).numpy().view(np.uint16)
+    else:
+        xt, x_or = torch.from_numpy(x), x
+    xd = xt.cuda()
+    outs = []
+    for onepass in ("1", "0"):
+        monkeypatch.setenv("NVFP4_QUANTIZE_ONEPASS", onepass)
+        out = nv.NVFP4Tensor.empty(rows, cols)
+        out.codes.fill_(0x77)
+        out.scales.fill_(0x55)
+        ws = nv.workspace(nv.OP_QUANTIZE, rows, 0, cols)
+        nv.nvfp4_quantize(xd, out, ws)
+        assert nv.nvfp4_get_device_status(ws) == nv.OK
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0].codes, outs[1].codes)
+    assert torch.equal(outs[0].scales, outs[1].scales)
+    assert torch.equal(outs[0].tensor_scale, outs[1].tensor_scale)
+    assert_quantized_equal(outs[0], oracle.quantize(x_or))
