@@ -92,7 +92,9 @@ typedef enum {
     NVFP4_ERR_WORKSPACE = 4,             /* ws NULL or smaller than required */
     NVFP4_ERR_CUDA = 5,                  /* a CUDA runtime/driver call or launch failed */
     NVFP4_ERR_TIMEOUT = 6,               /* a device-side bounded wait gave up */
-    NVFP4_ERR_ARCH = 7                   /* current device is not sm_100 */
+    NVFP4_ERR_ARCH = 7,                  /* current device is not sm_100 */
+    NVFP4_ERR_BOUNDS = 8                 /* debug build only (libnvfp4_debug.so): a kernel's store
+                                            fell outside its buffer and was skipped */
 } nvfp4_status;
 
 typedef enum {

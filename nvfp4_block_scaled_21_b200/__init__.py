@@ -13,7 +13,10 @@ import os
 from dataclasses import dataclass
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
+# NVFP4_LIBRARY=debug loads the debug build, whose kernels check every direct
+# global store against its buffer (ERR_BOUNDS in the status word on a miss).
+DEBUG_BUILD = os.environ.get("NVFP4_LIBRARY", "") == "debug"
+LIB_PATH = os.path.join(_PKG, "libnvfp4_debug.so" if DEBUG_BUILD else "libnvfp4.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -24,7 +27,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 # status codes (include/nvfp4.h)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_WORKSPACE, ERR_CUDA, \
-    ERR_TIMEOUT, ERR_ARCH = range(8)
+    ERR_TIMEOUT, ERR_ARCH, ERR_BOUNDS = range(9)
 F32, BF16 = 0, 1
 OP_QUANTIZE, OP_DEQUANTIZE, OP_GEMM, OP_LINEAR_FUSED, OP_LINEAR_FUSED_SILU, OP_GEMM_REQUANT, OP_W4A16, \
     OP_W4A8_LINEAR = range(8)

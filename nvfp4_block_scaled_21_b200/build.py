@@ -12,6 +12,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libnvfp4.so")
+# the same sources with every kernel's direct global stores bounds-checked
+DEBUG_LIB = os.path.join(PKG, "libnvfp4_debug.so")
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
@@ -38,30 +40,35 @@ def deps():
     return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "nvfp4.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(d) <= t for d in deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Build libnvfp4.so, or with debug=True libnvfp4_debug.so (NVFP4_DEBUG_CHECKS)."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    extra = ["-DNVFP4_DEBUG_CHECKS"] if debug else []
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
     res = subprocess.run(cmd, capture_output=True, text=True)
     log = res.stdout + res.stderr
-    with open(os.path.join(PKG, "build.log"), "w") as f:
+    with open(os.path.join(PKG, "build_debug.log" if debug else "build.log"), "w") as f:
         f.write(" ".join(cmd) + "\n" + log)
     if res.returncode != 0:
         sys.stderr.write(log)
-        raise RuntimeError("nvcc failed building libnvfp4.so")
+        raise RuntimeError(f"nvcc failed building {os.path.basename(lib)}")
     if verbose:
         sys.stderr.write(log)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True)
+    if "--debug" in sys.argv:
+        build(force="--force" in sys.argv, debug=True)

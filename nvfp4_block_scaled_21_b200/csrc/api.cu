@@ -207,9 +207,10 @@ static nvfp4_status zero_quantized(const nvfp4_tensor *q, cudaStream_t stream) {
 // The quantizer's encode pass on y as stored, from the per-CTA maxima the
 // GEMM's epilogue wrote: y_q gets its own tensor scale over all of y.
 static nvfp4_status requant_output(const void *y, nvfp4_dtype yt, int64_t ldy, const nvfp4_tensor *y_q,
-                                   const float *partials, int nparts, int num_sms, cudaStream_t stream) {
+                                   const float *partials, int nparts, int num_sms, cudaStream_t stream,
+                                   uint32_t *status) {
     return from_cuda(launch_encode(y, yt == NVFP4_BF16, y_q->rows, y_q->cols, ldy, partials, nparts,
-                                   y_q->codes, y_q->scales, y_q->tensor_scale, num_sms, stream));
+                                   y_q->codes, y_q->scales, y_q->tensor_scale, num_sms, stream, status));
 }
 
 // weights_ready: b was not written by the kernel launched just before (true
@@ -235,7 +236,7 @@ static nvfp4_status gemm_impl(const nvfp4_tensor *a, const nvfp4_tensor *b, void
                                                   wait_timeout_ns(), num_sms, stream, weights_ready, splitk,
                                                   y_q ? partials : nullptr, y_q ? &nparts : nullptr));
     if (st != NVFP4_OK || !y_q) return st;
-    return requant_output(y, yt, ldy, y_q, partials, nparts, num_sms, stream);
+    return requant_output(y, yt, ldy, y_q, partials, nparts, num_sms, stream, status);
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor *a, const nvfp4_tensor *b, void *y, nvfp4_dtype yt,
@@ -314,7 +315,7 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
                                           x_q ? x_q->tensor_scale : nullptr, status, wait_timeout_ns(), dev.sms,
                                           stream, y_q ? partials : nullptr, y_q ? &nparts : nullptr));
         if (st != NVFP4_OK || !y_q) return st;
-        return requant_output(y, yt, ldy, y_q, partials, nparts, dev.sms, stream);
+        return requant_output(y, yt, ldy, y_q, partials, nparts, dev.sms, stream, status);
     }
 
     // Quantized activations: caller's buffers or carved from the workspace.
@@ -380,7 +381,7 @@ nvfp4_status nvfp4_linear_fused(const void *x, nvfp4_dtype xt, int64_t M, int64_
                               wait_timeout_ns(), dev.sms, stream, true, nullptr, nullptr, nullptr, nullptr) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     return from_cuda(launch_encode_f32(h, M, N, ldh, partials, nparts, y_q->codes, y_q->scales,
-                                       y_q->tensor_scale, dev.sms, stream));
+                                       y_q->tensor_scale, dev.sms, stream, status));
 }
 
 // ---------------------------------------------------------------------------
@@ -620,6 +621,7 @@ const char *nvfp4_status_string(nvfp4_status s) {
     case NVFP4_ERR_CUDA: return "CUDA error";
     case NVFP4_ERR_TIMEOUT: return "device-side wait timed out";
     case NVFP4_ERR_ARCH: return "device is not sm_100";
+    case NVFP4_ERR_BOUNDS: return "device-side store out of bounds (debug build)";
     }
     return "unknown status";
 }

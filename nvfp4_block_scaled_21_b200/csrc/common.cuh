@@ -65,4 +65,30 @@ template <> __device__ __forceinline__ void YMax::add<__nv_bfloat16>(__nv_bfloat
 constexpr size_t kWsStatusBytes = 256;
 constexpr int kMaxAmaxPartials = 4096;
 
+// Debug build (compiled with NVFP4_DEBUG_CHECKS): every direct global store
+// of the kernels is checked against the extent of the buffer it writes; a
+// store that would leave it is skipped and NVFP4_ERR_BOUNDS is recorded in
+// the status word (no trap).  In the release build the check compiles away.
+constexpr uint32_t kStatusBoundsBit = 1u << 8;      // bit index == NVFP4_ERR_BOUNDS
+#ifdef NVFP4_DEBUG_CHECKS
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ bool store_ok(const void *p, size_t bytes, const void *base, size_t extent,
+                                         uint32_t *status) {
+    if constexpr (!kDebugChecks) {
+        return true;
+    } else {
+        const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(base);
+        const bool ok = a >= b && a + bytes <= b + extent;
+        if (!ok && status != nullptr) atomicOr(status, kStatusBoundsBit);
+        return ok;
+    }
+}
+// Bytes of a row-major [rows][cols] matrix with row pitch ld (elements of eb bytes).
+__host__ __device__ __forceinline__ size_t matrix_extent(int64_t rows, int64_t cols, int64_t ld, int64_t eb) {
+    return rows <= 0 || cols <= 0 ? 0 : static_cast<size_t>(((rows - 1) * ld + cols) * eb);
+}
+
 }  // namespace nvfp4

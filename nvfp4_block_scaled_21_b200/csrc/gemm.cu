@@ -488,6 +488,10 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int row = quarter * 32 + lane;        // accumulator row (MMA M index)
         const float alpha = __fmul_rn(args.ga ? *args.ga : 1.0f, args.gb ? *args.gb : 1.0f);   // MXFP4: none
         constexpr bool kFastDrain = !SWAP && sizeof(OutT) == 2 && BN >= 64;
+        // debug-build store checks: y is [M][N] with pitch ldy (M = Q when swapped)
+        const size_t y_bytes = matrix_extent(SWAP ? args.Q : args.P, SWAP ? args.P : args.Q, args.ldy, sizeof(OutT));
+        const size_t acc_bytes = static_cast<size_t>(args.num_p_tiles) * 128 * args.q_pad * sizeof(float);
+        auto y_ok = [&](const void *ptr, size_t bytes) { return store_ok(ptr, bytes, args.y, y_bytes, args.status); };
         uint32_t acc = 0, acc_phase = 0;
         uint32_t npart = 0;      // partial (stream-K) work items so far: epi_done/epi_flag phase
         // Largest |y| this thread stores.  Accumulator rows and columns past P
@@ -525,8 +529,9 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         tmem_ld_acc<CH, NACC, BN>(tbase + c0 + c * CH, nvalid, r);
 #pragma unroll
                         for (int i = 0; i < CH; i += 4)
-                            red_add_v4_f32(accrow + c * CH + i, __uint_as_float(r[i]), __uint_as_float(r[i + 1]),
-                                           __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+                            if (store_ok(accrow + c * CH + i, 16, args.acc_ws, acc_bytes, args.status))
+                                red_add_v4_f32(accrow + c * CH + i, __uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                                               __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
                     }
                 }
                 tc_fence_before();
@@ -584,7 +589,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                             const int q = qt * BN + lane * 4;
                             if (pr < args.P && lane * 4 < BN) {
                                 OutT *dst = y + static_cast<int64_t>(pr) * args.ldy + q;
-                                if (q + 4 <= args.Q) {
+                                if (q + 4 <= args.Q && y_ok(dst, 4 * sizeof(OutT))) {
                                     if constexpr (sizeof(OutT) == 2) {
                                         __nv_bfloat162 lo = __floats2bfloat162_rn(v0, v1);
                                         __nv_bfloat162 hi = __floats2bfloat162_rn(v2, v3);
@@ -596,11 +601,11 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                                         *reinterpret_cast<float4 *>(dst) = make_float4(v0, v1, v2, v3);
                                         ym.f32(v0); ym.f32(v1); ym.f32(v2); ym.f32(v3);
                                     }
-                                } else {
+                                } else if (q + 4 > args.Q) {
                                     const float vv[4] = {v0, v1, v2, v3};
 #pragma unroll
                                     for (int k = 0; k < 4; ++k)
-                                        if (q + k < args.Q) {
+                                        if (q + k < args.Q && y_ok(dst + k, sizeof(OutT))) {
                                             const OutT o = to_out<OutT>(vv[k]);
                                             dst[k] = o;
                                             ym.add<OutT>(o);
@@ -626,7 +631,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                                 const int rr = lane + 32 * i;
                                 const int pr = pt * 128 + rr;
                                 const float o = __fmul_rn(v[j][i], alpha);
-                                if (pr < args.P && q < args.Q) {
+                                if (pr < args.P && q < args.Q && y_ok(y + static_cast<int64_t>(q) * args.ldy + pr, sizeof(OutT))) {
                                     const OutT oo = to_out<OutT>(o);
                                     y[static_cast<int64_t>(q) * args.ldy + pr] = oo;
                                     ym.add<OutT>(oo);
@@ -659,16 +664,18 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     const int q0 = qt * BN + half * HC + c * 32;
                     if (p < args.P) {
                         if (q0 + 32 <= args.Q) {
+                            if (y_ok(yrow + q0, 32 * sizeof(OutT))) {
 #pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                *reinterpret_cast<uint4 *>(yrow + q0 + 8 * i) =
-                                    make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                                for (int i = 0; i < 4; ++i)
+                                    *reinterpret_cast<uint4 *>(yrow + q0 + 8 * i) =
+                                        make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                            }
                         } else {
 #pragma unroll
                             for (int i = 0; i < 16; ++i) {
-                                if (q0 + 2 * i < args.Q)
+                                if (q0 + 2 * i < args.Q && y_ok(yrow + q0 + 2 * i, 2))
                                     reinterpret_cast<unsigned short *>(yrow)[q0 + 2 * i] = static_cast<unsigned short>(pk[i] & 0xffffu);
-                                if (q0 + 2 * i + 1 < args.Q)
+                                if (q0 + 2 * i + 1 < args.Q && y_ok(yrow + q0 + 2 * i + 1, 2))
                                     reinterpret_cast<unsigned short *>(yrow)[q0 + 2 * i + 1] = static_cast<unsigned short>(pk[i] >> 16);
                             }
                         }
@@ -712,7 +719,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
                                 for (int i = 0; i < CH; ++i) {
                                     const int q = q0 + i;
-                                    if (q < args.Q) {
+                                    if (q < args.Q && y_ok(y + static_cast<int64_t>(q) * args.ldy + p, sizeof(OutT))) {
                                         if constexpr (sizeof(OutT) == 2)
                                             y[static_cast<int64_t>(q) * args.ldy + p] = __float2bfloat16_rn(v[i]);
                                         else
@@ -724,7 +731,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                             // y[p][q0 .. q0+CH): one contiguous run per thread
                             if (p < args.P) {
                                 OutT *yrow = static_cast<OutT *>(args.y) + static_cast<int64_t>(p) * args.ldy;
-                                if (q0 + CH <= args.Q) {
+                                if (q0 + CH <= args.Q && y_ok(yrow + q0, CH * sizeof(OutT))) {
                                     if constexpr (sizeof(OutT) == 2) {
 #pragma unroll
                                         for (int i = 0; i < CH; i += 8) {
@@ -743,10 +750,10 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                                             *reinterpret_cast<float4 *>(yrow + q0 + i) =
                                                 make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
                                     }
-                                } else {
+                                } else if (q0 + CH > args.Q) {
 #pragma unroll
                                     for (int i = 0; i < CH; ++i) {
-                                        if (q0 + i < args.Q) {
+                                        if (q0 + i < args.Q && y_ok(yrow + q0 + i, sizeof(OutT))) {
                                             if constexpr (sizeof(OutT) == 2)
                                                 yrow[q0 + i] = __float2bfloat16_rn(v[i]);
                                             else

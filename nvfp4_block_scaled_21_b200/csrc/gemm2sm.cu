@@ -80,9 +80,11 @@ struct PairCfg {
 };
 
 // (columns past N are exact zeros: folding them into ym cannot raise it)
+// (y_base, y_bytes, status: the debug build's store checks)
 template <typename OutT>
 __device__ __forceinline__ void pair_store_chunk(const uint32_t (&r)[32], float alpha, OutT *yrow,
-                                                 int q0, int N, YMax &ym) {
+                                                 int q0, int N, YMax &ym, const void *y_base, size_t y_bytes,
+                                                 uint32_t *status) {
     if constexpr (sizeof(OutT) == 2) {
         uint32_t pk[16];
 #pragma unroll
@@ -93,16 +95,18 @@ __device__ __forceinline__ void pair_store_chunk(const uint32_t (&r)[32], float 
             ym.bf16x2(pk[k]);
         }
         if (q0 + 32 <= N) {
+            if (store_ok(yrow + q0, 64, y_base, y_bytes, status)) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<uint4 *>(yrow + q0 + 8 * i) =
-                    make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                for (int i = 0; i < 4; ++i)
+                    *reinterpret_cast<uint4 *>(yrow + q0 + 8 * i) =
+                        make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
         } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                if (q0 + 2 * i < N)
+                if (q0 + 2 * i < N && store_ok(yrow + q0 + 2 * i, 2, y_base, y_bytes, status))
                     reinterpret_cast<unsigned short *>(yrow)[q0 + 2 * i] = static_cast<unsigned short>(pk[i] & 0xffffu);
-                if (q0 + 2 * i + 1 < N)
+                if (q0 + 2 * i + 1 < N && store_ok(yrow + q0 + 2 * i + 1, 2, y_base, y_bytes, status))
                     reinterpret_cast<unsigned short *>(yrow)[q0 + 2 * i + 1] = static_cast<unsigned short>(pk[i] >> 16);
             }
         }
@@ -110,7 +114,7 @@ __device__ __forceinline__ void pair_store_chunk(const uint32_t (&r)[32], float 
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const float v = __fmul_rn(__uint_as_float(r[i]), alpha);
-            if (q0 + i < N) yrow[q0 + i] = v;
+            if (q0 + i < N && store_ok(yrow + q0 + i, 4, y_base, y_bytes, status)) yrow[q0 + i] = v;
             ym.f32(v);
         }
     }
@@ -378,7 +382,8 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                     OutT *yrow = static_cast<OutT *>(args.y) + static_cast<int64_t>(p) * args.ldy;
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
-                        pair_store_chunk<OutT>(r[c], alpha, yrow, qn * 256 + half * 128 + c * 32, args.N, ym);
+                        pair_store_chunk<OutT>(r[c], alpha, yrow, qn * 256 + half * 128 + c * 32, args.N, ym, args.y,
+                                               matrix_extent(args.M, args.N, args.ldy, sizeof(OutT)), args.status);
                 }
             }
             return true;

@@ -352,7 +352,9 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                                                    8 * (kb & 1)) = cw;
                         if ((lane & 3) == 0) sfw[gq * 16 + r] = word;
                         if (write_xq)
-                            *reinterpret_cast<uint2 *>(args.xq_codes + static_cast<int64_t>(r) * (args.K / 2) + kb * 8) = cw;
+                            if (store_ok(args.xq_codes + static_cast<int64_t>(r) * (args.K / 2) + kb * 8, 8, args.xq_codes,
+                                         static_cast<size_t>(args.M) * (args.K / 2), args.status))
+                                *reinterpret_cast<uint2 *>(args.xq_codes + static_cast<int64_t>(r) * (args.K / 2) + kb * 8) = cw;
                     }
                 }
             }
@@ -384,8 +386,9 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
             for (int i = qt; i < ksteps * 32; i += C::kQThreads) {
                 const int gq = i >> 5, l = i & 31;
                 const uint32_t w0 = l < C::kN ? sfw[gq * 16 + l] : 0u;
-                *reinterpret_cast<uint4 *>(args.xq_scales + static_cast<int64_t>(gq) * 512 + l * 16) =
-                    make_uint4(w0, 0u, 0u, 0u);
+                uint8_t *sp = args.xq_scales + static_cast<int64_t>(gq) * 512 + l * 16;
+                if (store_ok(sp, 16, args.xq_scales, static_cast<size_t>(ksteps) * 512, args.status))
+                    *reinterpret_cast<uint4 *>(sp) = make_uint4(w0, 0u, 0u, 0u);
             }
         }
 
@@ -466,7 +469,9 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                     OutT *y = static_cast<OutT *>(args.y);
 #pragma unroll
                     for (int i = 0; i < C::kN; ++i) {
-                        if (i < args.M) {
+                        if (i < args.M &&
+                            store_ok(y + static_cast<int64_t>(i) * args.ldy + p, sizeof(OutT), args.y,
+                                     matrix_extent(args.M, args.N, args.ldy, sizeof(OutT)), args.status)) {
                             const OutT o = to_out<OutT>(__fmul_rn(r[i], alpha));
                             y[static_cast<int64_t>(i) * args.ldy + p] = o;
                             ym.add<OutT>(o);

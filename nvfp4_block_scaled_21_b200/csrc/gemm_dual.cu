@@ -327,14 +327,18 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                 }
                 const int q0 = qt * 128 + half * 64 + c * 32;
                 if (args.h != nullptr && p < args.M) {
+                    const size_t h_bytes = matrix_extent(args.M, args.N, args.ldh, 4);   // debug-build checks
                     if (q0 + 32 <= args.N) {
+                        if (store_ok(hrow + q0, 128, args.h, h_bytes, args.status)) {
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4 *>(hrow + q0 + i) = make_float4(h[i], h[i + 1], h[i + 2], h[i + 3]);
+                            for (int i = 0; i < 32; i += 4)
+                                *reinterpret_cast<float4 *>(hrow + q0 + i) = make_float4(h[i], h[i + 1], h[i + 2], h[i + 3]);
+                        }
                     } else {
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
-                            if (q0 + i < args.N) hrow[q0 + i] = h[i];
+                            if (q0 + i < args.N && store_ok(hrow + q0 + i, 4, args.h, h_bytes, args.status))
+                                hrow[q0 + i] = h[i];
                     }
                 }
             }
@@ -399,16 +403,19 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                                                          exact_only);
                     const uint2 cw = block_codes<float, 16>(w, block_rcp(sb, g));
                     word |= sb << (8 * b);
-                    if (p < args.M && kb0 + b < nblk)
-                        *reinterpret_cast<uint2 *>(args.hq_codes + static_cast<int64_t>(p) * (args.N / 2) +
-                                                   (kb0 + b) * 8) = cw;
+                    uint8_t *cp = args.hq_codes + static_cast<int64_t>(p) * (args.N / 2) + (kb0 + b) * 8;
+                    if (p < args.M && kb0 + b < nblk &&
+                        store_ok(cp, 8, args.hq_codes, static_cast<size_t>(args.M) * (args.N / 2), args.status))
+                        *reinterpret_cast<uint2 *>(cp) = cw;
                 }
                 // rows past M and blocks past N/16 are zero blocks: byte 0, the
                 // layout's padding value; blocks past kb4 are outside it
                 if (kb0 < args.kb4) {
                     const int64_t off = (static_cast<int64_t>(p >> 7) * (args.kb4 / 4) + (kb0 >> 2)) * 512 +
                                         (p & 31) * 16 + ((p >> 5) & 3) * 4;
-                    *reinterpret_cast<uint32_t *>(args.hq_scales + off) = word;
+                    if (store_ok(args.hq_scales + off, 4, args.hq_scales,
+                                 static_cast<size_t>(round_up(args.M, 128)) * args.kb4, args.status))
+                        *reinterpret_cast<uint32_t *>(args.hq_scales + off) = word;
                 }
             }
         }

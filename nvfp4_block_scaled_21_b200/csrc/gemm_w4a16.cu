@@ -349,7 +349,8 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
 #pragma unroll
                 for (int i = 0; i < C::kN; ++i) {
                     const int m = xt * C::kN + i;
-                    if (m < args.M)
+                    if (m < args.M && store_ok(y + static_cast<int64_t>(m) * args.ldy + p, sizeof(OutT), args.y,
+                                               matrix_extent(args.M, args.N, args.ldy, sizeof(OutT)), args.status))
                         y[static_cast<int64_t>(m) * args.ldy + p] = to_out<OutT>(__fmul_rn(__uint_as_float(acc[i]), gw));
                 }
             }

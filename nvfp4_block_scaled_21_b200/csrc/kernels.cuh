@@ -21,7 +21,7 @@ cudaError_t launch_quantize_onepass(const void *x, bool bf16, int64_t rows, int6
 
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scales, const float *g,
                               int64_t rows, int64_t cols, void *y, bool bf16, int64_t ldy,
-                              int num_sms, cudaStream_t stream);
+                              int num_sms, cudaStream_t stream, uint32_t *status = nullptr);
 
 // One GEMM operand as the GEMM kernel reads it.
 struct Operand {
@@ -89,13 +89,15 @@ cudaError_t launch_mx_quantize(const void *x, bool bf16, int64_t rows, int64_t c
 
 // The quantizer's second pass alone, on fp32 x whose first pass (max |x| per
 // part, num_partials values) was produced elsewhere.
+// status: the workspace status word (the debug build's store checks record
+// there), or null.
 cudaError_t launch_encode_f32(const float *x, int64_t rows, int64_t cols, int64_t ld, const float *partials,
                               int num_partials, uint8_t *codes, uint8_t *scales, float *g_out, int num_sms,
-                              cudaStream_t stream);
+                              cudaStream_t stream, uint32_t *status = nullptr);
 // The same for bf16 or fp32 x.
 cudaError_t launch_encode(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld, const float *partials,
                           int num_partials, uint8_t *codes, uint8_t *scales, float *g_out, int num_sms,
-                          cudaStream_t stream);
+                          cudaStream_t stream, uint32_t *status = nullptr);
 
 // h[M][N] = SiLU(x wg^T * gx*gwg) * (x wu^T * gx*gwu) in fp32 (128x128 tiles,
 // both products per tile), and max |h| per CTA into partials (the quantizer's

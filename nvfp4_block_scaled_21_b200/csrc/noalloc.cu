@@ -121,7 +121,7 @@ extern "C" nvfp4_status nvfp4_linear_noalloc(const void *x, nvfp4_dtype xt, int6
 
     if (cudaMemsetAsync(status, 0, sizeof(uint32_t), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (launch_quantize(x, xt == NVFP4_BF16, M, K, ldx, xq_codes, xq_scales, xq_g, partials, sms,
-                        stream) != cudaSuccess)
+                        stream, nullptr, status, wait_timeout_ns()) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     if (K == 0)
         return cudaMemset2DAsync(y, ldy * yeb, 0, N * yeb, M, stream) == cudaSuccess ? NVFP4_OK

@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, in
                                                      const float *__restrict__ partials,
                                                      int num_partials, uint8_t *__restrict__ codes,
                                                      uint8_t *__restrict__ scales,
-                                                     float *__restrict__ g_out) {
+                                                     float *__restrict__ g_out, uint32_t *status) {
     constexpr int W = sizeof(T) == 2 ? 8 : 16;        // 32-bit words per block
     const int64_t bpr = cols / kBlock;                  // blocks per row
     const int64_t total = rows * bpr;
@@ -152,6 +152,8 @@ __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, in
     const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int lane = threadIdx.x & 31;
     const bool word_scales = (cols % 64) == 0;
+    const size_t codes_bytes = static_cast<size_t>(rows * cols / 2);           // debug-build store checks
+    const size_t scales_bytes = static_cast<size_t>(round_up(rows, 128) * kb4);
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // let the GEMM queue up
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -210,12 +212,14 @@ __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, in
                 word |= __shfl_down_sync(0xffffffffu, sb, 2) << 16;
                 word |= __shfl_down_sync(0xffffffffu, sb, 3) << 24;
                 if (s0 + u < nstr && b < total32) {
-                    *reinterpret_cast<uint2 *>(codes + static_cast<size_t>(b) * 8) = cw;
+                    uint8_t *cp = codes + static_cast<size_t>(b) * 8;
+                    if (store_ok(cp, 8, codes, codes_bytes, status)) *reinterpret_cast<uint2 *>(cp) = cw;
                     const uint32_t off = ((r >> 7) * kb4q + (kb >> 2)) * 512u + (r & 31u) * 16u +
                                          ((r >> 5) & 3u) * 4u + (kb & 3u);
                     if (word_scales) {
-                        if ((lane & 3) == 0) *reinterpret_cast<uint32_t *>(scales + off) = word;
-                    } else {
+                        if ((lane & 3) == 0 && store_ok(scales + off, 4, scales, scales_bytes, status))
+                            *reinterpret_cast<uint32_t *>(scales + off) = word;
+                    } else if (store_ok(scales + off, 1, scales, scales_bytes, status)) {
                         scales[off] = static_cast<uint8_t>(sb);
                     }
                 }
@@ -246,12 +250,14 @@ __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, in
             word |= __shfl_down_sync(0xffffffffu, sb, 2) << 16;
             word |= __shfl_down_sync(0xffffffffu, sb, 3) << 24;
             if (valid) {
-                *reinterpret_cast<uint2 *>(codes + c.r * (cols / 2) + c.j * 8) = cw;
+                uint8_t *cp = codes + c.r * (cols / 2) + c.j * 8;
+                if (store_ok(cp, 8, codes, codes_bytes, status)) *reinterpret_cast<uint2 *>(cp) = cw;
+                uint8_t *sp = scales + scale_offset(c.r, c.j, kb4);
                 if (word_scales) {
-                    if ((lane & 3) == 0)
-                        *reinterpret_cast<uint32_t *>(scales + scale_offset(c.r, c.j, kb4)) = word;
-                } else {
-                    scales[scale_offset(c.r, c.j, kb4)] = static_cast<uint8_t>(sb);
+                    if ((lane & 3) == 0 && store_ok(sp, 4, scales, scales_bytes, status))
+                        *reinterpret_cast<uint32_t *>(sp) = word;
+                } else if (store_ok(sp, 1, scales, scales_bytes, status)) {
+                    *sp = static_cast<uint8_t>(sb);
                 }
             }
             c.advance(dr, dj, bpr);
@@ -265,11 +271,13 @@ __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, in
     const int64_t pad_b_words = (r128 - rows) * (kb4 / 4);
     for (int64_t i = t; i < pad_a; i += S) {
         const int64_t r = i / (kb4 - bpr), q = bpr + (i - r * (kb4 - bpr));
-        scales[scale_offset(r, q, kb4)] = 0;
+        uint8_t *sp = scales + scale_offset(r, q, kb4);
+        if (store_ok(sp, 1, scales, scales_bytes, status)) *sp = 0;
     }
     for (int64_t i = t; i < pad_b_words; i += S) {
         const int64_t r = rows + i / (kb4 / 4), q = 4 * (i % (kb4 / 4));
-        *reinterpret_cast<uint32_t *>(scales + scale_offset(r, q, kb4)) = 0u;
+        uint8_t *sp = scales + scale_offset(r, q, kb4);
+        if (store_ok(sp, 4, scales, scales_bytes, status)) *reinterpret_cast<uint32_t *>(sp) = 0u;
     }
 }
 
@@ -281,8 +289,9 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restri
                                                          const uint8_t *__restrict__ scales,
                                                          const float *__restrict__ g_ptr,
                                                          int64_t rows, int64_t cols,
-                                                         OutT *__restrict__ y, int64_t ldy) {
+                                                         OutT *__restrict__ y, int64_t ldy, uint32_t *status) {
     const int64_t ipr = cols / 8;
+    const size_t y_bytes = matrix_extent(rows, cols, ldy, sizeof(OutT));       // debug-build store checks
     const int64_t total = rows * ipr;
     const int64_t kb4 = kb4_of(cols);
     const float g = *g_ptr;
@@ -309,6 +318,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restri
             out[2 * k + 1] = __fmul_rn(__fmul_rn(e1, s), g);
         }
         OutT *dst = y + r * ldy + j * 8;
+        if (!store_ok(dst, 8 * sizeof(OutT), y, y_bytes, status)) continue;
         if constexpr (sizeof(OutT) == 2) {
             uint4 pk;
             uint32_t *p = reinterpret_cast<uint32_t *>(&pk);
@@ -392,15 +402,15 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
     if (bf16)
         return cudaLaunchKernelEx(&cfg, encode_kernel<__nv_bfloat16>,
                                   static_cast<const __nv_bfloat16 *>(x), rows, cols, ld,
-                                  static_cast<const float *>(partials), g1, codes, scales, g_out);
+                                  static_cast<const float *>(partials), g1, codes, scales, g_out, status);
     return cudaLaunchKernelEx(&cfg, encode_kernel<float>, static_cast<const float *>(x), rows,
                               cols, ld, static_cast<const float *>(partials), g1, codes, scales,
-                              g_out);
+                              g_out, status);
 }
 
 cudaError_t launch_encode(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld, const float *partials,
                           int num_partials, uint8_t *codes, uint8_t *scales, float *g_out, int num_sms,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, uint32_t *status) {
     static const int occ_encode[2] = {resident_ctas(encode_kernel<float>),
                                       resident_ctas(encode_kernel<__nv_bfloat16>)};
     const int g2 = quantize_grid(rows, cols, 1, num_sms, occ_encode[bf16]);
@@ -415,30 +425,31 @@ cudaError_t launch_encode(const void *x, bool bf16, int64_t rows, int64_t cols, 
     cfg.numAttrs = 1;
     if (bf16)
         return cudaLaunchKernelEx(&cfg, encode_kernel<__nv_bfloat16>, static_cast<const __nv_bfloat16 *>(x), rows,
-                                  cols, ld, partials, num_partials, codes, scales, g_out);
+                                  cols, ld, partials, num_partials, codes, scales, g_out, status);
     return cudaLaunchKernelEx(&cfg, encode_kernel<float>, static_cast<const float *>(x), rows, cols, ld, partials,
-                              num_partials, codes, scales, g_out);
+                              num_partials, codes, scales, g_out, status);
 }
 
 cudaError_t launch_encode_f32(const float *x, int64_t rows, int64_t cols, int64_t ld, const float *partials,
                               int num_partials, uint8_t *codes, uint8_t *scales, float *g_out, int num_sms,
-                              cudaStream_t stream) {
-    return launch_encode(x, false, rows, cols, ld, partials, num_partials, codes, scales, g_out, num_sms, stream);
+                              cudaStream_t stream, uint32_t *status) {
+    return launch_encode(x, false, rows, cols, ld, partials, num_partials, codes, scales, g_out, num_sms, stream,
+                         status);
 }
 
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scales, const float *g,
                               int64_t rows, int64_t cols, void *y, bool bf16, int64_t ldy,
-                              int num_sms, cudaStream_t stream) {
+                              int num_sms, cudaStream_t stream, uint32_t *status) {
     const int64_t items = rows * (cols / 8);
     int64_t blocks = ceil_div(items, 256);
     const int64_t cap = static_cast<int64_t>(num_sms) * 8;
     blocks = blocks < 1 ? 1 : (blocks < cap ? blocks : cap);
     if (bf16)
         dequantize_kernel<__nv_bfloat16><<<static_cast<int>(blocks), 256, 0, stream>>>(
-            codes, scales, g, rows, cols, static_cast<__nv_bfloat16 *>(y), ldy);
+            codes, scales, g, rows, cols, static_cast<__nv_bfloat16 *>(y), ldy, status);
     else
         dequantize_kernel<float><<<static_cast<int>(blocks), 256, 0, stream>>>(
-            codes, scales, g, rows, cols, static_cast<float *>(y), ldy);
+            codes, scales, g, rows, cols, static_cast<float *>(y), ldy, status);
     return cudaGetLastError();
 }
 

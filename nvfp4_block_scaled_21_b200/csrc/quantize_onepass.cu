@@ -98,6 +98,8 @@ __global__ void __launch_bounds__(kOpThreads, 1) quantize_onepass_kernel(const _
     const int R = min(nb - S, RB * T_);                        // in registers
     const int spill_lo = S + R;                                // read again in pass B
     const uint8_t *xb = static_cast<const uint8_t *>(a.x) + b0 * C::kBlockBytes;
+    const size_t codes_bytes = static_cast<size_t>(a.rows * a.cols / 2);          // debug-build store checks
+    const size_t scales_bytes = static_cast<size_t>(round_up(a.rows, 128) * kb4);
 
     if (t == 0) {
         mbar_init(&bar, 1);
@@ -221,11 +223,12 @@ __global__ void __launch_bounds__(kOpThreads, 1) quantize_onepass_kernel(const _
         word |= __shfl_down_sync(0xffffffffu, sb, 3) << 24;
         if (valid) {
             const int64_t b = b0 + i;
-            *reinterpret_cast<uint2 *>(a.codes + b * 8) = cw;
+            if (store_ok(a.codes + b * 8, 8, a.codes, codes_bytes, a.status)) *reinterpret_cast<uint2 *>(a.codes + b * 8) = cw;
             if ((lane & 3) == 0) {
                 const int64_t r = b / bpr, kb = b - r * bpr;
                 const int64_t off = ((r >> 7) * (kb4 >> 2) + (kb >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4;
-                *reinterpret_cast<uint32_t *>(a.scales + off) = word;
+                if (store_ok(a.scales + off, 4, a.scales, scales_bytes, a.status))
+                    *reinterpret_cast<uint32_t *>(a.scales + off) = word;
             }
         }
     };
@@ -275,8 +278,8 @@ __global__ void __launch_bounds__(kOpThreads, 1) quantize_onepass_kernel(const _
     const int64_t p_lo = pad_words * blockIdx.x / gridDim.x, p_hi = pad_words * (blockIdx.x + 1) / gridDim.x;
     for (int64_t i = p_lo + t; i < p_hi; i += T_) {
         const int64_t r = a.rows + i / (kb4 / 4), q = 4 * (i % (kb4 / 4));
-        *reinterpret_cast<uint32_t *>(a.scales + ((r >> 7) * (kb4 >> 2) + (q >> 2)) * 512 + (r & 31) * 16 +
-                                      ((r >> 5) & 3) * 4) = 0u;
+        uint8_t *sp = a.scales + ((r >> 7) * (kb4 >> 2) + (q >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4;
+        if (store_ok(sp, 4, a.scales, scales_bytes, a.status)) *reinterpret_cast<uint32_t *>(sp) = 0u;
     }
 }
 
