@@ -34,8 +34,8 @@ L2_BYTES = 126 * 1024 * 1024
 # from one ncu capture of the current kernels (dram__bytes_read.sum +
 # dram__bytes_write.sum); None where the kernel changed after its capture or
 # the capture did not cover every kernel of the dominant call.
-NCU_TRAFFIC = {"prefill": 157_946_112, "decode": 50_256_896, "quantize": 172_076_288, "mlp": 103_521_536,
-               "prefill_requant": 402_010_112, "mx_prefill": 153_014_272, "w4a16_decode": 50_272_000,
+NCU_TRAFFIC = {"prefill": 157_946_112, "decode": 50_256_896, "quantize": None, "mlp": None,
+               "prefill_requant": None, "mx_prefill": 153_014_272, "w4a16_decode": 50_272_000,
                "w4a8_prefill": 162_502_656}
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0

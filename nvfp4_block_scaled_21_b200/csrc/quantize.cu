@@ -15,6 +15,7 @@
 //   conversions; codes go out as one 8-byte store per block and scales as one
 //   32-bit word per four blocks in the tiled layout the tensor cores read.
 #include "common.cuh"
+#include <cstdlib>
 #include "encode.cuh"
 #include "kernels.cuh"
 
@@ -126,6 +127,43 @@ __device__ __forceinline__ float reduce_partials(const float *__restrict__ parti
     }
     __syncthreads();
     return result;
+}
+
+// ---------------------------------------------------------------------------
+// Zero the padding of the tiled scale layout: blocks kb in [bpr, kb4) of the
+// real rows (bytes) and every block of the rows [rows, roundup(rows, 128))
+// (32-bit words), as thread tid of nthr.  Each thread divides once and then
+// steps its (row, column) position incrementally.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void zero_scale_padding(uint8_t *scales, int64_t rows, int64_t bpr, int64_t kb4,
+                                                   int64_t tid, int64_t nthr, size_t scales_bytes,
+                                                   uint32_t *status) {
+    const int64_t npad = kb4 - bpr;                     // padded blocks per real row (0..3)
+    if (npad > 0) {
+        const int64_t total = rows * npad;
+        int64_t r = tid / npad, q = tid - r * npad;
+        const int64_t dr = nthr / npad, dq = nthr - dr * npad;
+        for (int64_t i = tid; i < total; i += nthr) {
+            uint8_t *sp = scales + scale_offset(r, bpr + q, kb4);
+            if (store_ok(sp, 1, scales, scales_bytes, status)) *sp = 0;
+            r += dr;
+            q += dq;
+            if (q >= npad) { q -= npad; ++r; }
+        }
+    }
+    const int64_t wpr = kb4 / 4;                        // scale words per row
+    const int64_t total_w = (round_up(rows, 128) - rows) * wpr;
+    if (total_w > 0) {
+        int64_t r = rows + tid / wpr, q = tid % wpr;
+        const int64_t dr = nthr / wpr, dq = nthr % wpr;
+        for (int64_t i = tid; i < total_w; i += nthr) {
+            uint8_t *sp = scales + ((r >> 7) * wpr + q) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4;
+            if (store_ok(sp, 4, scales, scales_bytes, status)) *reinterpret_cast<uint32_t *>(sp) = 0u;
+            r += dr;
+            q += dq;
+            if (q >= wpr) { q -= wpr; ++r; }
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -264,21 +302,7 @@ __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, in
         }
     }
 
-    // Zero the padding of the scale layout: blocks kb in [cols/16, kb4) of
-    // real rows, and every block of rows in [rows, roundup(rows, 128)).
-    const int64_t pad_a = rows * (kb4 - bpr);
-    const int64_t r128 = round_up(rows, 128);
-    const int64_t pad_b_words = (r128 - rows) * (kb4 / 4);
-    for (int64_t i = t; i < pad_a; i += S) {
-        const int64_t r = i / (kb4 - bpr), q = bpr + (i - r * (kb4 - bpr));
-        uint8_t *sp = scales + scale_offset(r, q, kb4);
-        if (store_ok(sp, 1, scales, scales_bytes, status)) *sp = 0;
-    }
-    for (int64_t i = t; i < pad_b_words; i += S) {
-        const int64_t r = rows + i / (kb4 / 4), q = 4 * (i % (kb4 / 4));
-        uint8_t *sp = scales + scale_offset(r, q, kb4);
-        if (store_ok(sp, 4, scales, scales_bytes, status)) *reinterpret_cast<uint32_t *>(sp) = 0u;
-    }
+    zero_scale_padding(scales, rows, bpr, kb4, t, S, scales_bytes, status);
 }
 
 // ---------------------------------------------------------------------------
