@@ -36,7 +36,7 @@ L2_BYTES = 126 * 1024 * 1024
 # the capture did not cover every kernel of the dominant call.
 NCU_TRAFFIC = {"prefill": 157_946_112, "decode": 50_256_896, "quantize": None, "mlp": None,
                "prefill_requant": None, "mx_prefill": 153_014_272, "w4a16_decode": 50_272_000,
-               "w4a8_prefill": 162_502_656}
+               "w4a8_prefill": 173_520_128}
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP4_PER_BF16 = 4.0          # dense FP4 : dense BF16 on B200 (9 : 2.25 PFLOP/s nominal)
@@ -491,7 +491,7 @@ class W4A8Prefill:
         self.flops = 2.0 * self.M * self.N * self.K
         self.units = self.flops / 1e12
         self.launches = 2                       # MXFP8 quantize, GEMM
-        self.dominant = {"kernel": "gemm_nvf4_kernel<W4A8> (kind::mxf8f6f4, one CTA, 128x256 tiles)",
+        self.dominant = {"kernel": "gemm_nvf4_pair_kernel<W4A8> (kind::mxf8f6f4, CTA pair, 256x256 tiles)",
                          "bound": "tensor", "algorithmic": self.flops, "unit": "TFLOP/s",
                          "per_bf16": FP8_PER_BF16, "peak_name": "dense FP8"}
         self.config = {"workload": f"W4A8 prefill linear: quantize X bf16 {self.M}x{self.K} to MXFP8 per call, "

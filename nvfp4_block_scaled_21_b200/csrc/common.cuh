@@ -10,6 +10,12 @@
 namespace nvfp4 {
 
 constexpr int kBlock = 16;           // values per microblock (NVFP4 wiki page, "技術原理")
+
+// Operand formats of the GEMM kernels.
+constexpr int kFmtNV = 0;     // NVFP4: E2M1 (packed), UE4M3 per 16, kind::mxf4nvf4 4X, K = 64 per MMA
+constexpr int kFmtMX = 1;     // MXFP4: E2M1 (packed), UE8M0 per 32, kind::mxf4 2X, K = 64 per MMA
+constexpr int kFmtW4A8 = 2;   // MXFP4 weights x MXFP8 activations (8-bit containers in shared memory),
+                              // UE8M0 per 32, kind::mxf8f6f4 1X, K = 32 per MMA
 constexpr float kTensorScaleDiv = 2688.0f;   // 6 (E2M1 max) * 448 (E4M3 max)
 
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }

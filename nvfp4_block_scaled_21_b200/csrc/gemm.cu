@@ -165,12 +165,6 @@ __device__ __forceinline__ void tmem_ld_acc(uint32_t taddr, int nvalid, uint32_t
     }
 }
 
-// Operand formats of the one-CTA kernel.
-constexpr int kFmtNV = 0;     // NVFP4: E2M1 (packed), UE4M3 per 16, kind::mxf4nvf4 4X, K = 64 per MMA
-constexpr int kFmtMX = 1;     // MXFP4: E2M1 (packed), UE8M0 per 32, kind::mxf4 2X, K = 64 per MMA
-constexpr int kFmtW4A8 = 2;   // MXFP4 weights x MXFP8 activations (8-bit containers in shared memory),
-                              // UE8M0 per 32, kind::mxf8f6f4 1X, K = 32 per MMA
-
 // Scale atoms (512 bytes: 128 rows x 4 blocks) per ring stage and per 128-row
 // tile.  A stage is four MMA K steps: 256 values of K for the FP4 kinds, 128
 // for W4A8, and always 128 bytes per operand row in shared memory.  NVFP4 has
@@ -1005,9 +999,8 @@ static cudaError_t launch_gemm_fmt(const Operand &act, const Operand &wgt, int64
         NVFP4_SWAPPED(64)
 #undef NVFP4_SWAPPED
     }
-    if (FMT != kFmtW4A8 && pair_gemm_usable(M, N, num_sms))
-        return launch_gemm_pair(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, stream, ymax_part, nparts,
-                                FMT == kFmtMX);
+    if (pair_gemm_usable(M, N, num_sms))
+        return launch_gemm_pair(act, wgt, K, y, y_bf16, ldy, status, timeout_ns, stream, ymax_part, nparts, FMT);
     const int64_t ptiles = ceil_div(M, 128);
     const bool wide = ptiles * ceil_div(N, 256) >= 2 * num_sms;
     if (wide)

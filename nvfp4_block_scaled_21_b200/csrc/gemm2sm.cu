@@ -49,7 +49,7 @@ struct PairArgs {
     void *y;
     int64_t ldy;
     int32_t M, N;
-    int32_t num_k_steps;     // K / 64
+    int32_t num_k_steps;     // MMA K steps: K / 64 (FP4 kinds) or K / 32 (W4A8)
     int32_t num_pm, num_qn;  // 256-row / 256-column pair tiles
     int32_t tma_store;       // bf16 output written by TMA stores (needs N % 8 == 0)
     float *ymax_part;        // if set: this CTA's largest |y| as stored, at [blockIdx.x]
@@ -120,13 +120,21 @@ __device__ __forceinline__ void pair_store_chunk(const uint32_t (&r)[32], float 
     }
 }
 
-template <typename OutT, bool MX>
+template <typename OutT, int FMT>
 __global__ void __launch_bounds__(PairCfg::kThreads, 1)
 gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                       const __grid_constant__ CUtensorMap tmY, const __grid_constant__ PairArgs args) {
     using C = PairCfg;
     constexpr int STAGES = C::kStages;
+    constexpr bool MX = FMT == kFmtMX;
+    constexpr bool W8 = FMT == kFmtW4A8;          // MXFP8 A (activations) x MXFP4 B (weights, unpacked)
+    // scale atoms per stage and 128-row tile: one per K step (NVFP4, K = 64),
+    // one per two (MXFP4), one per stage (W4A8: four K steps of 32)
+    constexpr int kAtoms = MX ? 2 : (W8 ? 1 : 4);
+    // operand bytes both CTAs' copies signal on the leader's barrier: the
+    // unpacking copy of the W4A8 weights counts the packed bytes it reads
+    constexpr uint32_t kFullTx = 2u * (W8 ? C::kAStage + C::kBStage / 2 : C::kABBytes);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
@@ -209,15 +217,13 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                     }
                     const uint32_t bar = leader_full0 + 8u * stage;
                     if (issue) {
-                        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kABBytes);
+                        if (leader) mbar_arrive_expect_tx(&full[stage], kFullTx);
                         tma_load_2d_pair(sA + stage * C::kAStage, &tmA, bar, ks * 128, a_rt * 128, pol);
                         tma_load_2d_pair(sB + stage * C::kBStage, &tmB, bar, ks * 128, b_rt * 128, pol);
-                        // scale atoms of this stage: 4 (NVFP4) or 2 (MXFP4) per 128-row tile
-                        mbar_arrive_expect_tx(&sfull[stage], MX ? C::kSfBytes / 2 : C::kSfBytes);
-                        tma_load_3d(sSfa + stage * C::kSfaStage, &tmSA, &sfull[stage], 0, (MX ? 2 : 4) * ks, a_rt,
-                                    pol);
-                        tma_load_3d(sSfb + stage * C::kSfbStage, &tmSB, &sfull[stage], 0, (MX ? 2 : 4) * ks, 2 * qn,
-                                    pol);
+                        // scale atoms of this stage: kAtoms per 128-row tile
+                        mbar_arrive_expect_tx(&sfull[stage], C::kSfBytes / (4 / kAtoms));
+                        tma_load_3d(sSfa + stage * C::kSfaStage, &tmSA, &sfull[stage], 0, kAtoms * ks, a_rt, pol);
+                        tma_load_3d(sSfb + stage * C::kSfbStage, &tmSB, &sfull[stage], 0, kAtoms * ks, 2 * qn, pol);
                     }
                     __syncwarp();
                     ++issued;
@@ -243,6 +249,8 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             // and commits.
             const uint32_t issue = elect_one_sync() ? 1u : 0u;
             constexpr uint32_t idesc = make_idesc_nvf4_pair(256);
+            constexpr uint32_t idesc_w8[4] = {make_idesc_mxf8f6f4_pair(256, 0, 5, 0), make_idesc_mxf8f6f4_pair(256, 0, 5, 1),
+                                              make_idesc_mxf8f6f4_pair(256, 0, 5, 2), make_idesc_mxf8f6f4_pair(256, 0, 5, 3)};
             constexpr uint32_t idesc_mx0 = make_idesc_mxf4(256, 256, 0), idesc_mx1 = make_idesc_mxf4(256, 256, 1);
             const uint32_t a_base = smem_addr(sA), b_base = smem_addr(sB);
             uint32_t stage = 0, phase = 0;
@@ -281,7 +289,10 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                         // MXFP4: K step j reads the columns of atom j/2 and
                         // its bytes {0,1} or {2,3} (descriptor's scale IDs)
                         auto kstep = [&](int j) {
-                            if constexpr (MX)
+                            if constexpr (W8)   // atom 0 of the slab, byte j (scale ID), E4M3 x E2M1
+                                mma_mxf8f6f4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, idesc_w8[j], sf, sf + 16,
+                                                  (ks | j) != 0 ? 1u : 0u, issue);
+                            else if constexpr (MX)
                                 mma_mxf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, (j & 1) ? idesc_mx1 : idesc_mx0,
                                               sf + 4 * (j >> 1), sf + 16 + 8 * (j >> 1), (ks | j) != 0 ? 1u : 0u, issue);
                             else
@@ -411,9 +422,9 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                             const uint8_t *a_src = sSfa + st_i * C::kSfaStage + lane * 16;
                             const uint8_t *b_src = sSfb + st_i * C::kSfbStage + lane * 16;
                             // the B box holds both row tiles' atoms, tile after tile:
-                            // 4 atoms each (NVFP4) or 2 (MXFP4, whose atom slots 2
-                            // and 3 hold bytes no MMA reads)
-                            constexpr int kTile1 = MX ? 1024 : 2048;
+                            // kAtoms each (the atom slots past kAtoms hold bytes no
+                            // MMA reads)
+                            constexpr int kTile1 = kAtoms * 512;
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 const uint4 a = ld_shared_v4(a_src + j * 512);
@@ -477,20 +488,29 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
 // Host side
 // ---------------------------------------------------------------------------
 
-template <typename OutT, bool MX>
+template <typename OutT, int FMT>
 static cudaError_t run_pair(const Operand &act, const Operand &wgt, int64_t K, void *y, int64_t ldy,
                             uint32_t *status, uint64_t timeout_ns, int max_clusters, cudaStream_t stream,
                             float *ymax_part, int *nparts) {
     using C = PairCfg;
-    const uint64_t k_steps = static_cast<uint64_t>(K / 64);
-    // 512-byte scale atoms per 128-row tile: one per K step (NVFP4), one per two (MXFP4)
-    const uint64_t atoms_rt = MX ? (k_steps + 1) / 2 : k_steps;
+    constexpr bool MX = FMT == kFmtMX, W8 = FMT == kFmtW4A8;
+    // MMA K steps: 64 values (FP4 kinds) or 32 (W4A8)
+    const uint64_t k_steps = static_cast<uint64_t>(W8 ? K / 32 : K / 64);
+    // 512-byte scale atoms per 128-row tile: one per K step (NVFP4), one per
+    // two (MXFP4), one per four (W4A8)
+    const uint64_t atoms_rt = W8 ? (k_steps + 3) / 4 : (MX ? (k_steps + 1) / 2 : k_steps);
+    const uint32_t box_atoms = W8 ? 1 : (MX ? 2 : 4);
     CUtensorMap tmA, tmB, tmSA, tmSB;
-    if (encode_tensor_map_u8(&tmA, act.codes, K / 2, act.rows, 128, 128) != CUDA_SUCCESS ||
-        encode_tensor_map_u8(&tmB, wgt.codes, K / 2, wgt.rows, 128, 128) != CUDA_SUCCESS ||
-        encode_scale_map(&tmSA, act.scales, atoms_rt, ceil_div(act.rows, 128), 1, MX ? 2 : 4) != CUDA_SUCCESS ||
-        encode_scale_map(&tmSB, wgt.scales, atoms_rt, ceil_div(wgt.rows, 128), 2, MX ? 2 : 4) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
+    // A rows of 128 bytes per stage: 256 E2M1 values, or 128 E4M3 values
+    // (W4A8); W4A8's E2M1 weights are unpacked by the copy into 8-bit
+    // containers, 128 values per 128-byte row
+    const bool maps_ok =
+        encode_tensor_map_u8(&tmA, act.codes, W8 ? K : K / 2, act.rows, 128, 128) == CUDA_SUCCESS &&
+        (W8 ? encode_tensor_map_fp4_unpacked(&tmB, wgt.codes, K, wgt.rows, 128)
+            : encode_tensor_map_u8(&tmB, wgt.codes, K / 2, wgt.rows, 128, 128)) == CUDA_SUCCESS &&
+        encode_scale_map(&tmSA, act.scales, atoms_rt, ceil_div(act.rows, 128), 1, box_atoms) == CUDA_SUCCESS &&
+        encode_scale_map(&tmSB, wgt.scales, atoms_rt, ceil_div(wgt.rows, 128), 2, box_atoms) == CUDA_SUCCESS;
+    if (!maps_ok) return cudaErrorInvalidValue;
     CUtensorMap tmY;
     memset(&tmY, 0, sizeof(tmY));    // unused unless tma_store
     const bool tma_store = sizeof(OutT) == 2 && wgt.rows % 8 == 0;
@@ -514,7 +534,7 @@ static cudaError_t run_pair(const Operand &act, const Operand &wgt, int64_t K, v
     a.timeout_ns = timeout_ns;
     const int tiles = a.num_pm * a.num_qn;
     const int clusters = tiles < max_clusters ? tiles : max_clusters;
-    cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_pair_kernel<OutT, MX>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_pair_kernel<OutT, FMT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -532,7 +552,7 @@ static cudaError_t run_pair(const Operand &act, const Operand &wgt, int64_t K, v
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<OutT, MX>, tmA, tmB, tmSA, tmSB, tmY, a);
+    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<OutT, FMT>, tmA, tmB, tmSA, tmSB, tmY, a);
 }
 
 // How many 2-CTA clusters of the pair kernel can be resident at once (0 if
@@ -541,7 +561,7 @@ static cudaError_t run_pair(const Operand &act, const Operand &wgt, int64_t K, v
 static int pair_max_clusters_query() {
     int n = 0;
     bool ok = true;
-    auto kb = gemm_nvf4_pair_kernel<__nv_bfloat16, false>;
+    auto kb = gemm_nvf4_pair_kernel<__nv_bfloat16, kFmtNV>;
     ok = ok && cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::kSmemBytes) == cudaSuccess;
     if (ok) {
         cudaLaunchConfig_t cfg = {};
@@ -577,14 +597,16 @@ bool pair_gemm_usable(int64_t M, int64_t N, int num_sms) {
 
 cudaError_t launch_gemm_pair(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
                              int64_t ldy, uint32_t *status, uint64_t timeout_ns, cudaStream_t stream,
-                             float *ymax_part, int *nparts, bool mx) {
+                             float *ymax_part, int *nparts, int fmt) {
     const int maxc = pair_max_clusters();
     if (maxc <= 0) return cudaErrorLaunchOutOfResources;
-    if (mx)
-        return y_bf16 ? run_pair<__nv_bfloat16, true>(act, wgt, K, y, ldy, status, timeout_ns, maxc, stream, ymax_part, nparts)
-                      : run_pair<float, true>(act, wgt, K, y, ldy, status, timeout_ns, maxc, stream, ymax_part, nparts);
-    return y_bf16 ? run_pair<__nv_bfloat16, false>(act, wgt, K, y, ldy, status, timeout_ns, maxc, stream, ymax_part, nparts)
-                  : run_pair<float, false>(act, wgt, K, y, ldy, status, timeout_ns, maxc, stream, ymax_part, nparts);
+#define NVFP4_PAIR(F)                                                                                              \
+    return y_bf16 ? run_pair<__nv_bfloat16, F>(act, wgt, K, y, ldy, status, timeout_ns, maxc, stream, ymax_part, nparts) \
+                  : run_pair<float, F>(act, wgt, K, y, ldy, status, timeout_ns, maxc, stream, ymax_part, nparts);
+    if (fmt == kFmtMX) { NVFP4_PAIR(kFmtMX) }
+    if (fmt == kFmtW4A8) { NVFP4_PAIR(kFmtW4A8) }
+    NVFP4_PAIR(kFmtNV)
+#undef NVFP4_PAIR
 }
 
 }  // namespace nvfp4

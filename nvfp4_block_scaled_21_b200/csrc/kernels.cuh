@@ -50,10 +50,11 @@ size_t splitk_ws_bytes(int64_t M, int64_t N);
 // Two-CTA (cta_group::2) GEMM for large M: usable when enough 256x256 tiles
 // exist to fill the GPU with CTA pairs.
 bool pair_gemm_usable(int64_t M, int64_t N, int num_sms);
-// mx: MXFP4 operands (UE8M0 scales per 32 elements) instead of NVFP4.
+// fmt: kFmtNV, kFmtMX (MXFP4 operands) or kFmtW4A8 (MXFP8 activations, MXFP4
+// weights read by the unpacking copy; K % 128 == 0).
 cudaError_t launch_gemm_pair(const Operand &act, const Operand &wgt, int64_t K, void *y, bool y_bf16,
                              int64_t ldy, uint32_t *status, uint64_t timeout_ns, cudaStream_t stream,
-                             float *ymax_part = nullptr, int *nparts = nullptr, bool mx = false);
+                             float *ymax_part = nullptr, int *nparts = nullptr, int fmt = 0);
 
 // y[M][N] = A . B^T for MXFP4 operands (E2M1 codes, UE8M0 scales per 32
 // elements in the tiled layout with 32-element blocks, no tensor scales).

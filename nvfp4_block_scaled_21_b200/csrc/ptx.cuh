@@ -443,6 +443,11 @@ __host__ __device__ constexpr uint32_t make_idesc_mxf4(uint32_t n, uint32_t m, u
 __host__ __device__ constexpr uint32_t make_idesc_mxf8f6f4(uint32_t n, uint32_t a_fmt, uint32_t b_fmt, uint32_t j) {
     return (a_fmt << 7) | (b_fmt << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24) | (j << 29) | (j << 4);
 }
+// The same for the pair MMA (M = 256).
+__host__ __device__ constexpr uint32_t make_idesc_mxf8f6f4_pair(uint32_t n, uint32_t a_fmt, uint32_t b_fmt,
+                                                                uint32_t j) {
+    return (a_fmt << 7) | (b_fmt << 10) | ((n >> 3) << 17) | (1u << 23) | ((256u >> 4) << 24) | (j << 29) | (j << 4);
+}
 
 // ---------------------------------------------------------------------------
 // Two-CTA (cluster of 2) forms: the pair shares one block-scaled MMA
@@ -523,6 +528,19 @@ __device__ __forceinline__ void mma_mxf4_pair(uint32_t d_tmem, uint64_t a_desc, 
         "setp.ne.b32 p, %4, 0;\n\t"
         "setp.ne.b32 q, %7, 0;\n\t"
         "@q " "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X"
+        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem), "r"(issue)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                  uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                  uint32_t accumulate, uint32_t issue = 1u) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, %7, 0;\n\t"
+        "@q " "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.scale_vec::1X"
         " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem), "r"(issue)
         : "memory");

@@ -215,3 +215,21 @@ def test_mlp_workload_full(nv):
     """The fused MLP workload at full size: M=128, K=5120, N=17408 (seed 4)."""
     w = workloads.make("mlp")
     check_mlp(nv, w["X"], w["Wg"], w["Wu"], w["Wd"], 128, 5120, 17408)
+
+
+def test_mlp_fused_requant_reuses_one_workspace_across_grids(nv):
+    """The in-epilogue form's grid meeting point lives in the workspace and must
+    be back at its start after every call: one workspace serves calls whose
+    grids have 3, 18 and 6 CTAs, in that order and twice, each h_q bit-exact
+    against the oracle's quantization of the GPU's own h."""
+    shapes = [(32, 256, 384), (160, 256, 1040), (200, 320, 320)] * 2
+    big = max(nv.workspace_bytes(nv.OP_LINEAR_FUSED_SILU, M, N, K) for M, K, N in shapes)
+    ws = torch.zeros(big, dtype=torch.uint8, device="cuda")
+    for i, (M, K, N) in enumerate(shapes):
+        w = workloads.make("mlp", M=M, K=K, N=N, seed=50 + i)
+        wg, wu = quantize_gpu(nv, bf16_tensor(w["Wg"])), quantize_gpu(nv, bf16_tensor(w["Wu"]))
+        h = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        h_q = nv.NVFP4Tensor.empty(M, N)
+        nv.nvfp4_linear_fused(bf16_tensor(w["X"]), wg, ws, nv.EPI_SILU_MUL_REQUANT, y=h, w_up=wu, y_q=h_q)
+        assert nv.nvfp4_get_device_status(ws) == nv.OK
+        assert_quantized_equal(h_q, oracle.quantize(h.cpu().numpy()))

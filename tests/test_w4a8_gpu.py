@@ -84,7 +84,8 @@ W4A8_CASES = [
     (16, 1008, 1152, torch.float32, True),      # swapped, stream-K, ragged N
     (40, 2048, 1024, torch.bfloat16, True),     # swapped BN = 64
     (300, 1024, 640, torch.bfloat16, False),    # one-CTA 128-wide tiles, ragged M
-    (1024, 9472, 256, torch.bfloat16, False),   # one-CTA 256-wide tiles
+    (1024, 9472, 256, torch.bfloat16, False),   # CTA pair (256x256 tiles)
+    (1000, 9000, 512, torch.float32, False),    # CTA pair, ragged M and N, fp32 out
     (128, 2048, 5120, torch.float32, True),     # stream-K, not swapped
 ]
 
@@ -125,3 +126,26 @@ def test_w4a8_linear_decode_workload(nv):
     na = np.linalg.norm(oracle.mx8_dequantize_f64(xq_o), axis=1)
     nb = np.linalg.norm(oracle.mx_dequantize_f64(wq_o), axis=1)
     assert_gemm_close(to_numpy_f64(y), ref, na[:, None], nb[None, :], K, True, "w4a8 decode")
+
+
+def test_w4a8_pair_and_one_cta_kernels_agree_with_the_oracle(nv, monkeypatch):
+    """The same prefill-shaped W4A8 GEMM (M = 1024: CTA-pair tiles) on the CTA
+    pair and, with NVFP4_GEMM_CTA_PAIR=0, on the one-CTA kernel: both within
+    the GEMM tolerance of the oracle."""
+    M, N, K = 1024, 4608, 1024
+    x = activations(M, K, 7)
+    w = (np.random.default_rng(8).standard_normal((N, K)) * 0.02).astype(np.float32)
+    xq_o, wq_o = oracle.mx8_quantize(x), oracle.mx_quantize(w)
+    xq = nv.MXFP8Tensor.empty(M, K)
+    nv.nvfp4_mx8_quantize(f32_tensor(x), xq)
+    wq = nv.mx_quantize(f32_tensor(w))
+    ref = oracle.w4a8_gemm_f64(xq_o, wq_o)
+    na = np.linalg.norm(oracle.mx8_dequantize_f64(xq_o), axis=1)
+    nb = np.linalg.norm(oracle.mx_dequantize_f64(wq_o), axis=1)
+    for pair in ("1", "0"):
+        monkeypatch.setenv("NVFP4_GEMM_CTA_PAIR", pair)
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ws = nv.workspace(nv.OP_GEMM, M, N, K)
+        nv.nvfp4_w4a8_gemm(xq, wq, y, ws)
+        assert nv.nvfp4_get_device_status(ws) == nv.OK
+        assert_gemm_close(to_numpy_f64(y), ref, na[:, None], nb[None, :], K, True, f"w4a8 pair={pair}")
