@@ -14,10 +14,12 @@
 //   scale and the E2M1 codes come from the hardware RNE-satfinite
 //   conversions; codes go out as one 8-byte store per block and scales as one
 //   32-bit word per four blocks in the tiled layout the tensor cores read.
-#include "common.cuh"
+#include <atomic>
 #include <cstdlib>
+#include "common.cuh"
 #include "encode.cuh"
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace nvfp4 {
 
@@ -306,6 +308,145 @@ __global__ void __launch_bounds__(256) encode_kernel(const T *__restrict__ x, in
 }
 
 // ---------------------------------------------------------------------------
+// Small tensors (at most kMeetMaxCtas * 256 blocks of 16, e.g. the few
+// activation rows of a decode step): both passes in one cooperative launch
+// of a few CTAs.  Each thread holds one block in registers; each CTA
+// publishes its max |x|, the CTAs meet once (grid_meet), and every thread
+// encodes its block with the same arithmetic as encode_kernel.  One launch
+// instead of two dependent ones, and x is read once.
+// ---------------------------------------------------------------------------
+constexpr int kMeetThreads = 256;
+constexpr int kMeetMaxCtas = 32;
+
+template <typename T>
+__global__ void __launch_bounds__(kMeetThreads) quantize_meet_kernel(
+        const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, uint8_t *__restrict__ codes,
+        uint8_t *__restrict__ scales, float *__restrict__ g_out, float *partials, uint32_t *grid_bar,
+        uint32_t *status, uint64_t timeout_ns) {
+    constexpr int W = sizeof(T) == 2 ? 8 : 16;          // 32-bit words per block
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int bpr = static_cast<int>(cols / kBlock);
+    const int total = static_cast<int>(rows) * bpr;
+    const int b = static_cast<int>(blockIdx.x) * kMeetThreads + t;
+    const int64_t kb4 = kb4_of(cols);
+    const bool word_scales = (cols % 64) == 0;
+    const size_t codes_bytes = static_cast<size_t>(rows * cols / 2);           // debug-build store checks
+    const size_t scales_bytes = static_cast<size_t>(round_up(rows, 128) * kb4);
+    __shared__ float wmax[kMeetThreads / 32];
+    __shared__ float s_amax;
+    __shared__ uint32_t s_go;
+    __shared__ float rcp_table[128];
+    __shared__ uint32_t abort_word;
+    volatile uint32_t *abort_flag = &abort_word;
+    if (t == 0) abort_word = 0u;
+    // x may be the previous kernel's output, and that kernel may still read
+    // the codes this one writes
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    uint32_t v[W];
+    int r = 0, kb = 0;
+    if (b < total) {
+        r = b / bpr;
+        kb = b - r * bpr;
+        load_block(x + static_cast<int64_t>(r) * ld + static_cast<int64_t>(kb) * kBlock, v);
+    } else {
+#pragma unroll
+        for (int i = 0; i < W; ++i) v[i] = 0u;
+    }
+    float m = block_absmax(v, static_cast<T *>(nullptr));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) wmax[warp] = m;
+    __syncthreads();
+    // x is in registers: the next kernel (the GEMM) may launch and start
+    // streaming its weights (earlier, that stream would queue ahead of x)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (warp == 0) {
+        uint32_t go = 0u;
+        if (lane == 0) {
+            float cm = 0.0f;
+            for (int k = 0; k < kMeetThreads / 32; ++k) cm = fmaxf(cm, wmax[k]);
+            partials[blockIdx.x] = cm;
+            // every CTA of the cooperative launch is resident and arrives
+            // exactly once; bounded
+            go = grid_meet(grid_bar, timeout_ns, abort_flag, status) ? 1u : 0u;
+        }
+        go = __shfl_sync(0xffffffffu, go, 0);
+        float gm = 0.0f;
+        if (go)
+            for (int k = lane; k < static_cast<int>(gridDim.x); k += 32) gm = fmaxf(gm, __ldcg(partials + k));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+        if (lane == 0) {
+            s_amax = gm;
+            s_go = go;
+        }
+    }
+    __syncthreads();
+    if (!s_go) return;
+    const float g = __fdiv_rn(s_amax, kTensorScaleDiv);
+    const float six_g = __fmul_rn(6.0f, g);
+    const float inv6g = __frcp_rn(six_g);
+    const bool exact_only = !(six_g > 0.0f) || isinf(inv6g);
+    if (blockIdx.x == 0 && t == 0) *g_out = g;
+    if (t < 128) rcp_table[t] = block_rcp(static_cast<uint32_t>(t), g);
+    __syncthreads();
+
+    // the 4 blocks of a scale word sit in 4 neighbouring lanes (b % 4 == lane % 4)
+    const uint32_t sb = block_scale_byte(block_absmax(v, static_cast<T *>(nullptr)), six_g, inv6g, exact_only);
+    const uint2 cw = block_codes<T, W>(v, rcp_table[sb]);
+    uint32_t word = sb;
+    word |= __shfl_down_sync(0xffffffffu, sb, 1) << 8;
+    word |= __shfl_down_sync(0xffffffffu, sb, 2) << 16;
+    word |= __shfl_down_sync(0xffffffffu, sb, 3) << 24;
+    if (b < total) {
+        uint8_t *cp = codes + static_cast<int64_t>(r) * (cols / 2) + kb * 8;
+        if (store_ok(cp, 8, codes, codes_bytes, status)) *reinterpret_cast<uint2 *>(cp) = cw;
+        uint8_t *sp = scales + scale_offset(r, kb, kb4);
+        if (word_scales) {
+            if ((lane & 3) == 0 && store_ok(sp, 4, scales, scales_bytes, status))
+                *reinterpret_cast<uint32_t *>(sp) = word;
+        } else if (store_ok(sp, 1, scales, scales_bytes, status)) {
+            *sp = static_cast<uint8_t>(sb);
+        }
+    }
+    zero_scale_padding(scales, rows, bpr, kb4, b, static_cast<int64_t>(gridDim.x) * kMeetThreads, scales_bytes,
+                       status);
+}
+
+template <typename T>
+static cudaError_t launch_meet_t(const T *x, int64_t rows, int64_t cols, int64_t ld, uint8_t *codes, uint8_t *scales,
+                                 float *g_out, float *partials, uint32_t *grid_bar, uint32_t *status,
+                                 uint64_t timeout_ns, int grid, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kMeetThreads);
+    cfg.stream = stream;
+    // cooperative (the CTAs meet once), and a programmatic dependent of the
+    // kernel before it if the driver takes both; cooperative alone otherwise
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
+    static std::atomic<int> coop_pdl{1};
+    if (coop_pdl.load()) {
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_meet_kernel<T>, x, rows, cols, ld, codes, scales,
+                                                 g_out, partials, grid_bar, status, timeout_ns);
+        if (e == cudaSuccess) return e;
+        if (e != cudaErrorInvalidValue && e != cudaErrorNotSupported) return e;
+        (void)cudaGetLastError();      // a refused configuration, not a failed launch
+        coop_pdl.store(0);
+    }
+    cfg.attrs = attr + 1;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, quantize_meet_kernel<T>, x, rows, cols, ld, codes, scales, g_out, partials,
+                              grid_bar, status, timeout_ns);
+}
+
+// ---------------------------------------------------------------------------
 // Dequantize: y = fl32(fl32(e * dec(s)) * g), eight values per thread.
 // ---------------------------------------------------------------------------
 template <typename OutT>
@@ -386,6 +527,18 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
                             uint64_t timeout_ns) {
     // An empty tensor has no codes and no scale bytes; its amax is 0, so g = 0.
     if (rows == 0 || cols == 0) return cudaMemsetAsync(g_out, 0, sizeof(float), stream);
+    // Small tensors: one cooperative launch of a few CTAs (NVFP4_QUANTIZE_MEET=0:
+    // the two passes).
+    const char *meet_opt = getenv("NVFP4_QUANTIZE_MEET");
+    const int64_t nblocks = rows * (cols / kBlock);
+    if (grid_bar != nullptr && status != nullptr && (meet_opt == nullptr || meet_opt[0] != '0') &&
+        nblocks <= int64_t(kMeetMaxCtas) * kMeetThreads) {
+        const int grid = static_cast<int>(ceil_div(nblocks, kMeetThreads));
+        return bf16 ? launch_meet_t(static_cast<const __nv_bfloat16 *>(x), rows, cols, ld, codes, scales, g_out,
+                                    partials, grid_bar, status, timeout_ns, grid, stream)
+                    : launch_meet_t(static_cast<const float *>(x), rows, cols, ld, codes, scales, g_out, partials,
+                                    grid_bar, status, timeout_ns, grid, stream);
+    }
     // Large contiguous tensors: one cooperative pass that reads x once.
     if (grid_bar != nullptr && status != nullptr && quantize_onepass_usable(rows, cols, ld, bf16)) {
         const cudaError_t e = launch_quantize_onepass(x, bf16, rows, cols, codes, scales, g_out, partials, grid_bar,

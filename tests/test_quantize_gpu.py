@@ -247,3 +247,27 @@ def test_quantize_onepass(nv, rows, cols, dtype, monkeypatch):
     assert torch.equal(outs[0].scales, outs[1].scales)
     assert torch.equal(outs[0].tensor_scale, outs[1].tensor_scale)
     assert_quantized_equal(outs[0], oracle.quantize(x_or))
+
+
+# Small tensors (at most 32 x 256 blocks of 16) take one cooperative launch
+# of a few CTAs that meet once for the tensor amax; NVFP4_QUANTIZE_MEET=0
+# keeps them on the two passes.  Both bit-exact against the oracle, on shapes
+# with partial scale words (cols % 64 != 0), padding rows, a row pitch wider
+# than cols, and the largest size the cooperative form takes.
+@pytest.mark.parametrize("rows,cols,dtype,ld", [(7, 96, torch.float32, None), (33, 80, torch.bfloat16, 96),
+                                                (130, 320, torch.bfloat16, None), (8, 5120, torch.bfloat16, None),
+                                                (16, 8192, torch.float32, None), (1, 16, torch.bfloat16, None)])
+def test_quantize_small_cooperative_and_two_pass(nv, rows, cols, dtype, ld, monkeypatch):
+    rng = np.random.default_rng(rows * 7 + cols)
+    x = rng.standard_normal((rows, cols)).astype(np.float32)
+    x[rng.random(x.shape) < 2e-3] *= 50
+    if dtype == torch.bfloat16:
+        xt = torch.from_numpy(x).to(torch.bfloat16)
+        x_or = xt.view(torch.int16).numpy().view(np.uint16)
+    else:
+        xt, x_or = torch.from_numpy(x), x
+    want = oracle.quantize(x_or)
+    for meet in ("1", "0"):
+        monkeypatch.setenv("NVFP4_QUANTIZE_MEET", meet)
+        out = quantize_gpu(nv, xt.cuda(), ld)
+        assert_quantized_equal(out, want)
