@@ -34,8 +34,8 @@ L2_BYTES = 126 * 1024 * 1024
 # from one ncu capture of the current kernels (dram__bytes_read.sum +
 # dram__bytes_write.sum); None where the kernel changed after its capture or
 # the capture did not cover every kernel of the dominant call.
-NCU_TRAFFIC = {"prefill": 157_946_112, "decode": 50_256_896, "quantize": None, "mlp": None,
-               "prefill_requant": None, "mx_prefill": 153_014_272, "w4a16_decode": 50_272_000,
+NCU_TRAFFIC = {"prefill": 157_946_112, "decode": 50_256_384, "quantize": 172_837_376, "mlp": 106_568_448,
+               "prefill_requant": 401_925_888, "mx_prefill": 153_014_272, "w4a16_decode": 50_272_000,
                "w4a8_prefill": 173_520_128}
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -225,10 +225,11 @@ class Decode(Prefill):
         # algorithmic bytes of the step: W codes + W scales, X bf16 in, Y bf16 out
         self.bytes = w_bytes + M * K * 2 + M * N * 2
         self.units = self.bytes / 1e9
-        # Per step: the quantizer's two passes over X, then the swapped GEMM
-        # (weights on the MMA's M, the 8 tokens on N = 16), which streams its
-        # first weight stages before the quantizer has finished.
-        self.launches = 3
+        # Per step: the quantizer (one cooperative launch at this size: its
+        # CTAs meet once for the amax), then the swapped GEMM (weights on the
+        # MMA's M, the 8 tokens on N = 16), which streams its first weight
+        # stages before the quantizer has finished.
+        self.launches = 2
         self.dominant = {"kernel": "gemm_nvf4_kernel<16, swapped> (128x16 MMA tiles, four accumulators)",
                          "bound": "hbm", "algorithmic": w_bytes + M * K // 2 + M * K // 16 + M * N * 2,
                          "unit": "GB/s"}
