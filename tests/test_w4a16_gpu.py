@@ -56,6 +56,15 @@ def test_w4a16_parity(nv, M, N, K, yt, pitch):
     run(nv, w["X"], quantize_gpu(nv, bf16_tensor(w["W"])), wq_o, M, N, K, yt, pitch)
 
 
+def test_w4a16_many_tiles(nv):
+    """More tiles than SMs (3 activation tiles x 136 weight tiles): several
+    tiles per CTA, the accumulator handed between them."""
+    M, N, K = 40, 17408, 256
+    w = workloads.make("decode", M=M, K=K, N=N, seed=7)
+    wq_o = oracle.quantize(w["W"])
+    run(nv, w["X"], quantize_gpu(nv, bf16_tensor(w["W"])), wq_o, M, N, K, torch.bfloat16)
+
+
 def test_w4a16_decode_workload(nv):
     """The decode workload's shape and data (M=8, N=17408, K=5120, seed 2):
     every output against the oracle."""
