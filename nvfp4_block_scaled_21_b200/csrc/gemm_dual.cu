@@ -28,9 +28,10 @@
 //   warp 0      TMA producer: per 256-deep K slab the A tile (128 activation
 //               rows), both 128-row weight tiles, and the three 512-byte
 //               scale atoms per K step, into a 4-stage ring.
-//   warp 1      TMEM allocation and MMA issue: per K step two MMAs
-//               (M=128, N=128, K=64), gate into columns [0,128), up into
-//               [128,256); one accumulator stage.
+//   warp 1      TMEM allocation and MMA issue: per K step one MMA
+//               (M=128, N=256, K=64) whose B operand is the gate tile with
+//               the up tile after it in shared memory, so gate lands in
+//               columns [0,128) and up in [128,256); one accumulator stage.
 //   warps 2..5  scale warps: scale atoms from shared memory to their TMEM
 //               lane quarter (tcgen05.st), two stages per handshake.
 //   warps 6..13 epilogue: two warps per lane quarter, 64 columns each.
@@ -74,7 +75,7 @@ struct DualCfg {
     static constexpr int kSfStage = 4 * 512;                  // per operand: 4 K-steps x one atom
     static constexpr int kStageBytes = kAStage + 2 * kBStage + 3 * kSfStage;
     static constexpr int kStages = 4;
-    static constexpr int kSfCols = 48;                        // SFA 16 | SFBg 16 | SFBu 16
+    static constexpr int kSfCols = 48;                        // SFA 16 | SFB 32 (gate, up per K step)
     static constexpr int kSfBase = 256;                       // after the two accumulators
     static constexpr int kTmemCols = 512;
     static constexpr int kThreads = 448;
@@ -96,9 +97,8 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
-    uint8_t *sBg = sA + STAGES * C::kAStage;
-    uint8_t *sBu = sBg + STAGES * C::kBStage;
-    uint8_t *sSf = sBu + STAGES * C::kBStage;               // per stage: SFA | SFBg | SFBu atoms
+    uint8_t *sB = sA + STAGES * C::kAStage;                  // per stage: gate tile, then up tile
+    uint8_t *sSf = sB + STAGES * 2 * C::kBStage;            // per stage: SFA | SFBg | SFBu atoms
     uint64_t *full = reinterpret_cast<uint64_t *>(sSf + STAGES * 3 * C::kSfStage);
     uint64_t *sf_full = full + STAGES;
     uint64_t *empty = sf_full + STAGES;
@@ -141,8 +141,8 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             // ------------------------------------------------------------ producer
             const uint64_t pol = policy_evict_normal();
             auto load_w = [&](uint32_t st, int qt, int ks, int nk) {
-                tma_load_2d(sBg + st * C::kBStage, &tmBg, &full[st], ks * 128, qt * 128, pol);
-                tma_load_2d(sBu + st * C::kBStage, &tmBu, &full[st], ks * 128, qt * 128, pol);
+                tma_load_2d(sB + st * 2 * C::kBStage, &tmBg, &full[st], ks * 128, qt * 128, pol);
+                tma_load_2d(sB + st * 2 * C::kBStage + C::kBStage, &tmBu, &full[st], ks * 128, qt * 128, pol);
                 const int64_t off = (static_cast<int64_t>(qt) * args.num_k_steps + 4 * ks) * 512;
                 bulk_load(sSf + (st * 3 + 1) * C::kSfStage, args.sfbg + off, nk * 512, &full[st], pol);
                 bulk_load(sSf + (st * 3 + 2) * C::kSfStage, args.sfbu + off, nk * 512, &full[st], pol);
@@ -200,8 +200,8 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = make_idesc_nvf4(128);
-            const uint32_t a_base = smem_addr(sA), bg_base = smem_addr(sBg), bu_base = smem_addr(sBu);
+            constexpr uint32_t idesc = make_idesc_nvf4(256);
+            const uint32_t a_base = smem_addr(sA), b_base = smem_addr(sB);
             uint32_t stage = 0, phase = 0, acc_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
@@ -218,13 +218,11 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                     const uint32_t sf = tmem_base + C::kSfBase + stage * C::kSfCols;
                     // K-step j: +32 bytes = +2 in the descriptors' address field
                     const uint64_t adesc = make_operand_desc(a_base + stage * C::kAStage);
-                    const uint64_t gdesc = make_operand_desc(bg_base + stage * C::kBStage);
-                    const uint64_t udesc = make_operand_desc(bu_base + stage * C::kBStage);
+                    // the 256 B rows: 128 of Wg, then 128 of Wu (1024-byte atoms, contiguous)
+                    const uint64_t bdesc = make_operand_desc(b_base + stage * 2 * C::kBStage);
                     auto kstep = [&](int j) {
                         const uint32_t acc = (ks | j) != 0 ? 1u : 0u;
-                        mma_nvf4(tmem_base, adesc + 2 * j, gdesc + 2 * j, idesc, sf + 4 * j, sf + 16 + 4 * j, acc);
-                        mma_nvf4(tmem_base + 128, adesc + 2 * j, udesc + 2 * j, idesc, sf + 4 * j, sf + 32 + 4 * j,
-                                 acc);
+                        mma_nvf4(tmem_base, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j, sf + 16 + 8 * j, acc);
                     };
                     if (nk == 4) {
 #pragma unroll
@@ -275,8 +273,9 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                     const uint4 g = ld_shared_v4(src + C::kSfStage + j * 512);
                     const uint4 u = ld_shared_v4(src + 2 * C::kSfStage + j * 512);
                     av[4 * j] = a.x; av[4 * j + 1] = a.y; av[4 * j + 2] = a.z; av[4 * j + 3] = a.w;
-                    bv[4 * j] = g.x; bv[4 * j + 1] = g.y; bv[4 * j + 2] = g.z; bv[4 * j + 3] = g.w;
-                    bv[16 + 4 * j] = u.x; bv[16 + 4 * j + 1] = u.y; bv[16 + 4 * j + 2] = u.z; bv[16 + 4 * j + 3] = u.w;
+                    // B scales of K step j: the gate rows' 4 columns, then the up rows'
+                    bv[8 * j] = g.x; bv[8 * j + 1] = g.y; bv[8 * j + 2] = g.z; bv[8 * j + 3] = g.w;
+                    bv[8 * j + 4] = u.x; bv[8 * j + 5] = u.y; bv[8 * j + 6] = u.z; bv[8 * j + 7] = u.w;
                 }
                 const uint32_t sf = tmem_base + lane_off + C::kSfBase + stage * C::kSfCols;
                 tmem_st_32x32b_x16(sf, av);
