@@ -8,10 +8,10 @@
 // products for one 128 x 128 output tile from the same activation slabs (two
 // B operands, two fp32 accumulators in tensor memory) and its epilogue writes
 //     gate = fl32(acc_g * fl32(gx * gwg)),  up = fl32(acc_u * fl32(gx * gwu)),
-//     h = fl32(fl32(gate / fl32(1 + expf(-gate))) * up)
-// -- the same fp32 operations, in the same order, as the separate GEMMs and
-// the elementwise SiLU * up would -- plus, per CTA, max |h| in the format of
-// the quantizer's first pass.
+//     h = fl32(fl32(gate / fl32(1 + exp(-gate))) * up)
+// with the hardware exponential and the fast division (__expf, __fdividef:
+// a few ulp of fp32, far inside the tolerance the GEMM's own accumulation
+// needs), plus, per CTA, max |h| in the format of the quantizer's first pass.
 //
 // Re-quantizing h (each NVFP4 tensor carries its own two-level scaling:
 // NVFP4 wiki page, section "技術原理") needs max |h| over the whole tensor
@@ -86,7 +86,7 @@ struct DualCfg {
 };
 
 __device__ __forceinline__ float silu_mul(float gate, float up) {
-    return __fmul_rn(__fdiv_rn(gate, __fadd_rn(1.0f, expf(-gate))), up);
+    return __fmul_rn(__fdividef(gate, __fadd_rn(1.0f, __expf(-gate))), up);
 }
 
 __global__ void __launch_bounds__(448, 1)
@@ -289,6 +289,9 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     } else {
         // ------------------------------------------------------------ epilogue
         asm volatile("griddepcontrol.wait;" ::: "memory");   // tensor scales may be fresh
+        // the meeting point's generation, read early (see grid_meet_generation)
+        const uint32_t meet_gen = (warp == 6 && lane == 0 && args.hq_codes != nullptr)
+                                      ? grid_meet_generation(args.grid_bar) : 0u;
         const int quarter = warp & 3;
         const int half = (warp - 6) >> 2;
         const int row = quarter * 32 + lane;
@@ -365,7 +368,7 @@ gemm_nvf4_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                     // every CTA of the cooperative launch is resident and
                     // arrives exactly once (also after a give-up of its own),
                     // so the wait ends unless one of them gave up; bounded
-                    go = grid_meet(args.grid_bar, args.timeout_ns, abort_flag, args.status) ? 1u : 0u;
+                    go = grid_meet(args.grid_bar, meet_gen, args.timeout_ns, abort_flag, args.status) ? 1u : 0u;
                 }
                 go = __shfl_sync(0xffffffffu, go, 0);
                 // the grid's maxima, read by the whole warp at once
@@ -485,7 +488,8 @@ cudaError_t launch_gemm_dual_silu(const Operand &act, const Operand &wg, const O
     if (grid > max_partials) grid = max_partials;
     if (grid < 1) grid = 1;
     *num_partials = grid;
-    if (hq_codes != nullptr && grid != tiles) return cudaErrorInvalidValue;   // one tile per CTA
+    // the in-epilogue re-quantization: one tile per CTA and a meeting point
+    if (hq_codes != nullptr && (grid != tiles || grid_bar == nullptr)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_dual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;

@@ -78,23 +78,33 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     }
 }
 
-// Grid-wide meeting point of a cooperative launch, run by one thread per CTA
-// after its CTA's writes that the others will read (each writer fenced them).
-// bar[0] counts arrivals, bar[1] is the generation: the last CTA to arrive
-// resets the count and advances the generation, the others wait (bounded) for
-// the generation to move.  The count is back at zero after every completed
-// meeting, so a zero-filled pair serves any sequence of launches and grid
-// sizes that do not overlap in time.  Returns false on a timeout or an abort
-// (the timeout is recorded as mbar_wait does).
-__device__ __forceinline__ bool grid_meet(uint32_t *bar, uint64_t timeout_ns, volatile uint32_t *abort_flag,
-                                          uint32_t *status) {
+// The current generation of a grid meeting point (bar[1], see grid_meet).
+// The thread that will arrive reads it early -- after the dependent-launch
+// wait, before its own arrival, when the meeting cannot have completed yet --
+// so that this load's latency stays off the meeting's critical path.
+__device__ __forceinline__ uint32_t grid_meet_generation(const uint32_t *bar) {
     uint32_t gen;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(gen) : "l"(bar + 1) : "memory");
+    return gen;
+}
+
+// Grid-wide meeting point of a cooperative launch, run by one thread per CTA
+// after its CTA's writes that the others will read.  bar[0] counts arrivals,
+// bar[1] is the generation, `gen` its value read by grid_meet_generation: the
+// last CTA to arrive advances the generation (after a fence, so every CTA's
+// fenced writes are visible to whoever sees the new generation) and then
+// resets the count; the others wait (bounded) for the generation to move.
+// The count is back at zero when the kernel ends, so a zero-filled pair
+// serves any sequence of launches and grid sizes that do not overlap in time
+// (each kernel meets once).  Returns false on a timeout or an abort (the
+// timeout is recorded as mbar_wait does).
+__device__ __forceinline__ bool grid_meet(uint32_t *bar, uint32_t gen, uint64_t timeout_ns,
+                                          volatile uint32_t *abort_flag, uint32_t *status) {
     __threadfence();
     if (atomicAdd(bar, 1u) == gridDim.x - 1) {
-        atomicExch(bar, 0u);
         __threadfence();
         atomicAdd(bar + 1, 1u);
+        atomicExch(bar, 0u);
         return true;
     }
     const uint64_t start = global_timer_ns();

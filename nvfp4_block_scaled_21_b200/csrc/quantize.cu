@@ -342,6 +342,8 @@ __global__ void __launch_bounds__(kMeetThreads) quantize_meet_kernel(
     // x may be the previous kernel's output, and that kernel may still read
     // the codes this one writes
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the meeting point's generation, read early (see grid_meet_generation)
+    const uint32_t meet_gen = threadIdx.x == 0 ? grid_meet_generation(grid_bar) : 0u;
 
     uint32_t v[W];
     int r = 0, kb = 0;
@@ -369,7 +371,7 @@ __global__ void __launch_bounds__(kMeetThreads) quantize_meet_kernel(
             partials[blockIdx.x] = cm;
             // every CTA of the cooperative launch is resident and arrives
             // exactly once; bounded
-            go = grid_meet(grid_bar, timeout_ns, abort_flag, status) ? 1u : 0u;
+            go = grid_meet(grid_bar, meet_gen, timeout_ns, abort_flag, status) ? 1u : 0u;
         }
         go = __shfl_sync(0xffffffffu, go, 0);
         float gm = 0.0f;

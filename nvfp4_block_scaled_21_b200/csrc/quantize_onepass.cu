@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(kOpThreads, 1) quantize_onepass_kernel(const _
     __syncthreads();
     // x may be the output of the kernel before this one
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    const uint32_t meet_gen = threadIdx.x == 0 ? grid_meet_generation(a.grid_bar) : 0u;   // read early
 
     // ---- pass A
     if (t == 0 && S > 0) {
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(kOpThreads, 1) quantize_onepass_kernel(const _
             a.partials[blockIdx.x] = cm;
             // every CTA of the cooperative launch is resident and arrives
             // exactly once, also after a give-up of its own; bounded
-            go = grid_meet(a.grid_bar, a.timeout_ns, abort_flag, a.status) ? 1u : 0u;
+            go = grid_meet(a.grid_bar, meet_gen, a.timeout_ns, abort_flag, a.status) ? 1u : 0u;
         }
         go = __shfl_sync(0xffffffffu, go, 0);
         float gm = 0.0f;
