@@ -78,7 +78,6 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 // status word (offset 0) and the grid meeting point of the cooperative
 // kernels (offset 128: arrival count, generation; back at zero after every
 // completed meeting).
-constexpr size_t kGridBarOff = 128;
 constexpr size_t kPartialsOff = kWsStatusBytes;
 constexpr size_t kPartialsBytes = kMaxAmaxPartials * sizeof(float);
 constexpr size_t kQuantizeWs = kPartialsOff + kPartialsBytes;

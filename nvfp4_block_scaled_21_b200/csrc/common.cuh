@@ -69,6 +69,7 @@ template <> __device__ __forceinline__ void YMax::add<__nv_bfloat16>(__nv_bfloat
 
 // Workspace layout: [0,16) status words, [256, ...) scratch.
 constexpr size_t kWsStatusBytes = 256;
+constexpr size_t kGridBarOff = 128;    // grid meeting point: arrival count, generation
 constexpr int kMaxAmaxPartials = 4096;
 
 // Debug build (compiled with NVFP4_DEBUG_CHECKS): every direct global store

@@ -34,13 +34,17 @@
 // When the output tiles would leave at least half of the SMs idle, CTAs take
 // equal runs of (tile, K slab) units instead of whole tiles (stream-K): partial
 // tiles are added in fp32 in the workspace and the CTA that completes a
-// tile's K range writes it.
+// tile's K range writes it.  That launch is cooperative: the epilogue warps
+// zero-fill the CTA's share of the partial-sum buffer and its counters and
+// meet the grid once before the first partial sum lands, while the first
+// work item's loads and MMAs run.
 // When the weights are known not to come from the kernel launched just before
 // (inside nvfp4_linear_fused), the producer starts streaming them before the
 // programmatic-dependent-launch wait, hiding the pipeline fill behind the
 // activation quantizer.
 // Every wait is bounded; a timeout sets the status word and winds the CTA
 // down without leaving tensor memory allocated.
+#include <atomic>
 #include <cstdlib>
 #include "common.cuh"
 #include "kernels.cuh"
@@ -63,8 +67,10 @@ struct GemmArgs {
     int32_t weights_are_a;   // 1: the weights are the MMA A operand (swapped)
     int32_t streamk;         // 1: CTAs take equal contiguous runs of (tile, K slab) units
     int32_t q_pad;           // row pitch (floats) of acc_ws: num_q_tiles * BN
-    float *acc_ws;           // stream-K: fp32 partial sums [num_p_tiles*128][q_pad], zeroed per call
-    int32_t *tile_cnt;       // stream-K: K slabs added per tile so far, zeroed per call
+    float *acc_ws;           // stream-K: fp32 partial sums [num_p_tiles*128][q_pad], zeroed in-kernel
+    int32_t *tile_cnt;       // stream-K: K slabs added per tile so far (follows acc_ws), zeroed in-kernel
+    int64_t zero_words;      // stream-K: 32-bit words from acc_ws that the grid zero-fills
+    uint32_t *grid_bar;      // stream-K: grid meeting point (the workspace header's)
     float *ymax_part;        // if set: this CTA's largest |y| as stored, at [blockIdx.x]
     uint32_t *status;
     uint64_t timeout_ns;
@@ -488,6 +494,26 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         auto y_ok = [&](const void *ptr, size_t bytes) { return store_ok(ptr, bytes, args.y, y_bytes, args.status); };
         uint32_t acc = 0, acc_phase = 0;
         uint32_t npart = 0;      // partial (stream-K) work items so far: epi_done/epi_flag phase
+        if (args.streamk) {
+            // Zero-fill this CTA's share of the partial sums and counters (a
+            // previous call may have left anything there; the dependent-launch
+            // wait above covers a previous kernel still using them), then meet
+            // the grid: no partial sum is added before every share is zero.
+            const uint32_t meet_gen = (warp == 6 && lane == 0) ? grid_meet_generation(args.grid_bar) : 0u;
+            const int64_t per = (args.zero_words / 4 + gridDim.x - 1) / gridDim.x;      // uint4 per CTA
+            uint4 *zb = reinterpret_cast<uint4 *>(args.acc_ws);
+            const int64_t lo = per * blockIdx.x, hi = min(per * (blockIdx.x + 1), args.zero_words / 4);
+            for (int64_t i = lo + (threadIdx.x - 6 * 32); i < hi; i += 8 * 32) zb[i] = make_uint4(0u, 0u, 0u, 0u);
+            __threadfence();
+            asm volatile("bar.sync 1, 256;" ::: "memory");             // the 8 epilogue warps
+            if (warp == 6) {
+                uint32_t go = 0u;
+                if (lane == 0) go = grid_meet(args.grid_bar, meet_gen, args.timeout_ns, abort_flag, args.status) ? 1u : 0u;
+                go = __shfl_sync(0xffffffffu, go, 0);
+                if (lane == 0 && !go) *abort_flag = 1u;
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+        }
         // Largest |y| this thread stores.  Accumulator rows and columns past P
         // and Q are exact zeros (their operand rows are zero-filled by the
         // loads), so folding a whole computed chunk cannot raise it.
@@ -956,12 +982,15 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     a.q_pad = a.num_q_tiles * BN;
     a.acc_ws = sk ? reinterpret_cast<float *>(splitk_ws) : nullptr;
     a.tile_cnt = sk ? reinterpret_cast<int32_t *>(splitk_ws + skl.acc_bytes) : nullptr;
+    // The stream-K scratch is zero-filled by the kernel itself for every call
+    // (so it may share a workspace with whatever other calls left there); its
+    // CTAs meet at the meeting point in the workspace header, which `status`
+    // starts.
+    a.zero_words = sk ? static_cast<int64_t>(skl.bytes / 4) : 0;
+    a.grid_bar = sk ? reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(status) + kGridBarOff) : nullptr;
     auto kern = gemm_nvf4_kernel<BN, SWAP, OutT, FMT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    // The stream-K scratch is zero-filled for every call, so it may share a
-    // workspace with whatever other calls left there.
-    if (sk && (e = cudaMemsetAsync(splitk_ws, 0, skl.bytes, stream)) != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     const int64_t work = sk ? units : tiles;
     cfg.gridDim = dim3(static_cast<unsigned>(work < num_sms ? work : num_sms));
@@ -969,10 +998,26 @@ static cudaError_t run_gemm(const Operand &pa, const Operand &qb, int64_t K, voi
     cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
     cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (!sk) return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
+    // stream-K: cooperative (one grid-wide meeting), and a programmatic
+    // dependent of the kernel before it if the driver takes both
+    static std::atomic<int> coop_pdl{1};
+    if (coop_pdl.load()) {
+        cfg.numAttrs = 2;
+        e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
+        if (e == cudaSuccess) return e;
+        if (e != cudaErrorInvalidValue && e != cudaErrorNotSupported) return e;
+        (void)cudaGetLastError();      // a refused configuration, not a failed launch
+        coop_pdl.store(0);
+    }
+    cfg.attrs = attr + 1;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
 }

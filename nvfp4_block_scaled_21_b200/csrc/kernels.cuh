@@ -35,7 +35,9 @@ struct Operand {
 // weights_ready: the weights were not written by the kernel launched just
 // before (they may be streamed before the programmatic-dependent-launch wait).
 // splitk_ws: splitk_ws_bytes(M, N) bytes of scratch (or null: no stream-K);
-// any contents (the call zero-fills what it uses).
+// any contents (the kernel zero-fills what it uses).  With it, `status` must
+// be the workspace's start: the stream-K CTAs meet at the header's meeting
+// point.
 // ymax_part (optional): every CTA writes the largest |y| it stored (the value
 // as stored, after rounding to y's dtype) to ymax_part[blockIdx.x], the
 // quantizer's first-pass format; *nparts receives the grid size (<= 4096).
