@@ -34,7 +34,7 @@ L2_BYTES = 126 * 1024 * 1024
 # from one ncu capture of the current kernels (dram__bytes_read.sum +
 # dram__bytes_write.sum); None where the kernel changed after its capture or
 # the capture did not cover every kernel of the dominant call.
-NCU_TRAFFIC = {"prefill": 157_946_112, "decode": 50_256_384, "quantize": 172_837_376, "mlp": 106_568_448,
+NCU_TRAFFIC = {"prefill": 157_946_112, "decode": 50_260_224, "quantize": 172_837_376, "mlp": 106_699_264,
                "prefill_requant": 401_925_888, "mx_prefill": 153_014_272, "w4a16_decode": 50_272_000,
                "w4a8_prefill": 173_520_128}
 FALLBACK_HBM_GBS = 6650.0
@@ -321,8 +321,8 @@ class Mlp:
         # amax and encode passes on x; gate+up GEMM, which re-quantizes h in
         # its epilogue (its 136 tiles fit the SMs); down GEMM
         self.launches = 4
-        # The largest share of the step is the gate+up kernel (ncu: 40.4 us
-        # against 27.8 us for the down projection).  It runs inside the
+        # The largest share of the step is the gate+up kernel (ncu: 31.7 us
+        # against 28.9 us for the down projection).  It runs inside the
         # fused call together with the two quantizer passes on x, so the
         # roofline is taken over that call: gate and up weights, x in, h_q out.
         self.dominant = {"kernel": "gemm_nvf4_dual_kernel (gate+up, SiLU*up epilogue re-quantizing h) in the "
