@@ -503,7 +503,9 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const int64_t per = (args.zero_words / 4 + gridDim.x - 1) / gridDim.x;      // uint4 per CTA
             uint4 *zb = reinterpret_cast<uint4 *>(args.acc_ws);
             const int64_t lo = per * blockIdx.x, hi = min(per * (blockIdx.x + 1), args.zero_words / 4);
-            for (int64_t i = lo + (threadIdx.x - 6 * 32); i < hi; i += 8 * 32) zb[i] = make_uint4(0u, 0u, 0u, 0u);
+            for (int64_t i = lo + (threadIdx.x - 6 * 32); i < hi; i += 8 * 32)
+                if (store_ok(zb + i, 16, args.acc_ws, static_cast<size_t>(args.zero_words) * 4, args.status))
+                    zb[i] = make_uint4(0u, 0u, 0u, 0u);
             __threadfence();
             asm volatile("bar.sync 1, 256;" ::: "memory");             // the 8 epilogue warps
             if (warp == 6) {
