@@ -164,6 +164,31 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype xt, int64_t row
                             nvfp4_stream_t stream);
 
 /*
+ * The quantizer's two halves for a tensor split across GPUs by rows (tensor
+ * parallelism).  Every NVFP4 tensor has one FP32 tensor scale over all of it
+ * (NVFP4 wiki page, section "技術原理"), so the ranks holding parts of one
+ * tensor must agree on its amax before any block is encoded:
+ *   nvfp4_amax                 *amax = max |x| over this rank's rows (one
+ *                              fp32 in device memory; the first pass of
+ *                              nvfp4_quantize, reduced on the device);
+ *   (the caller all-reduces the ranks' amax with MAX: one float);
+ *   nvfp4_quantize_with_amax   nvfp4_quantize's second pass with g =
+ *                              fl32(*amax / 2688) from the given amax instead
+ *                              of this rank's own.
+ * The codes and scales of each rank's rows then equal those of the same rows
+ * of the whole tensor quantized at once, and every rank's tensor_scale is
+ * the whole tensor's.  Arguments, alignment and errors as nvfp4_quantize;
+ * `amax` is device memory owned by the caller; ws as for NVFP4_OP_QUANTIZE.
+ * An empty x gives *amax = 0 (nvfp4_amax) and still writes tensor_scale
+ * (nvfp4_quantize_with_amax).
+ */
+NVFP4_API nvfp4_status nvfp4_amax(const void *x, nvfp4_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                                  float *amax, void *ws, size_t ws_bytes, nvfp4_stream_t stream);
+NVFP4_API nvfp4_status nvfp4_quantize_with_amax(const void *x, nvfp4_dtype xt, int64_t rows, int64_t cols,
+                                                int64_t ld, const float *amax, const nvfp4_tensor *out,
+                                                void *ws, size_t ws_bytes, nvfp4_stream_t stream);
+
+/*
  * Dequantize q into y [q->rows][q->cols] (row pitch ldy elements, dtype yt):
  * y = fl32(fl32(e * dec(s)) * g), rounded to bf16 by RNE when yt is BF16.
  * This is the decode step a W4A16 path would run before a 16-bit GEMM

@@ -39,7 +39,7 @@ EXPORTED = (
     "nvfp4_selftest_bounded_wait", "nvfp4_set_wait_timeout_us", "nvfp4_status_string",
     "nvfp4_version", "nvfp4_linear_noalloc", "nvfp4_gemm_requant", "nvfp4_mx_scales_bytes",
     "nvfp4_mx_quantize", "nvfp4_mx_gemm", "nvfp4_w4a16_linear", "nvfp4_mx8_quantize", "nvfp4_w4a8_gemm",
-    "nvfp4_w4a8_linear",
+    "nvfp4_w4a8_linear", "nvfp4_amax", "nvfp4_quantize_with_amax",
 )
 
 
@@ -75,6 +75,10 @@ _lib.nvfp4_workspace_bytes.argtypes = [_I, _I64, _I64, _I64]
 _lib.nvfp4_workspace_bytes.restype = _SZ
 _lib.nvfp4_quantize.argtypes = [_P, _I, _I64, _I64, _I64, _T, _P, _SZ, _P]
 _lib.nvfp4_quantize.restype = _I
+_lib.nvfp4_amax.argtypes = [_P, _I, _I64, _I64, _I64, _P, _P, _SZ, _P]
+_lib.nvfp4_amax.restype = _I
+_lib.nvfp4_quantize_with_amax.argtypes = [_P, _I, _I64, _I64, _I64, _P, _T, _P, _SZ, _P]
+_lib.nvfp4_quantize_with_amax.restype = _I
 _lib.nvfp4_dequantize.argtypes = [_T, _P, _I, _I64, _P]
 _lib.nvfp4_dequantize.restype = _I
 _lib.nvfp4_gemm.argtypes = [_T, _T, _P, _I, _I64, _P, _SZ, _P]
@@ -230,7 +234,7 @@ def _rows(*ts) -> None:
     ABI describes with a pointer and a row pitch.  A plain check, not an assert,
     so that it also holds under python -O."""
     for t in ts:
-        if t is not None and (t.dim() != 2 or t.stride(1) != 1):
+        if t is not None and (t.dim() != 2 or (t.numel() != 0 and t.stride(1) != 1)):
             raise ValueError(f"nvfp4: expected a 2-D tensor with contiguous rows, got shape "
                              f"{tuple(t.shape)} strides {tuple(t.stride())}")
 
@@ -328,9 +332,49 @@ def nvfp4_quantize(x, out: NVFP4Tensor, ws, stream=None) -> NVFP4Tensor:
     _buffers(out)
     _on_device(x, out, ws)
     ct = out.c()
-    st = _lib.nvfp4_quantize(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], x.stride(0),
+    st = _lib.nvfp4_quantize(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], _ld(x),
                              ctypes.byref(ct), ws.data_ptr(), _ws_bytes(ws), _stream(stream))
     _check(st, "nvfp4_quantize")
+    return out
+
+
+def _ld(x) -> int:
+    """Row pitch (elements) of a 2-D tensor; an empty one is never read, and
+    its strides may be anything, so it gets the plain pitch cols."""
+    return x.stride(0) if x.numel() != 0 else x.shape[1]
+
+
+def _amax_buffer(amax) -> None:
+    """One fp32 on the device: the library writes or reads exactly that."""
+    if amax.dtype != _torch().float32 or amax.numel() < 1 or not amax.is_contiguous():
+        raise ValueError("nvfp4: amax must be a contiguous fp32 tensor of at least one element")
+
+
+def nvfp4_amax(x, amax, ws, stream=None):
+    """amax[0] = max |x| over a 2-D bf16/fp32 CUDA tensor (the quantizer's
+    first pass, reduced on the device): this rank's share of a tensor split
+    across ranks by rows, before an all-reduce MAX."""
+    _rows(x)
+    _amax_buffer(amax)
+    _on_device(x, amax, ws)
+    st = _lib.nvfp4_amax(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], _ld(x), amax.data_ptr(),
+                         ws.data_ptr(), _ws_bytes(ws), _stream(stream))
+    _check(st, "nvfp4_amax")
+    return amax
+
+
+def nvfp4_quantize_with_amax(x, amax, out: NVFP4Tensor, ws, stream=None) -> NVFP4Tensor:
+    """nvfp4_quantize with the tensor amax given (amax[0], device fp32) instead
+    of computed from x: g = amax / 2688."""
+    _rows(x)
+    _amax_buffer(amax)
+    _buffers(out)
+    _on_device(x, amax, out, ws)
+    ct = out.c()
+    st = _lib.nvfp4_quantize_with_amax(x.data_ptr(), _dtype_code(x), x.shape[0], x.shape[1], _ld(x),
+                                       amax.data_ptr(), ctypes.byref(ct), ws.data_ptr(), _ws_bytes(ws),
+                                       _stream(stream))
+    _check(st, "nvfp4_quantize_with_amax")
     return out
 
 

@@ -53,6 +53,8 @@ nvfp4_status current_device(DevInfo *out) {
     return NVFP4_OK;
 }
 
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
 nvfp4_status check_tensor(const nvfp4_tensor *t, int64_t rows, int64_t cols) {
     if (!t || !t->tensor_scale) return NVFP4_ERR_INVALID_ARG;
     if (t->rows != rows || t->cols != cols || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
@@ -155,6 +157,42 @@ nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype xt, int64_t rows, int64_t
                                      reinterpret_cast<cudaStream_t>(stream),
                                      reinterpret_cast<uint32_t *>(ws_at(ws, kGridBarOff)),
                                      static_cast<uint32_t *>(ws), wait_timeout_ns()));
+}
+
+nvfp4_status nvfp4_amax(const void *x, nvfp4_dtype xt, int64_t rows, int64_t cols, int64_t ld, float *amax,
+                        void *ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    if ((!x && rows * cols != 0) || !amax || (xt != NVFP4_F32 && xt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
+    if (cols % 16) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const int eb = xt == NVFP4_BF16 ? 2 : 4;
+    if (rows * cols != 0 && (!aligned16(x) || (ld * eb) % 16)) return NVFP4_ERR_MISALIGNED;
+    if (!aligned4(amax)) return NVFP4_ERR_MISALIGNED;
+    nvfp4_status st = check_ws(ws, ws_bytes, kQuantizeWs);
+    if (st != NVFP4_OK) return st;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    return from_cuda(launch_amax(x, xt == NVFP4_BF16, rows, cols, ld,
+                                 reinterpret_cast<float *>(ws_at(ws, kPartialsOff)), amax, dev.sms,
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_quantize_with_amax(const void *x, nvfp4_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                                      const float *amax, const nvfp4_tensor *out, void *ws, size_t ws_bytes,
+                                      nvfp4_stream_t stream) {
+    if ((!x && rows * cols != 0) || !amax || (xt != NVFP4_F32 && xt != NVFP4_BF16)) return NVFP4_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_tensor(out, rows, cols);
+    if (st != NVFP4_OK) return st;
+    const int eb = xt == NVFP4_BF16 ? 2 : 4;
+    if (rows * cols != 0 && (!aligned16(x) || (ld * eb) % 16)) return NVFP4_ERR_MISALIGNED;
+    if (!aligned4(amax)) return NVFP4_ERR_MISALIGNED;
+    if ((st = check_ws(ws, ws_bytes, kQuantizeWs)) != NVFP4_OK) return st;
+    DevInfo dev;
+    if ((st = current_device(&dev)) != NVFP4_OK) return st;
+    // the encode pass reduces its "partial maxima": here the one given amax
+    return from_cuda(launch_encode(x, xt == NVFP4_BF16, rows, cols, ld, amax, 1, out->codes, out->scales,
+                                   out->tensor_scale, dev.sms, reinterpret_cast<cudaStream_t>(stream),
+                                   static_cast<uint32_t *>(ws)));
 }
 
 nvfp4_status nvfp4_dequantize(const nvfp4_tensor *q, void *y, nvfp4_dtype yt, int64_t ldy,

@@ -97,6 +97,10 @@ cudaError_t launch_mx_quantize(const void *x, bool bf16, int64_t rows, int64_t c
 cudaError_t launch_encode_f32(const float *x, int64_t rows, int64_t cols, int64_t ld, const float *partials,
                               int num_partials, uint8_t *codes, uint8_t *scales, float *g_out, int num_sms,
                               cudaStream_t stream, uint32_t *status = nullptr);
+// The quantizer's first pass on its own: *amax = max |x| (device fp32), via
+// per-CTA partial maxima (at most kMaxAmaxPartials floats of scratch).
+cudaError_t launch_amax(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld, float *partials,
+                        float *amax, int num_sms, cudaStream_t stream);
 // The same for bf16 or fp32 x.
 cudaError_t launch_encode(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld, const float *partials,
                           int num_partials, uint8_t *codes, uint8_t *scales, float *g_out, int num_sms,

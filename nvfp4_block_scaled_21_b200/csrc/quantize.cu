@@ -587,6 +587,41 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
                               g_out, status);
 }
 
+// One CTA: *amax = the largest of n partial maxima (the reduction the encode
+// pass starts with, as a value of its own).
+__global__ void __launch_bounds__(256) reduce_amax_kernel(const float *__restrict__ partials, int n,
+                                                         float *__restrict__ amax) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const float m = reduce_partials(partials, n);
+    if (threadIdx.x == 0) *amax = m;
+}
+
+cudaError_t launch_amax(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld, float *partials,
+                        float *amax, int num_sms, cudaStream_t stream) {
+    if (rows == 0 || cols == 0) return cudaMemsetAsync(amax, 0, sizeof(float), stream);
+    const int eb = bf16 ? 2 : 4;
+    static const int occ_amax[2] = {resident_ctas(amax_partials_kernel<float>),
+                                    resident_ctas(amax_partials_kernel<__nv_bfloat16>)};
+    int g1 = quantize_grid(rows, cols, eb, num_sms, occ_amax[bf16]);
+    if (g1 > kMaxAmaxPartials) g1 = kMaxAmaxPartials;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(g1);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = bf16 ? cudaLaunchKernelEx(&cfg, amax_partials_kernel<__nv_bfloat16>,
+                                              static_cast<const __nv_bfloat16 *>(x), rows, cols, ld, partials)
+                         : cudaLaunchKernelEx(&cfg, amax_partials_kernel<float>, static_cast<const float *>(x), rows,
+                                              cols, ld, partials);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(1);
+    return cudaLaunchKernelEx(&cfg, reduce_amax_kernel, static_cast<const float *>(partials), g1, amax);
+}
+
 cudaError_t launch_encode(const void *x, bool bf16, int64_t rows, int64_t cols, int64_t ld, const float *partials,
                           int num_partials, uint8_t *codes, uint8_t *scales, float *g_out, int num_sms,
                           cudaStream_t stream, uint32_t *status) {

@@ -97,6 +97,30 @@ def test_quantize_rejects_bad_arguments_without_launch():
     assert q(16, nv.BF16, 4, 64, 64, out, ws, 100) == nv.ERR_WORKSPACE
 
 
+def test_amax_and_quantize_with_amax_reject_bad_arguments_without_launch():
+    lib = nv.lib()
+    ws, amax = 4096, 1024
+    a = lambda x, xt, r, c, ld, am, w, wb: lib.nvfp4_amax(x, xt, r, c, ld, am, w, wb, None)
+    assert a(None, nv.BF16, 4, 64, 64, amax, ws, 1 << 20) == nv.ERR_INVALID_ARG
+    assert a(16, nv.BF16, 4, 64, 64, None, ws, 1 << 20) == nv.ERR_INVALID_ARG
+    assert a(16, 7, 4, 64, 64, amax, ws, 1 << 20) == nv.ERR_INVALID_ARG
+    assert a(16, nv.BF16, 4, 64, 32, amax, ws, 1 << 20) == nv.ERR_INVALID_ARG        # ld < cols
+    assert a(16, nv.BF16, 4, 24, 24, amax, ws, 1 << 20) == nv.ERR_UNSUPPORTED_SHAPE
+    assert a(18, nv.BF16, 4, 64, 64, amax, ws, 1 << 20) == nv.ERR_MISALIGNED
+    assert a(16, nv.BF16, 4, 64, 64, amax + 2, ws, 1 << 20) == nv.ERR_MISALIGNED
+    assert a(16, nv.BF16, 4, 64, 64, amax, None, 1 << 20) == nv.ERR_WORKSPACE
+    assert a(16, nv.BF16, 4, 64, 64, amax, ws, 100) == nv.ERR_WORKSPACE
+    out = _t()
+    q = lambda x, xt, r, c, ld, am, o, w, wb: lib.nvfp4_quantize_with_amax(
+        x, xt, r, c, ld, am, ctypes.byref(o) if o else None, w, wb, None)
+    assert q(16, nv.BF16, 4, 64, 64, None, out, ws, 1 << 20) == nv.ERR_INVALID_ARG
+    assert q(16, nv.BF16, 4, 64, 64, amax, None, ws, 1 << 20) == nv.ERR_INVALID_ARG
+    assert q(16, nv.BF16, 4, 64, 64, amax, _t(rows=5), ws, 1 << 20) == nv.ERR_INVALID_ARG
+    assert q(16, nv.BF16, 4, 24, 24, amax, _t(cols=24), ws, 1 << 20) == nv.ERR_UNSUPPORTED_SHAPE
+    assert q(16, nv.BF16, 4, 64, 64, amax + 1, out, ws, 1 << 20) == nv.ERR_MISALIGNED
+    assert q(16, nv.BF16, 4, 64, 64, amax, out, ws, 100) == nv.ERR_WORKSPACE
+
+
 def test_gemm_rejects_bad_arguments_without_launch():
     lib = nv.lib()
     a, b = _t(rows=8, cols=128), _t(rows=32, cols=128)
