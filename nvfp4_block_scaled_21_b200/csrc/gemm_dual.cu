@@ -5,8 +5,10 @@
 // NVFP4, section "核心差异：W4A4 vs W4A16": activations and weights both NVFP4
 // into the FP4 tensor cores) computes h = SiLU(x Wg^T) * (x Wu^T) and
 // re-quantizes h to NVFP4 for the down projection.  This kernel computes both
-// products for one 128 x 128 output tile from the same activation slabs (two
-// B operands, two fp32 accumulators in tensor memory) and its epilogue writes
+// products for one 128 x 128 output tile from the same activation slabs (the
+// gate and up weight tiles as one 256-row B operand, so the fp32 accumulator
+// in tensor memory holds gate in columns [0,128) and up in [128,256)) and its
+// epilogue writes
 //     gate = fl32(acc_g * fl32(gx * gwg)),  up = fl32(acc_u * fl32(gx * gwu)),
 //     h = fl32(fl32(gate / fl32(1 + exp(-gate))) * up)
 // with the hardware exponential and the fast division (__expf, __fdividef:
@@ -76,7 +78,7 @@ struct DualCfg {
     static constexpr int kStageBytes = kAStage + 2 * kBStage + 3 * kSfStage;
     static constexpr int kStages = 4;
     static constexpr int kSfCols = 48;                        // SFA 16 | SFB 32 (gate, up per K step)
-    static constexpr int kSfBase = 256;                       // after the two accumulators
+    static constexpr int kSfBase = 256;                       // after the accumulator (gate | up)
     static constexpr int kTmemCols = 512;
     static constexpr int kThreads = 448;
     static constexpr int kBarBytes = 8 * (3 * kStages + 3) + 16;
