@@ -178,7 +178,9 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype xt, int64_t row
  * The codes and scales of each rank's rows then equal those of the same rows
  * of the whole tensor quantized at once, and every rank's tensor_scale is
  * the whole tensor's.  Arguments, alignment and errors as nvfp4_quantize;
- * `amax` is device memory owned by the caller; ws as for NVFP4_OP_QUANTIZE.
+ * `amax` is one fp32 of device memory owned by the caller (4-byte aligned,
+ * else NVFP4_ERR_MISALIGNED; null: NVFP4_ERR_INVALID_ARG); ws as for
+ * NVFP4_OP_QUANTIZE (nvfp4_amax keeps its partial maxima there).
  * An empty x gives *amax = 0 (nvfp4_amax) and still writes tensor_scale
  * (nvfp4_quantize_with_amax).
  */
