@@ -52,7 +52,9 @@
  *   - Kernel choice is automatic.  Environment switches, read at each call,
  *     exist for A/B measurements: NVFP4_GEMM_CTA_PAIR=0 keeps large-M GEMMs
  *     on the one-CTA kernel; NVFP4_GEMM_STREAMK=0 disables the split-K
- *     (stream-K) path for GEMMs with few output tiles; NVFP4_DECODE_FUSED=1
+ *     (stream-K) path for GEMMs with few output tiles (a cooperative launch
+ *     of one CTA per SM: a context limited to fewer SMs than the device has
+ *     gets NVFP4_ERR_CUDA from it and should set this); NVFP4_DECODE_FUSED=1
  *     runs nvfp4_linear_fused's STORE form for M <= 16 as one kernel that
  *     quantizes x itself; NVFP4_MLP_FUSED_REQUANT=0 keeps the SiLU form's
  *     re-quantization of h in a separate encode pass (by default the gate/up
