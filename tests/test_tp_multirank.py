@@ -115,3 +115,25 @@ def test_tp_two_gloo_ranks_share_amax_and_sum_the_down_projection():
         assert p.returncode == 0, err[-3000:]
     seen = sorted(json.loads(l)["rank"] for out, _ in outs for l in out.splitlines() if l.strip())
     assert seen == [0, 1]
+
+
+def test_mlp_tensor_parallel_refuses_shares_that_split_a_block():
+    """Each rank's share of the hidden size must be a multiple of 16 (one
+    scale block of h must not straddle two ranks); refused before any call."""
+    import pytest
+    from nvfp4_block_scaled_21_b200 import tp
+
+    class W:
+        def __init__(self, rows):
+            self.rows = rows
+
+    class NoLib:
+        def __getattr__(self, name):
+            raise AssertionError(f"no library call expected, got {name}")
+
+    class X:
+        shape = (8, 64)
+        device = "cpu"
+
+    with pytest.raises(ValueError, match="multiple of 16"):
+        tp.mlp_tensor_parallel(X(), W(40), W(40), W(64), lib=NoLib())
